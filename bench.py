@@ -1,0 +1,531 @@
+#!/usr/bin/env python
+"""Benchmark of the Parallax forward pass (decode + causal prefill) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--sweep] [--compute-matched]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  * decode: one plx_decode call on a Qwen3-0.6B-shaped layer, B=64, context
+    4096 (equal seqlens), Hq=16, Hkv=8, d=128, bf16 KV cache;
+  * prefill: one plx_fwd call at the pretraining shape B=8, N=4096, Hq=16,
+    Hkv=8, d=128, causal, returning out and lse.
+`value` is the decode throughput in GB/s of algorithmic bytes (every cached
+key/value row read once, q/r/out once, lse), summed over all ranks; the
+prefill TFLOP/s and both kernels' roofline fractions ride along.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the same per-GPU
+workload on its own GPU with no collective on the data path (weak scaling);
+the timed region is bracketed by a barrier + synchronize on both sides and
+the max over ranks is taken.
+
+--impl reference times the fp64 CPU oracle (the only reference there is) on
+a bounded sample of the same decode workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode attn HBM GB/s & µs/step; prefill TFLOP/s; % of B200 roofline"
+
+DEC = dict(B=64, Hq=16, Hkv=8, S=4096, d=128)
+PRE = dict(B=8, Hq=16, Hkv=8, N=4096, d=128)
+L2_BYTES = 126 * 1024 * 1024
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ work counts
+def decode_bytes(B, Hq, Hkv, d, seqlens):
+    """Algorithmic bytes of one decode step: each cached K and V row of the
+    live context once (bf16), q, r and out once (bf16), lse (fp32)."""
+    kv = sum(int(s) for s in seqlens) * Hkv * 2 * d * 2
+    return kv + 3 * B * Hq * d * 2 + 4 * B * Hq
+
+
+def decode_flops(Hq, d, seqlens):
+    """8d per (query head, key): q.k, rho.k, p v, p s v (2d each)."""
+    return 8 * d * Hq * sum(int(s) for s in seqlens)
+
+
+def prefill_flops(B, Hq, N, d, causal=True):
+    """8d per unmasked (query, key) pair: QK^T, RK^T, PV, (P*S)V."""
+    pairs = N * (N + 1) // 2 if causal else N * N
+    return 8 * d * pairs * B * Hq
+
+
+def prefill_bytes(B, Hq, Hkv, N, d):
+    return (3 * B * Hq + 2 * B * Hkv) * N * d * 2 + 4 * B * Hq * N
+
+
+# ------------------------------------------------------------------ environment
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "parameterized_local_linear_plx_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (profiles/ncu_traffic.json); else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    e = t.get(kernel_key)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x, world, device=None):
+    """Max of a float over all ranks (used only outside the timed region)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world, device=None):
+    if world == 1:
+        return
+    import torch.distributed as dist
+    if device is not None and device.type == "cuda":
+        dist.barrier(device_ids=[device.index])
+    else:
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_decode_sample(q, r, kc, vc, sl, budget_s=10.0, max_entries=None):
+    """Run the oracle's effective-weight decode on batch entries one at a time
+    until ~budget_s of CPU time is used.  Returns (entries, seconds, bytes)."""
+    import oracle
+    B, Hq, d = q.shape
+    Hkv = kc.shape[1]
+    done, t0, nbytes = 0, time.perf_counter(), 0
+    limit = max_entries or B
+    while done < limit:
+        b = done
+        oracle.decode_effective(q[b:b + 1], r[b:b + 1], kc[b:b + 1], vc[b:b + 1], sl[b:b + 1])
+        nbytes += decode_bytes(1, Hq, Hkv, d, sl[b:b + 1].tolist())
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return done, time.perf_counter() - t0, nbytes
+
+
+def run_reference(args, world, rank):
+    """--impl reference: the fp64 CPU oracle on a bounded sample per step."""
+    if rank != 0:
+        return 0
+    import torch
+    from parameterized_local_linear_plx_b200 import inputs
+    q, kc, vc, r, sl = inputs.decode_inputs(4, DEC["Hq"], DEC["Hkv"], DEC["S"], DEC["d"], seed=0)
+    per_step = 2  # batch entries of the B=64 decode step per timed step
+    for _ in range(args.warmup):
+        oracle_decode_sample(q, r, kc, vc, sl, budget_s=1e9, max_entries=1)
+    times, nbytes = [], 0
+    for _ in range(args.steps):
+        n, t, b = oracle_decode_sample(q, r, kc, vc, sl, budget_s=1e9, max_entries=per_step)
+        times.append(t)
+        nbytes += b
+    total = sum(times)
+    value = nbytes / total / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": "decode: Qwen3-0.6B-shaped layer B=64 ctx=4096 Hq=16 Hkv=8 d=128 bf16 KV cache, "
+                               "equal seqlens (oracle: 2 of the 64 batch entries per step)"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"{per_step} batch entries x {DEC['Hq']} heads x {DEC['S']} keys per step, "
+                                   "effective-weight fp64 form"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+    from parameterized_local_linear_plx_b200 import build, inputs
+    if rank == 0:
+        build.build()
+    if world > 1:
+        barrier(world)  # wait for rank 0's build (CPU barrier before CUDA init)
+    from parameterized_local_linear_plx_b200 import plx
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- inputs, resident in HBM (generated on the device, seeded per rank)
+    q, kc, vc, r, sl = inputs.decode_inputs(DEC["B"], DEC["Hq"], DEC["Hkv"], DEC["S"], DEC["d"],
+                                            seed=rank, device=dev)
+    seqlens = [DEC["S"]] * DEC["B"]
+    ws_bytes = plx.plx_decode_workspace_size(DEC["B"], DEC["Hq"], DEC["Hkv"], DEC["S"], DEC["d"], 0)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    dout = torch.empty_like(q)
+    dlse = torch.empty(DEC["B"], DEC["Hq"], dtype=torch.float32, device=dev)
+    pq, pk, pv, pr = inputs.prefill_inputs(PRE["B"], PRE["Hq"], PRE["Hkv"], PRE["N"], PRE["d"], seed=100 + rank,
+                                           device=dev)
+    pout = torch.empty_like(pq)
+    plse = torch.empty(PRE["B"], PRE["Hq"], PRE["N"], dtype=torch.float32, device=dev)
+    n_splits = plx.plx_decode_num_splits(DEC["B"], DEC["Hq"], DEC["Hkv"], DEC["S"], DEC["d"])
+    launches_per_step = (2 if n_splits > 1 else 1) + 1
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        plx.plx_decode(q, kc, vc, sl, r, out=dout, lse=dlse, workspace=ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        plx.plx_fwd(pq, pk, pv, pr, causal=True, out=pout, lse=plse, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = plx.plx_check_device_status(stream)
+    if st != plx.PLX_OK:
+        raise RuntimeError(f"device status after warm-up: {plx.plx_status_string(st)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    total_ms = t_start.elapsed_time(t_end)
+    dec_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    pre_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    st = plx.plx_check_device_status(stream)
+    if st != plx.PLX_OK:
+        raise RuntimeError(f"device status after timing: {plx.plx_status_string(st)}")
+
+    total_ms_max = max_over_ranks(total_ms, world, dev)
+    dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), world, dev)
+    pre_avg = max_over_ranks(sum(pre_ms) / len(pre_ms), world, dev)
+
+    d_bytes = decode_bytes(DEC["B"], DEC["Hq"], DEC["Hkv"], DEC["d"], seqlens)
+    d_flops = decode_flops(DEC["Hq"], DEC["d"], seqlens)
+    p_flops = prefill_flops(PRE["B"], PRE["Hq"], PRE["N"], PRE["d"], True)
+    # whole-job decode throughput: bytes of all ranks over the slowest rank's decode time
+    value = world * d_bytes / (dec_avg * 1e-3) / 1e9
+    prefill_tflops = world * p_flops / (pre_avg * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    long_region = total_ms > 1000.0
+    tf_key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+    tf_peak = float(peaks.get(tf_key, FALLBACK_PEAKS[tf_key]))
+    dec_achieved = d_bytes / (dec_avg * 1e-3) / 1e9
+    pre_achieved = p_flops / (pre_avg * 1e-3) / 1e12
+    roof_dec = {"bound": "hbm", "achieved": dec_achieved, "peak": hbm, "unit": "GB/s",
+                "frac": dec_achieved / hbm, "traffic": load_traffic("decode"),
+                "kernel": "plx_decode (split + combine), per call",
+                "peak_source": f"{peak_src} hbm_gbs"}
+    roof_pre = {"bound": "tensor", "achieved": pre_achieved, "peak": tf_peak, "unit": "TFLOP/s",
+                "frac": pre_achieved / tf_peak, "traffic": load_traffic("prefill"),
+                "kernel": "plx_fwd_kernel<128,true>", "peak_source": f"{peak_src} {tf_key}"}
+
+    # ---- end to end through the public API: pinned host buffers, copies timed
+    e2e = run_e2e(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes)
+
+    # ---- CPU baseline: the oracle on this host, rank 0, N=1 only
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        qh, kh, vh, rh, slh = (t[:8].cpu() for t in (q, kc, vc, r, sl))
+        n, secs, nb = oracle_decode_sample(qh, rh, kh, vh, slh, budget_s=10.0)
+        cpu = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{n} of {DEC['B']} batch entries of the decode step (all {DEC['Hq']} heads, "
+                         f"{DEC['S']} keys), effective-weight fp64 form, {secs:.1f} s"}
+
+    clocks = clk.summary()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": "decode: Qwen3-0.6B-shaped layer B=64 ctx=4096 (equal seqlens) Hq=16 Hkv=8 d=128 "
+                            "bf16 KV cache; prefill: B=8 N=4096 Hq=16 Hkv=8 d=128 causal bf16, out+lse",
+                "decode_splits": n_splits,
+                "l2": "inputs larger than L2 (decode KV 1.07 GB, prefill 0.54 GB per step)",
+                "parallelism": f"replicas x{world}, no collective on the data path",
+            },
+            "decode": {"gbs": value, "us_per_step": dec_avg * 1e3, "bytes_per_step": d_bytes,
+                       "tflops": world * d_flops / (dec_avg * 1e-3) / 1e12},
+            "prefill": {"tflops": prefill_tflops, "ms_per_step": pre_avg, "flops_per_step": p_flops,
+                        "gbs_io": world * prefill_bytes(**PRE) / (pre_avg * 1e-3) / 1e9,
+                        "roofline": roof_pre},
+            "roofline": roof_dec,
+            "roofline_prefill": roof_pre,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_e2e(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes):
+    """Decode measured through plx_decode with the step's inputs (q, r,
+    seqlens) copied from pinned host memory and its result (out, lse) read
+    back, all inside the timed region.  The KV cache is the engine's resident
+    state and is not re-sent each step."""
+    import torch
+    hq = q.cpu().pin_memory()
+    hr = r.cpu().pin_memory()
+    hsl = sl.cpu().pin_memory()
+    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    hlse = torch.empty(q.shape[:2], dtype=torch.float32).pin_memory()
+    dq, dr, dsl = torch.empty_like(q), torch.empty_like(r), torch.empty_like(sl)
+    h2d = hq.numel() * 2 + hr.numel() * 2 + hsl.numel() * 4
+    d2h = hout.numel() * 2 + hlse.numel() * 4
+
+    def one():
+        dq.copy_(hq, non_blocking=True)
+        dr.copy_(hr, non_blocking=True)
+        dsl.copy_(hsl, non_blocking=True)
+        o, l = plx.plx_decode(dq, kc, vc, dsl, dr, stream=stream)
+        hout.copy_(o, non_blocking=True)
+        hlse.copy_(l, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        one()
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        one()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    return {"value": world * d_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "us_per_step": ms * 1e3}
+
+
+# ------------------------------------------------------------------ extra reports
+def run_sweep(args):
+    """Decode sweep: B x context with ragged seqlens in [ctx/2, ctx]; one JSON line per point."""
+    import torch
+    from parameterized_local_linear_plx_b200 import build, inputs
+    build.build()
+    from parameterized_local_linear_plx_b200 import plx
+    dev = torch.device("cuda", 0)
+    for B in (1, 8, 64, 256, 1024, 2048):
+        for ctx in (128, 1024, 4096, 16384, 32768):
+            alloc = B * ctx * 8 * 2 * 128 * 2
+            if alloc > 150e9:
+                print(json.dumps({"sweep": [B, ctx], "skipped": "KV cache above 150 GB"}), flush=True)
+                continue
+            q, kc, vc, r, sl = inputs.decode_inputs(B, 16, 8, ctx, 128, seed=0, seqlens="ragged", device=dev)
+            ws = torch.empty(max(16, plx.plx_decode_workspace_size(B, 16, 8, ctx, 128, 0)), dtype=torch.uint8,
+                             device=dev)
+            out = torch.empty_like(q)
+            lse = torch.empty(B, 16, dtype=torch.float32, device=dev)
+            flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if alloc < 4 * L2_BYTES else None
+            for _ in range(5):
+                plx.plx_decode(q, kc, vc, sl, r, out=out, lse=lse, workspace=ws)
+            ts = []
+            for _ in range(20):
+                if flush is not None:
+                    flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                plx.plx_decode(q, kc, vc, sl, r, out=out, lse=lse, workspace=ws)
+                b.record()
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            ms = statistics.median(ts)
+            nb = decode_bytes(B, 16, 8, 128, sl.tolist())
+            print(json.dumps({"sweep": [B, ctx], "us": ms * 1e3, "gbs": nb / (ms * 1e-3) / 1e9, "bytes": nb,
+                              "splits": plx.plx_decode_num_splits(B, 16, 8, ctx, 128)}), flush=True)
+            del q, kc, vc, r, sl, ws, out, lse, flush
+            torch.cuda.empty_cache()
+
+
+def run_compute_matched(args):
+    """Parallax at d=64 vs the library's softmax-only path (r = NULL) at d=128,
+    B=128, context 32768, Hq=16, Hkv=8."""
+    import torch
+    from parameterized_local_linear_plx_b200 import build, inputs
+    build.build()
+    from parameterized_local_linear_plx_b200 import plx
+    dev = torch.device("cuda", 0)
+    res = {}
+    for name, d, use_r in (("parallax_d64", 64, True), ("softmax_d128", 128, False)):
+        q, kc, vc, r, sl = inputs.decode_inputs(128, 16, 8, 32768, d, seed=0, device=dev)
+        for _ in range(5):
+            plx.plx_decode(q, kc, vc, sl, r if use_r else None)
+        ts = []
+        for _ in range(20):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            plx.plx_decode(q, kc, vc, sl, r if use_r else None)
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = statistics.median(ts)
+        nb = decode_bytes(128, 16, 8, d, sl.tolist())
+        res[name] = {"us": ms * 1e3, "gbs": nb / (ms * 1e-3) / 1e9, "gflop": decode_flops(16, d, sl.tolist()) / 1e9
+                     * (1 if use_r else 0.5)}
+        del q, kc, vc, r, sl
+        torch.cuda.empty_cache()
+    res["speedup_parallax_d64_over_softmax_d128"] = res["softmax_d128"]["us"] / res["parallax_d64"]["us"]
+    print(json.dumps({"compute_matched": res}), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["plx", "reference"], default="plx")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="decode sweep lines instead of the bench line")
+    ap.add_argument("--compute-matched", action="store_true", help="compute-matched decode comparison")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    if args.gpus != world and world > 1:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    if args.sweep:
+        return run_sweep(args)
+    if args.compute_matched:
+        return run_compute_matched(args)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        return run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

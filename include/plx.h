@@ -1,0 +1,158 @@
+/*
+ * plx.h -- C ABI of libplx.so: the Parallax attention forward pass on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation.  For each query i (per batch entry b and query head h):
+ *
+ *     w_ij   = softmax_j(scale * q_i . k_j)            over the key set J_i
+ *     o_SA_i = sum_j w_ij v_j
+ *     Sigma_i = sum_j w_ij (v_j - o_SA_i)(k_j - k_bar_i)^T,  k_bar_i = sum_j w_ij k_j
+ *     out_i  = o_SA_i - Sigma_i rho_i
+ *     lse_i  = ln sum_j exp(scale * q_i . k_j)
+ *
+ * This is the output equation of gist.science, "Technical overview:
+ * Parallax - parameterized local linear attention for language modeling",
+ * section "Method: Parallax / Core mechanism", with the boundary
+ * amplification factor eta set to zero as the same section states; the
+ * softmax-weighted, un-Bessel-corrected covariance and the unscaled probe
+ * score s_ij = rho_i . k_j are the plain readings of that equation.  The
+ * kernels compute it in the streamed form of news.chathome.org, "Parallax:
+ * a parameterized local linear attention ...", section "Hardware argument":
+ * two score branches (q.k and rho.k) that share one online max, one
+ * rescale factor and the same K/V tiles, accumulating l = sum p,
+ * c = sum p s, O1 = sum p v and O2 = sum p s v and emitting
+ * out = O1/l - (O2/l - (c/l)(O1/l)).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, row-major, bf16 (IEEE bfloat16 stored as uint16)
+ *     unless stated; every pointer is a DEVICE pointer, 16-byte aligned.
+ *   - GQA: query head h reads key/value head h / (Hq / Hkv); Hq % Hkv == 0.
+ *     rho (argument r) is given per query head.
+ *   - Head dimension d (= d_k = d_v) is 64 or 128.
+ *   - scale multiplies q.k only; pass 1/sqrt(d) for the usual choice.
+ *   - r == NULL means rho = 0, which is exactly softmax attention (the same
+ *     page, section "How the mechanism works": probe norm zero reduces to
+ *     softmax); the kernels then skip the rho branch.
+ *   - lse may be NULL (not written).
+ *   - The caller owns every buffer.  The library allocates no device or
+ *     host memory; it keeps one device word that records a bounded-wait
+ *     timeout (see plx_check_device_status).
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it.  Argument errors are returned synchronously
+ *     before anything is launched; launch failures return PLX_ERR_CUDA.
+ *   - Return value: a plx_status (0 = PLX_OK, negative = error).
+ */
+#ifndef PLX_H_
+#define PLX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum plx_status {
+  PLX_OK = 0,
+  PLX_ERR_NULL = -1,            /* a required pointer is NULL */
+  PLX_ERR_SHAPE = -2,           /* a size is out of range (B, H, N, S_max < 1, ...) */
+  PLX_ERR_HEADDIM = -3,         /* d not in {64, 128} */
+  PLX_ERR_GQA = -4,             /* Hq % Hkv != 0 */
+  PLX_ERR_ALIGN = -5,           /* a pointer is not 16-byte aligned */
+  PLX_ERR_WORKSPACE = -6,       /* workspace NULL or smaller than required */
+  PLX_ERR_CUDA = -7,            /* a CUDA runtime/driver call failed */
+  PLX_ERR_DEVICE_TIMEOUT = -8,  /* a kernel gave up a bounded wait (device word set) */
+  PLX_ERR_ARCH = -9             /* current device is not sm_100 */
+} plx_status;
+
+/* Library version, major*10000 + minor*100 + patch. */
+int plx_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* plx_status_string(int status);
+
+/*
+ * plx_fwd -- prefill / full-sequence forward.
+ *
+ *   q   [B, Hq,  N, d] bf16   queries
+ *   k   [B, Hkv, N, d] bf16   keys
+ *   v   [B, Hkv, N, d] bf16   values
+ *   r   [B, Hq,  N, d] bf16   probes rho (NULL: rho = 0)
+ *   out [B, Hq,  N, d] bf16   output (written)
+ *   lse [B, Hq,  N]    fp32   natural-log LSE of the scaled q.k scores (NULL: skipped)
+ *   causal != 0: J_i = {j <= i} (diagonal included); causal == 0: all j < N.
+ *
+ * Requirements: B, Hq, Hkv, N >= 1; d in {64, 128}; Hq % Hkv == 0;
+ * all pointers 16-byte aligned; out must not alias an input.
+ * Runs one kernel (tcgen05 tensor cores, TMA-fed) on `stream`.
+ */
+int plx_fwd(const void* q, const void* k, const void* v, const void* r,
+            void* out, float* lse,
+            int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+            void* stream);
+
+/*
+ * plx_decode_num_splits -- the split count plx_decode uses when passed
+ * num_splits = 0 (a function of the shapes only; >= 1).
+ */
+int plx_decode_num_splits(int B, int Hq, int Hkv, int S_max, int d);
+
+/*
+ * plx_decode_workspace_size -- bytes of workspace plx_decode needs for these
+ * shapes and split count (0 = the automatic count).  0 when one split is used.
+ */
+size_t plx_decode_workspace_size(int B, int Hq, int Hkv, int S_max, int d, int num_splits);
+
+/*
+ * plx_decode -- one decode step against a KV cache, split over the keys.
+ *
+ *   q       [B, Hq, d]           bf16   one query per (b, h)
+ *   r       [B, Hq, d]           bf16   its probe rho (NULL: rho = 0)
+ *   kcache  [B, Hkv, S_max, d]   bf16   key cache
+ *   vcache  [B, Hkv, S_max, d]   bf16   value cache
+ *   seqlens [B]                  int32  DEVICE array; query (b, .) attends the
+ *                                       cached keys j < seqlens[b] (values above
+ *                                       S_max are clamped to S_max; <= 0 gives
+ *                                       out = 0 and lse = -inf)
+ *   out     [B, Hq, d]           bf16   output (written)
+ *   lse     [B, Hq]              fp32   (NULL: skipped)
+ *   num_splits: key chunks per (b, kv head); 0 = automatic.  With more than
+ *     one split the partial states (m, l, c, O1, O2) go to `workspace` and a
+ *     second kernel merges them; the result does not depend on the count
+ *     beyond rounding.
+ *   workspace / workspace_bytes: caller-owned device scratch of at least
+ *     plx_decode_workspace_size(...) bytes, 16-byte aligned (may be NULL when
+ *     that size is 0).  Its contents are overwritten.
+ *
+ * Requirements: B, Hq, Hkv, S_max >= 1; d in {64, 128}; Hq % Hkv == 0.
+ */
+int plx_decode(const void* q, const void* r, const void* kcache, const void* vcache,
+               const int32_t* seqlens, void* out, float* lse,
+               int B, int Hq, int Hkv, int S_max, int d, float scale, int num_splits,
+               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * plx_check_device_status -- synchronises `stream`, then reads and clears the
+ * library's device error word.  Every wait inside the kernels (on an
+ * mbarrier fed by TMA or by tensor-core completion) is bounded in time; a
+ * kernel that gives up sets the word, releases what it holds and returns.
+ * Returns PLX_OK, PLX_ERR_DEVICE_TIMEOUT (word was set; it is now clear) or
+ * PLX_ERR_CUDA.  After a timeout the outputs of calls made before this check
+ * are undefined.
+ */
+int plx_check_device_status(void* stream);
+
+/*
+ * plx_selftest_wait_timeout -- test hook for the bounded-wait path: launches
+ * one tiny kernel that waits on an mbarrier nothing ever completes, with a
+ * limit of `limit_cycles` SM clock cycles, so that the wait runs out and sets
+ * the device error word.  Follow with plx_check_device_status, which must
+ * return PLX_ERR_DEVICE_TIMEOUT.  Faults nothing; the context stays usable.
+ */
+int plx_selftest_wait_timeout(unsigned long long limit_cycles, void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* PLX_H_ */

@@ -1,0 +1,309 @@
+// plx.cu -- the C ABI of libplx.so (declared in include/plx.h): argument
+// validation, TMA descriptor set-up, split selection and kernel launches.
+// No device or host memory is allocated here; the caller owns every buffer.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/plx.h"
+#include "plx_decode.cuh"
+#include "plx_fwd.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kSmCount = 148;  // B200
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- device checks
+int g_arch_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 not sm_100
+std::mutex g_mu;
+
+int check_arch(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PLX_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PLX_ERR_CUDA;
+  *dev_out = dev;
+  if (g_arch_ok[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return PLX_ERR_CUDA;
+    g_arch_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return g_arch_ok[dev] == 1 ? PLX_OK : PLX_ERR_ARCH;
+}
+
+// ---------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return PLX_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return PLX_ERR_CUDA;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return PLX_OK;
+}
+
+// A bf16 tensor [planes, rows, D] (D contiguous) as a 3-D TMA map with a
+// box of {64 elements, box_rows, 1} and 128-byte swizzle.  Loads past `rows`
+// (inside a plane) are zero-filled, so ragged tails never read a neighbour.
+int make_map_3d(CUtensorMap* map, const void* base, int D, long long rows, long long planes,
+                int box_rows) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2u,
+                           static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(D) * 2u};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult rc = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS ? PLX_OK : PLX_ERR_CUDA;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+template <typename K>
+int ensure_smem(K kernel, int bytes, bool* done) {
+  if (*done) return PLX_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  *done = true;
+  return PLX_OK;
+}
+
+// ---------------------------------------------------------------- decode
+struct SplitPlan {
+  int splits, chunk;
+};
+
+SplitPlan plan_splits(int B, int Hq, int Hkv, int S_max, int num_splits) {
+  const int G = Hq / Hkv;
+  const int n_hg = (G + 7) / 8;
+  const long long units = static_cast<long long>(B) * Hkv * n_hg;
+  int splits = num_splits;
+  if (splits <= 0) {
+    const long long target = 4LL * 2 * kSmCount;  // about four waves of two CTAs per SM
+    long long s = (target + units - 1) / units;
+    const long long max_s = (S_max + 127) / 128;  // chunks of at least 128 keys
+    if (s > max_s) s = max_s;
+    if (s < 1) s = 1;
+    splits = static_cast<int>(s);
+  }
+  if (splits > S_max) splits = S_max;
+  int chunk = (S_max + splits - 1) / splits;
+  chunk = (chunk + plx::kDecTileKeys - 1) / plx::kDecTileKeys * plx::kDecTileKeys;
+  splits = (S_max + chunk - 1) / chunk;
+  return {splits, chunk};
+}
+
+size_t workspace_bytes_for(int B, int Hq, int d, int splits) {
+  if (splits <= 1) return 0;
+  return static_cast<size_t>(B) * Hq * splits * (2 * d + 4) * sizeof(float);
+}
+
+template <int D, bool HAS_R>
+int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const plx::DecodeParams& p, int n_hg,
+                  cudaStream_t st) {
+  using Cfg = plx::DecodeCfg<D>;
+  static bool done[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto kern = plx::plx_decode_split_kernel<D, HAS_R>;
+  if (ensure_smem(kern, Cfg::kSmemBytes, &done[dev]) != PLX_OK) return PLX_ERR_CUDA;
+  dim3 grid(p.splits, p.Hkv * n_hg, p.B);
+  kern<<<grid, plx::kDecThreads, Cfg::kSmemBytes, st>>>(km, vm, p);
+  if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+  if (p.splits > 1) {
+    plx::plx_decode_combine_kernel<D><<<p.B * p.Hq, D, 0, st>>>(p.ws, p.out, p.lse, p.splits);
+    if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+  }
+  return PLX_OK;
+}
+
+template <int D, bool HAS_R>
+int launch_fwd(const CUtensorMap& qm, const CUtensorMap& rm, const CUtensorMap& km, const CUtensorMap& vm,
+               const plx::FwdParams& p, unsigned grid, cudaStream_t st) {
+  using Cfg = plx::FwdCfg<D>;
+  static bool done[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto kern = plx::plx_fwd_kernel<D, HAS_R>;
+  if (ensure_smem(kern, Cfg::kSmemBytes, &done[dev]) != PLX_OK) return PLX_ERR_CUDA;
+  kern<<<grid, plx::kFwdThreads, Cfg::kSmemBytes, st>>>(qm, rm, km, vm, p);
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int plx_version(void) { return 100; }
+
+const char* plx_status_string(int status) {
+  switch (status) {
+    case PLX_OK: return "PLX_OK";
+    case PLX_ERR_NULL: return "PLX_ERR_NULL: a required pointer is NULL";
+    case PLX_ERR_SHAPE: return "PLX_ERR_SHAPE: a size is out of range";
+    case PLX_ERR_HEADDIM: return "PLX_ERR_HEADDIM: head dim must be 64 or 128";
+    case PLX_ERR_GQA: return "PLX_ERR_GQA: Hq must be a multiple of Hkv";
+    case PLX_ERR_ALIGN: return "PLX_ERR_ALIGN: pointers must be 16-byte aligned";
+    case PLX_ERR_WORKSPACE: return "PLX_ERR_WORKSPACE: workspace missing or too small";
+    case PLX_ERR_CUDA: return "PLX_ERR_CUDA: a CUDA call failed";
+    case PLX_ERR_DEVICE_TIMEOUT: return "PLX_ERR_DEVICE_TIMEOUT: a kernel gave up a bounded wait";
+    case PLX_ERR_ARCH: return "PLX_ERR_ARCH: the current device is not sm_100";
+    default: return "PLX: unknown status";
+  }
+}
+
+int plx_fwd(const void* q, const void* k, const void* v, const void* r, void* out, float* lse, int B,
+            int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  if (!q || !k || !v || !out) return PLX_ERR_NULL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return PLX_ERR_SHAPE;
+  if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
+  if (Hq % Hkv) return PLX_ERR_GQA;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (r && !aligned16(r)) || !aligned16(out) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return PLX_ERR_ALIGN;
+  const int G = Hq / Hkv;
+  const int pair_heads = (G % 2 == 0) ? 1 : 0;
+  const int n_pairs = pair_heads ? Hq / 2 : Hq;
+  const int n_qblocks = pair_heads ? (N + plx::kFwdBM - 1) / plx::kFwdBM : (N + 2 * plx::kFwdBM - 1) / (2 * plx::kFwdBM);
+  const long long grid = static_cast<long long>(B) * n_pairs * n_qblocks;
+  if (grid > 0x7fffffffLL) return PLX_ERR_SHAPE;
+  int dev = 0;
+  int rc = check_arch(&dev);
+  if (rc != PLX_OK) return rc;
+  if ((rc = get_encoder()) != PLX_OK) return rc;
+
+  CUtensorMap qm, rm, km, vm;
+  const long long pq = static_cast<long long>(B) * Hq, pkv = static_cast<long long>(B) * Hkv;
+  if (make_map_3d(&qm, q, d, N, pq, 16) != PLX_OK || make_map_3d(&km, k, d, N, pkv, plx::kFwdBN) != PLX_OK ||
+      make_map_3d(&vm, v, d, N, pkv, plx::kFwdBN) != PLX_OK)
+    return PLX_ERR_CUDA;
+  if (r) {
+    if (make_map_3d(&rm, r, d, N, pq, 16) != PLX_OK) return PLX_ERR_CUDA;
+  } else {
+    rm = qm;  // unused
+  }
+  plx::FwdParams p;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.G = G;
+  p.pair_heads = pair_heads; p.n_pairs = n_pairs; p.n_qblocks = n_qblocks;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * plx::kLog2e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned g = static_cast<unsigned>(grid);
+  if (d == 128) return r ? launch_fwd<128, true>(qm, rm, km, vm, p, g, st) : launch_fwd<128, false>(qm, rm, km, vm, p, g, st);
+  return r ? launch_fwd<64, true>(qm, rm, km, vm, p, g, st) : launch_fwd<64, false>(qm, rm, km, vm, p, g, st);
+}
+
+int plx_decode_num_splits(int B, int Hq, int Hkv, int S_max, int d) {
+  (void)d;
+  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv) return 1;
+  return plan_splits(B, Hq, Hkv, S_max, 0).splits;
+}
+
+size_t plx_decode_workspace_size(int B, int Hq, int Hkv, int S_max, int d, int num_splits) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128)) return 0;
+  return workspace_bytes_for(B, Hq, d, plan_splits(B, Hq, Hkv, S_max, num_splits).splits);
+}
+
+int plx_decode(const void* q, const void* r, const void* kcache, const void* vcache,
+               const int32_t* seqlens, void* out, float* lse, int B, int Hq, int Hkv, int S_max,
+               int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
+               void* stream) {
+  if (!q || !kcache || !vcache || !seqlens || !out) return PLX_ERR_NULL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || num_splits < 0) return PLX_ERR_SHAPE;
+  if (B > 65535) return PLX_ERR_SHAPE;
+  if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
+  if (Hq % Hkv) return PLX_ERR_GQA;
+  if (!aligned16(q) || (r && !aligned16(r)) || !aligned16(kcache) || !aligned16(vcache) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return PLX_ERR_ALIGN;
+  const SplitPlan plan = plan_splits(B, Hq, Hkv, S_max, num_splits);
+  const size_t need = workspace_bytes_for(B, Hq, d, plan.splits);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return PLX_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return PLX_ERR_ALIGN;
+  }
+  const int G = Hq / Hkv;
+  const int n_hg = (G + 7) / 8;
+  if (static_cast<long long>(Hkv) * n_hg > 65535) return PLX_ERR_SHAPE;
+  int dev = 0;
+  int rc = check_arch(&dev);
+  if (rc != PLX_OK) return rc;
+  if ((rc = get_encoder()) != PLX_OK) return rc;
+
+  CUtensorMap km, vm;
+  const long long planes = static_cast<long long>(B) * Hkv;
+  if (make_map_3d(&km, kcache, d, S_max, planes, plx::kDecTileKeys) != PLX_OK ||
+      make_map_3d(&vm, vcache, d, S_max, planes, plx::kDecTileKeys) != PLX_OK)
+    return PLX_ERR_CUDA;
+
+  plx::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.r = static_cast<const __nv_bfloat16*>(r);
+  p.seqlens = seqlens;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.ws = static_cast<float*>(workspace);
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.S_max = S_max; p.G = G; p.n_hgroups = n_hg;
+  p.splits = plan.splits; p.chunk = plan.chunk;
+  p.scale_log2 = scale * plx::kLog2e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 128) return r ? launch_decode<128, true>(km, vm, p, n_hg, st) : launch_decode<128, false>(km, vm, p, n_hg, st);
+  return r ? launch_decode<64, true>(km, vm, p, n_hg, st) : launch_decode<64, false>(km, vm, p, n_hg, st);
+}
+
+int plx_check_device_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PLX_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_plx_error, sizeof(word)) != cudaSuccess) return PLX_ERR_CUDA;
+  if (word == 0u) return PLX_OK;
+  const unsigned int zero = 0u;
+  if (cudaMemcpyToSymbol(g_plx_error, &zero, sizeof(zero)) != cudaSuccess) return PLX_ERR_CUDA;
+  return PLX_ERR_DEVICE_TIMEOUT;
+}
+
+}  // extern "C"
+
+namespace {
+// One mbarrier that expects one arrival which never comes: the wait runs out.
+__global__ void plx_selftest_wait_kernel(long long limit) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    plx::mbar_init(plx::smem_u32(&bar), 1);
+    plx::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = plx::mbar_wait(plx::smem_u32(&bar), 0, plx::kErrSelftest, limit);
+    if (ok) plx::set_error(0xDEADu);  // cannot happen: nothing arrives
+  }
+}
+}  // namespace
+
+extern "C" int plx_selftest_wait_timeout(unsigned long long limit_cycles, void* stream) {
+  int dev = 0;
+  int rc = check_arch(&dev);
+  if (rc != PLX_OK) return rc;
+  if (limit_cycles > (1ULL << 32)) return PLX_ERR_SHAPE;  // keep the test short (~2 s max)
+  plx_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<long long>(limit_cycles));
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}

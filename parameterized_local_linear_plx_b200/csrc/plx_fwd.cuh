@@ -1,0 +1,433 @@
+// plx_fwd.cuh -- Parallax prefill / full-sequence forward on sm_100a.
+//
+// Method (gist.science, "Technical overview: Parallax - parameterized local
+// linear attention for language modeling", section "Method: Parallax / Core
+// mechanism"): out_i = o_SA_i - Sigma_i rho_i.  Streamed as in
+// news.chathome.org, "Parallax: a parameterized local linear attention ...",
+// section "Hardware argument": two score branches share the online max, the
+// rescale factor and the K/V tiles.
+//
+// Design (one CTA per pair of 64-query tiles, 320 threads):
+//   * A query tile and its probes form ONE stacked MMA operand [Q;R] of 128
+//     rows, interleaved in blocks of 16: rows 32w..32w+15 hold queries
+//     16w..16w+15 and rows 32w+16..32w+31 hold their probes.  One tcgen05 MMA
+//     (M=128, N=128 keys, K=d) gives both branches, a = q.k in TMEM lanes
+//     32w+r and s = rho.k in lanes 32w+16+r.  A 16x256b tensor-memory load
+//     at lane 32w and another at 32w+16 hand every thread a and s for the
+//     SAME (query, key) pairs, so the shared softmax needs no data exchange.
+//   * The value product uses the same stacking: P (bf16) is written over the
+//     a rows and P*S over the s rows of the score columns in TMEM, and one
+//     MMA [P ; P*S] x V (A from tensor memory) accumulates O1 = sum p v and
+//     O2 = sum p s v in the matching rows of one 128-lane accumulator.
+//   * Two query tiles share every K/V tile: heads (h, h+1) of one KV group at
+//     the same rows when the group size is even, otherwise rows (q0, q0+64)
+//     of one head.  Tensor memory: [S0 | O0 | S1 | O1], 128 columns each.
+//   * Warps 0-3 and 4-7: softmax + epilogue of tile 0 and tile 1;
+//     warp 8: TMA loads (Q/R once, K/V ring); warp 9: TMEM allocation and
+//     the single thread that issues every MMA.  The MMA order
+//     PV0(j), S0(j+1), PV1(j), S1(j+1) lets each softmax overlap the other
+//     tile's MMAs.
+//   * The running max is updated lazily: O is rescaled in tensor memory only
+//     when a row max grows by more than 2^8 (so p <= 256 before the final
+//     normalisation, which bf16 P holds without loss of relative precision).
+#pragma once
+
+#include "plx_ptx.cuh"
+#include "plx_tcgen05.cuh"
+
+namespace plx {
+
+constexpr int kFwdBM = 64;        // queries per tile (128 stacked rows with their probes)
+constexpr int kFwdBN = 128;       // keys per K/V tile
+constexpr int kFwdThreads = 320;  // 8 softmax warps + TMA warp + MMA warp
+constexpr int kFwdTmaWarp = 8;
+constexpr int kFwdMmaWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kCB = D / 64;                 // 128-byte column blocks per row
+  static constexpr int kBlock = 128 * 128;           // bytes of one [128 rows x 128 B] block
+  static constexpr int kQRBytes = kCB * kBlock;      // stacked [Q;R] tile
+  static constexpr int kKVBytes = kCB * kBlock;      // one K or V tile (128 keys)
+  static constexpr int kStages = D == 128 ? 2 : 3;
+  static constexpr int kOffQR = 0;
+  static constexpr int kOffK = 2 * kQRBytes;
+  static constexpr int kOffV = kOffK + kStages * kKVBytes;
+  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+struct FwdParams {
+  __nv_bfloat16* out;  // [B, Hq, N, D]
+  float* lse;          // [B, Hq, N] or nullptr
+  int B, Hq, Hkv, N, G;
+  int pair_heads;      // 1: tiles are heads (2p, 2p+1) at rows 64*qb; 0: rows 128*qb (+64) of head p
+  int n_pairs;         // Hq / 2 or Hq
+  int n_qblocks;       // ceil(N/64) or ceil(N/128)
+  int causal;
+  float scale_log2;    // scale * log2(e)
+};
+
+template <int D, bool HAS_R>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap rmap,
+               const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+               const FwdParams p) {
+  using Cfg = FwdCfg<D>;
+  constexpr int NS = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* qr_full = bars;             // [2]
+  uint64_t* k_full = bars + 2;          // [NS]
+  uint64_t* k_empty = k_full + NS;      // [NS]
+  uint64_t* v_full = k_empty + NS;      // [NS]
+  uint64_t* v_empty = v_full + NS;      // [NS]
+  uint64_t* s_full = v_empty + NS;      // [2]
+  uint64_t* p_ready = s_full + 2;       // [2]
+  uint64_t* o_done = p_ready + 2;       // [2]
+  uint64_t* fin = o_done + 2;           // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: longest causal rows first
+  const int per = p.B * p.n_pairs;
+  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) / per;
+  const int rem = static_cast<int>(blockIdx.x) % per;
+  const int b = rem / p.n_pairs;
+  const int hp = rem % p.n_pairs;
+  // tile t in {0, 1}: query head head_of(t), first query row row0_of(t)
+  auto head_of = [&](int t) { return p.pair_heads ? 2 * hp + t : hp; };
+  auto row0_of = [&](int t) { return p.pair_heads ? qb * kFwdBM : (2 * qb + t) * kFwdBM; };
+  const int g = head_of(0) / p.G;
+  const int qmax = min(p.N - 1, row0_of(1) + kFwdBM - 1);
+  const int nkv_all = (p.N + kFwdBN - 1) / kFwdBN;
+  const int nkv = p.causal ? min(nkv_all, qmax / kFwdBN + 1) : nkv_all;
+
+  if (threadIdx.x == 0) {
+    // every barrier takes one arrival (+ TMA bytes / tcgen05.commit), except
+    // p_ready, which all 128 threads of a softmax warpgroup arrive on
+    for (int i = 0; i < 2 + 4 * NS + 7; ++i) {
+      uint64_t* bp = &bars[i];
+      mbar_init(smem_u32(bp), (bp == &p_ready[0] || bp == &p_ready[1]) ? 128u : 1u);
+    }
+    fence_barrier_init();
+  }
+  if (!HAS_R) {
+    // rho = 0: zero the probe rows of both stacked tiles once (TMA loads only Q).
+    uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < 2 * Cfg::kCB * 4 * 16 * 8; i += kFwdThreads) {
+      const int c16 = i & 7, row = (i >> 3) & 15, w = (i >> 7) & 3, cb = (i >> 9) % Cfg::kCB,
+                t = (i >> 9) / Cfg::kCB;
+      uint8_t* dst = smem + Cfg::kOffQR + t * Cfg::kQRBytes + cb * Cfg::kBlock + (32 * w + 16 + row) * 128 + c16 * 16;
+      *reinterpret_cast<uint4*>(dst) = z;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == kFwdMmaWarp) {
+    tc::tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  // tensor-memory columns: [S0 | O0 | S1 | O1]
+  auto col_s = [](int t) { return static_cast<uint32_t>(256 * t); };
+  auto col_o = [](int t) { return static_cast<uint32_t>(256 * t + 128); };
+  bool ok = true;
+
+  if (warp == kFwdTmaWarp) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&qmap);
+      if (HAS_R) tma_prefetch_desc(&rmap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      for (int t = 0; t < 2; ++t) {
+        const uint32_t fb = smem_u32(&qr_full[t]);
+        mbar_arrive_expect_tx(fb, HAS_R ? Cfg::kQRBytes : Cfg::kQRBytes / 2);
+        const uint32_t base = smem_u32(smem + Cfg::kOffQR + t * Cfg::kQRBytes);
+        const int plane = b * p.Hq + head_of(t);
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+          for (int cb = 0; cb < Cfg::kCB; ++cb) {
+            const uint32_t dst = base + cb * Cfg::kBlock + (32 * w) * 128;
+            tma_load_3d(&qmap, dst, fb, cb * 64, row0_of(t) + 16 * w, plane);
+            if (HAS_R) tma_load_3d(&rmap, dst + 16 * 128, fb, cb * 64, row0_of(t) + 16 * w, plane);
+          }
+      }
+      const int plane_kv = b * p.Hkv + g;
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(smem_u32(&k_empty[s]), ((j / NS) - 1) & 1, kErrFwdLoad)) { ok = false; break; }
+        {
+          const uint32_t fb = smem_u32(&k_full[s]);
+          mbar_arrive_expect_tx(fb, Cfg::kKVBytes);
+          const uint32_t dst = smem_u32(smem + Cfg::kOffK + s * Cfg::kKVBytes);
+#pragma unroll
+          for (int cb = 0; cb < Cfg::kCB; ++cb)
+            tma_load_3d(&kmap, dst + cb * Cfg::kBlock, fb, cb * 64, j * kFwdBN, plane_kv);
+          issued_k = j + 1;
+        }
+        if (j >= NS && !mbar_wait(smem_u32(&v_empty[s]), ((j / NS) - 1) & 1, kErrFwdLoad)) { ok = false; break; }
+        {
+          const uint32_t fb = smem_u32(&v_full[s]);
+          mbar_arrive_expect_tx(fb, Cfg::kKVBytes);
+          const uint32_t dst = smem_u32(smem + Cfg::kOffV + s * Cfg::kKVBytes);
+#pragma unroll
+          for (int cb = 0; cb < Cfg::kCB; ++cb)
+            tma_load_3d(&vmap, dst + cb * Cfg::kBlock, fb, cb * 64, j * kFwdBN, plane_kv);
+          issued_v = j + 1;
+        }
+      }
+      if (!ok) {  // let every issued load land before the CTA can exit
+        for (int t = 0; t < 2; ++t) mbar_wait(smem_u32(&qr_full[t]), 0, kErrFwdDrain);
+        for (int j = max(0, issued_k - NS); j < issued_k; ++j)
+          mbar_wait(smem_u32(&k_full[j % NS]), (j / NS) & 1, kErrFwdDrain);
+        for (int j = max(0, issued_v - NS); j < issued_v; ++j)
+          mbar_wait(smem_u32(&v_full[j % NS]), (j / NS) & 1, kErrFwdDrain);
+      }
+    }
+  } else if (warp == kFwdMmaWarp) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kFwdBN, 0, 0);  // [Q;R] x K^T, both K-major
+      constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, 0, 1);       // [P;PS] x V, V MN-major
+      const uint32_t qr_base = smem_u32(smem + Cfg::kOffQR);
+      const uint32_t k_base = smem_u32(smem + Cfg::kOffK);
+      const uint32_t v_base = smem_u32(smem + Cfg::kOffV);
+
+      auto issue_s = [&](int t, int j) {
+        const uint32_t a0 = qr_base + t * Cfg::kQRBytes;
+        const uint32_t b0 = k_base + (j % NS) * Cfg::kKVBytes;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * Cfg::kBlock + (ks & 3) * 32;
+          tc::mma_ss(tmem + col_s(t), tc::smem_desc_sw128(a0 + off, 16, 1024),
+                     tc::smem_desc_sw128(b0 + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+        }
+        tc::commit(smem_u32(&s_full[t]));
+      };
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t b0 = v_base + (j % NS) * Cfg::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < kFwdBN / 16; ++kk)
+          tc::mma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
+                     tc::smem_desc_sw128(b0 + kk * 2048, Cfg::kBlock, 1024), idesc_o,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+      };
+
+      ok = mbar_wait(smem_u32(&qr_full[0]), 0, kErrFwdMma) && mbar_wait(smem_u32(&qr_full[1]), 0, kErrFwdMma) &&
+           mbar_wait(smem_u32(&k_full[0]), 0, kErrFwdMma);
+      if (ok) {
+        tc::fence_after_sync();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        tc::commit(smem_u32(&k_empty[0]));
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int s = j % NS;
+        if (!mbar_wait(smem_u32(&v_full[s]), (j / NS) & 1, kErrFwdMma) ||
+            !mbar_wait(smem_u32(&p_ready[0]), j & 1, kErrFwdMma)) { ok = false; break; }
+        tc::fence_after_sync();
+        issue_pv(0, j);
+        const bool more = j + 1 < nkv;
+        if (more) {
+          if (!mbar_wait(smem_u32(&k_full[(j + 1) % NS]), ((j + 1) / NS) & 1, kErrFwdMma)) { ok = false; break; }
+          tc::fence_after_sync();
+          issue_s(0, j + 1);
+        }
+        if (!mbar_wait(smem_u32(&p_ready[1]), j & 1, kErrFwdMma)) { ok = false; break; }
+        tc::fence_after_sync();
+        issue_pv(1, j);
+        tc::commit(smem_u32(&v_empty[s]));
+        if (more) {
+          issue_s(1, j + 1);
+          tc::commit(smem_u32(&k_empty[(j + 1) % NS]));
+        } else {
+          tc::commit(smem_u32(&o_done[0]));
+          tc::commit(smem_u32(&o_done[1]));
+        }
+      }
+      // Every MMA issued must be complete before tensor memory is released.
+      tc::commit(smem_u32(&fin[0]));
+      mbar_wait(smem_u32(&fin[0]), 0, kErrFwdMma);
+    }
+  } else {
+    // ================================================================ softmax + epilogue
+    const int t = warp >> 2;     // query tile
+    const int wq = warp & 3;     // TMEM lane quadrant
+    const int c4 = lane & 3;
+    const uint32_t lane_a = static_cast<uint32_t>(32 * wq) << 16;
+    const uint32_t lane_s = static_cast<uint32_t>(32 * wq + 16) << 16;
+    const uint32_t ta = tmem + lane_a + col_s(t);
+    const uint32_t ts = tmem + lane_s + col_s(t);
+    const uint32_t to1 = tmem + lane_a + col_o(t);
+    const uint32_t to2 = tmem + lane_s + col_o(t);
+    const int q0 = row0_of(t);
+    const int q_lo = q0 + 16 * wq + (lane >> 2);
+    const int q_hi = q_lo + 8;
+    float m_lo = -INFINITY, m_hi = -INFINITY;
+    float l_lo = 0.f, l_hi = 0.f, c_lo = 0.f, c_hi = 0.f;  // this thread's column share
+
+    for (int j = 0; j < nkv; ++j) {
+      // warp-uniform: the .sync.aligned tensor-memory accesses below need every lane
+      const bool landed = mbar_wait(smem_u32(&s_full[t]), j & 1, kErrFwdSoftmax);
+      if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
+      tc::fence_after_sync();
+      uint32_t ra[64], rs[64];
+      tc::ld_16x256b_x8(ta, *reinterpret_cast<uint32_t(*)[32]>(&ra[0]));
+      tc::ld_16x256b_x8(ta + 64, *reinterpret_cast<uint32_t(*)[32]>(&ra[32]));
+      if (HAS_R) {
+        tc::ld_16x256b_x8(ts, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
+        tc::ld_16x256b_x8(ts + 64, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
+      }
+      tc::wait_ld();
+
+      // register i: half h = i/32, rep g = (i%32)/4, e = i%4;
+      // key = 64h + 8g + 2*c4 + (e&1); row lo for e < 2, row hi for e >= 2.
+      float x[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(ra[i]) * p.scale_log2;
+      const int kbase = j * kFwdBN;
+      const bool need_mask = (p.causal && kbase + kFwdBN - 1 > q0) || (kbase + kFwdBN > p.N);
+      if (need_mask) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int key = kbase + 64 * (i >> 5) + 8 * ((i & 31) >> 2) + 2 * c4 + (i & 1);
+          const int q = (i & 2) ? q_hi : q_lo;
+          const bool valid = key < p.N && (!p.causal || key <= q);
+          x[i] = valid ? x[i] : -INFINITY;
+        }
+      }
+      float mx_lo = -INFINITY, mx_hi = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; i += 4) {
+        mx_lo = fmaxf(mx_lo, fmaxf(x[i], x[i + 1]));
+        mx_hi = fmaxf(mx_hi, fmaxf(x[i + 2], x[i + 3]));
+      }
+      mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
+      mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
+      mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
+      mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
+      const bool grow = mx_lo > m_lo + kRescaleThreshold || mx_hi > m_hi + kRescaleThreshold;
+      if (__any_sync(0xffffffffu, grow)) {
+        const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
+        const float al_lo = mn_lo == -INFINITY ? 1.f : ex2(m_lo - mn_lo);
+        const float al_hi = mn_hi == -INFINITY ? 1.f : ex2(m_hi - mn_hi);
+        l_lo *= al_lo; c_lo *= al_lo; l_hi *= al_hi; c_hi *= al_hi;
+        m_lo = mn_lo; m_hi = mn_hi;
+        if (j > 0) {
+          // O rows of this warp: O1 at the a lanes, O2 at the s lanes; PV(j-1)
+          // has completed (it precedes S(j) in the MMA stream).
+#pragma unroll 1
+          for (int ch = 0; ch < D / 16; ++ch) {
+            uint32_t o1[8], o2[8];
+            tc::ld_16x256b_x2(to1 + 16 * ch, o1);
+            tc::ld_16x256b_x2(to2 + 16 * ch, o2);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float al = (i & 2) ? al_hi : al_lo;
+              o1[i] = __float_as_uint(__uint_as_float(o1[i]) * al);
+              o2[i] = __float_as_uint(__uint_as_float(o2[i]) * al);
+            }
+            tc::st_16x256b_x2(to1 + 16 * ch, o1);
+            tc::st_16x256b_x2(to2 + 16 * ch, o2);
+          }
+        }
+      }
+      const float mu_lo = m_lo == -INFINITY ? 0.f : m_lo;
+      const float mu_hi = m_hi == -INFINITY ? 0.f : m_hi;
+      float sl = 0.f, sh = 0.f, cl = 0.f, ch_ = 0.f;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float pv = ex2(x[i] - ((i & 2) ? mu_hi : mu_lo));
+        const float sv = HAS_R ? __uint_as_float(rs[i]) : 0.f;
+        const float psv = pv * sv;
+        if (i & 2) { sh += pv; ch_ += psv; } else { sl += pv; cl += psv; }
+        ra[i] = __float_as_uint(pv);
+        rs[i] = __float_as_uint(psv);
+      }
+      l_lo += sl; l_hi += sh; c_lo += cl; c_hi += ch_;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pp[16], pq[16];
+#pragma unroll
+        for (int gg = 0; gg < 8; ++gg) {
+          const int i = 32 * hf + 4 * gg;
+          pp[2 * gg] = pack_bf16(__uint_as_float(ra[i]), __uint_as_float(ra[i + 1]));
+          pp[2 * gg + 1] = pack_bf16(__uint_as_float(ra[i + 2]), __uint_as_float(ra[i + 3]));
+          pq[2 * gg] = pack_bf16(__uint_as_float(rs[i]), __uint_as_float(rs[i + 1]));
+          pq[2 * gg + 1] = pack_bf16(__uint_as_float(rs[i + 2]), __uint_as_float(rs[i + 3]));
+        }
+        tc::st_16x128b_x8(ta + 32 * hf, pp);
+        tc::st_16x128b_x8(ts + 32 * hf, pq);
+      }
+      tc::wait_st();
+      tc::fence_before_sync();
+      mbar_arrive(smem_u32(&p_ready[t]));
+    }
+
+    const bool fin_ok = ok && mbar_wait(smem_u32(&o_done[t]), 0, kErrFwdSoftmax);
+    if (__all_sync(0xffffffffu, fin_ok)) {
+      tc::fence_after_sync();
+      l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
+      l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
+      l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
+      l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+      c_lo += __shfl_xor_sync(0xffffffffu, c_lo, 1);
+      c_lo += __shfl_xor_sync(0xffffffffu, c_lo, 2);
+      c_hi += __shfl_xor_sync(0xffffffffu, c_hi, 1);
+      c_hi += __shfl_xor_sync(0xffffffffu, c_hi, 2);
+      const float inv_lo = l_lo > 0.f ? 1.f / l_lo : 0.f;
+      const float inv_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
+      const float sb_lo = c_lo * inv_lo, sb_hi = c_hi * inv_hi;  // s_bar = c / l
+      const size_t plane = static_cast<size_t>(b) * p.Hq + head_of(t);
+      __nv_bfloat16* out_lo = p.out + (plane * p.N + (q_lo < p.N ? q_lo : 0)) * D;
+      __nv_bfloat16* out_hi = p.out + (plane * p.N + (q_hi < p.N ? q_hi : 0)) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t o1[16], o2[16];
+        tc::ld_16x256b_x4(to1 + 32 * ch, o1);
+        tc::ld_16x256b_x4(to2 + 32 * ch, o2);
+        tc::wait_ld();
+#pragma unroll
+        for (int gg = 0; gg < 4; ++gg) {
+          const int dcol = 32 * ch + 8 * gg + 2 * c4;
+          float r[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float inv = (e & 2) ? inv_hi : inv_lo;
+            const float sb = (e & 2) ? sb_hi : sb_lo;
+            const float a1 = __uint_as_float(o1[4 * gg + e]) * inv;  // O1 / l
+            const float a2 = __uint_as_float(o2[4 * gg + e]) * inv;  // O2 / l
+            r[e] = a1 - (a2 - sb * a1);
+          }
+          if (q_lo < p.N) *reinterpret_cast<uint32_t*>(out_lo + dcol) = pack_bf16(r[0], r[1]);
+          if (q_hi < p.N) *reinterpret_cast<uint32_t*>(out_hi + dcol) = pack_bf16(r[2], r[3]);
+        }
+      }
+      if (p.lse && c4 == 0) {
+        if (q_lo < p.N) p.lse[plane * p.N + q_lo] = l_lo > 0.f ? (m_lo + __log2f(l_lo)) * kLn2 : -INFINITY;
+        if (q_hi < p.N) p.lse[plane * p.N + q_hi] = l_hi > 0.f ? (m_hi + __log2f(l_hi)) * kLn2 : -INFINITY;
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == kFwdMmaWarp) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace plx

@@ -1,0 +1,175 @@
+"""Python binding of libplx.so (include/plx.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls.  Tensors are
+PyTorch CUDA tensors (PyTorch provides device memory and the current
+stream); every step of the computation runs in the library's kernels.
+Importing this module loads the library and raises ImportError if it has not
+been built (``python -m parameterized_local_linear_plx_b200.build``): there is
+no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libplx.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build it with `python -m parameterized_local_linear_plx_b200.build` "
+        "(the library has no CPU fallback)")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+_lib.plx_version.restype = _I
+_lib.plx_version.argtypes = []
+_lib.plx_status_string.restype = ctypes.c_char_p
+_lib.plx_status_string.argtypes = [_I]
+_lib.plx_fwd.restype = _I
+_lib.plx_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
+_lib.plx_decode_num_splits.restype = _I
+_lib.plx_decode_num_splits.argtypes = [_I, _I, _I, _I, _I]
+_lib.plx_decode_workspace_size.restype = _SZ
+_lib.plx_decode_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I]
+_lib.plx_decode.restype = _I
+_lib.plx_decode.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P]
+_lib.plx_check_device_status.restype = _I
+_lib.plx_check_device_status.argtypes = [_P]
+_lib.plx_selftest_wait_timeout.restype = _I
+_lib.plx_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, _P]
+
+PLX_OK = 0
+PLX_ERR_NULL = -1
+PLX_ERR_SHAPE = -2
+PLX_ERR_HEADDIM = -3
+PLX_ERR_GQA = -4
+PLX_ERR_ALIGN = -5
+PLX_ERR_WORKSPACE = -6
+PLX_ERR_CUDA = -7
+PLX_ERR_DEVICE_TIMEOUT = -8
+PLX_ERR_ARCH = -9
+
+LIB_PATH = _LIB_PATH
+lib = _lib  # the raw ctypes handle, for callers that pass their own pointers
+
+
+class PlxError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {plx_status_string(status)} ({status})")
+
+
+def plx_version() -> int:
+    return _lib.plx_version()
+
+
+def plx_status_string(status: int) -> str:
+    return _lib.plx_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(t, name, dtype, ndim):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def plx_fwd(q, k, v, r=None, causal=True, scale=None, out=None, lse=None, return_lse=True, stream=None):
+    """Parallax forward over full sequences.
+
+    q [B, Hq, N, d], k/v [B, Hkv, N, d], r [B, Hq, N, d] or None (rho = 0), all
+    bf16 CUDA.  Returns (out [B, Hq, N, d] bf16, lse [B, Hq, N] fp32 or None).
+    """
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    if r is not None:
+        _check(r, "r", torch.bfloat16, 4)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape or (r is not None and r.shape != q.shape):
+        raise ValueError("shape mismatch between q, k, v, r")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
+    st = _lib.plx_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
+                      1 if causal else 0, float(scale), _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_fwd")
+    return out, lse
+
+
+def plx_decode_num_splits(B, Hq, Hkv, S_max, d) -> int:
+    return _lib.plx_decode_num_splits(B, Hq, Hkv, S_max, d)
+
+
+def plx_decode_workspace_size(B, Hq, Hkv, S_max, d, num_splits=0) -> int:
+    return int(_lib.plx_decode_workspace_size(B, Hq, Hkv, S_max, d, num_splits))
+
+
+def plx_decode(q, kcache, vcache, seqlens, r=None, scale=None, num_splits=0, out=None, lse=None,
+               workspace=None, return_lse=True, stream=None):
+    """One decode step.  q/r [B, Hq, d] bf16, caches [B, Hkv, S_max, d] bf16,
+    seqlens [B] int32 (device).  Returns (out [B, Hq, d] bf16, lse [B, Hq] fp32 or None).
+    workspace: optional uint8 CUDA tensor of at least plx_decode_workspace_size bytes."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(kcache, "kcache", torch.bfloat16, 4)
+    _check(vcache, "vcache", torch.bfloat16, 4)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    if r is not None:
+        _check(r, "r", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    Hkv, S_max = kcache.shape[1], kcache.shape[2]
+    if kcache.shape != (B, Hkv, S_max, d) or vcache.shape != kcache.shape or seqlens.shape != (B,) \
+            or (r is not None and r.shape != q.shape):
+        raise ValueError("shape mismatch between q, caches, seqlens, r")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    need = plx_decode_workspace_size(B, Hq, Hkv, S_max, d, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.plx_decode(_ptr(q), _ptr(r), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(out), _ptr(lse),
+                         B, Hq, Hkv, S_max, d, float(scale), int(num_splits), _ptr(workspace), ws_bytes,
+                         _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_decode")
+    return out, lse
+
+
+def plx_check_device_status(stream=None) -> int:
+    """Synchronise the stream, read and clear the device error word; returns the status."""
+    return _lib.plx_check_device_status(_stream(stream))
+
+
+def plx_selftest_wait_timeout(limit_cycles: int, stream=None) -> int:
+    return _lib.plx_selftest_wait_timeout(int(limit_cycles), _stream(stream))

@@ -1,0 +1,119 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/plx.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "plx.h")
+
+
+@pytest.fixture(scope="module")
+def plx():
+    from parameterized_local_linear_plx_b200 import build
+    build.build()
+    from parameterized_local_linear_plx_b200 import plx as m
+    return m
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(plx_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_entry_points()
+    for n in ["plx_fwd", "plx_decode", "plx_decode_workspace_size", "plx_decode_num_splits",
+              "plx_check_device_status", "plx_status_string", "plx_version", "plx_selftest_wait_timeout"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(plx):
+    out = subprocess.run(["nm", "-D", "--defined-only", plx.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (plx_[a-z0-9_]+)\b", out))
+    missing = [n for n in declared_entry_points() if n not in exported]
+    assert not missing, missing
+    for n in declared_entry_points():
+        assert hasattr(plx.lib, n)
+
+
+def test_header_is_plain_c():
+    """The header compiles as C99 with no CUDA or torch includes."""
+    src = '#include "plx.h"\nint main(void){ return plx_version() > 0 ? 0 : 1; }\n'
+    res = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-I", os.path.dirname(HEADER),
+                          "-x", "c", "-"], input=src, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+
+
+def test_status_strings(plx):
+    for code in range(-9, 1):
+        s = plx.plx_status_string(code)
+        assert s.startswith("PLX_")
+    assert "unknown" in plx.plx_status_string(-100)
+    assert plx.plx_version() >= 100
+
+
+P = ctypes.c_void_p
+A = 0x10000  # a 16-byte aligned fake device address; never dereferenced on these paths
+
+
+def fwd(plx, q=A, k=A, v=A, r=A, out=A, lse=A, B=1, Hq=2, Hkv=1, N=8, d=64, causal=1):
+    return plx.lib.plx_fwd(P(q), P(k), P(v), P(r), P(out), P(lse), B, Hq, Hkv, N, d, causal, 0.125, None)
+
+
+def dec(plx, q=A, r=A, kc=A, vc=A, sl=A, out=A, lse=A, B=1, Hq=2, Hkv=1, S=64, d=64, splits=1, ws=None, wsb=0):
+    return plx.lib.plx_decode(P(q), P(r), P(kc), P(vc), P(sl), P(out), P(lse), B, Hq, Hkv, S, d, 0.125,
+                              splits, P(ws), wsb, None)
+
+
+def test_fwd_argument_errors(plx):
+    assert fwd(plx, q=None) == plx.PLX_ERR_NULL
+    assert fwd(plx, k=None) == plx.PLX_ERR_NULL
+    assert fwd(plx, v=None) == plx.PLX_ERR_NULL
+    assert fwd(plx, out=None) == plx.PLX_ERR_NULL
+    for kw in [dict(B=0), dict(Hq=0), dict(Hkv=0), dict(N=0), dict(N=-3)]:
+        assert fwd(plx, **kw) == plx.PLX_ERR_SHAPE, kw
+    for d in [0, 32, 96, 256]:
+        assert fwd(plx, d=d) == plx.PLX_ERR_HEADDIM
+    assert fwd(plx, Hq=3, Hkv=2) == plx.PLX_ERR_GQA
+    assert fwd(plx, q=A + 8) == plx.PLX_ERR_ALIGN
+    assert fwd(plx, r=A + 2) == plx.PLX_ERR_ALIGN
+    assert fwd(plx, lse=A + 2) == plx.PLX_ERR_ALIGN
+
+
+def test_decode_argument_errors(plx):
+    assert dec(plx, q=None) == plx.PLX_ERR_NULL
+    assert dec(plx, kc=None) == plx.PLX_ERR_NULL
+    assert dec(plx, sl=None) == plx.PLX_ERR_NULL
+    assert dec(plx, B=0) == plx.PLX_ERR_SHAPE
+    assert dec(plx, S=0) == plx.PLX_ERR_SHAPE
+    assert dec(plx, splits=-1) == plx.PLX_ERR_SHAPE
+    assert dec(plx, d=100) == plx.PLX_ERR_HEADDIM
+    assert dec(plx, Hq=5, Hkv=2) == plx.PLX_ERR_GQA
+    assert dec(plx, vc=A + 4) == plx.PLX_ERR_ALIGN
+    assert dec(plx, sl=A + 2) == plx.PLX_ERR_ALIGN
+    # two splits need a workspace
+    assert dec(plx, S=256, splits=2) == plx.PLX_ERR_WORKSPACE
+    need = plx.plx_decode_workspace_size(1, 2, 1, 256, 64, 2)
+    assert dec(plx, S=256, splits=2, ws=A, wsb=need - 1) == plx.PLX_ERR_WORKSPACE
+    assert dec(plx, S=256, splits=2, ws=A + 4, wsb=need) == plx.PLX_ERR_ALIGN
+
+
+def test_split_planning(plx):
+    # one split needs no workspace
+    assert plx.plx_decode_workspace_size(4, 16, 8, 1000, 128, 1) == 0
+    # explicit count: (2d + 4) floats per (b, h, split)
+    assert plx.plx_decode_workspace_size(2, 4, 2, 1024, 128, 4) == 2 * 4 * 4 * (2 * 128 + 4) * 4
+    # the automatic count is at least one and never gives chunks below 128 keys
+    for B, S in [(1, 128), (1, 4096), (16, 4096), (64, 4096), (2048, 16384)]:
+        n = plx.plx_decode_num_splits(B, 16, 8, S, 128)
+        assert 1 <= n <= max(1, (S + 127) // 128)
+    assert plx.plx_decode_num_splits(1, 16, 8, 4096, 128) > 1
+    assert plx.plx_decode_num_splits(2048, 16, 8, 16384, 128) == 1
+    # bad shapes: count 1, size 0
+    assert plx.plx_decode_num_splits(0, 16, 8, 4096, 128) == 1
+    assert plx.plx_decode_workspace_size(1, 3, 2, 128, 128, 2) == 0

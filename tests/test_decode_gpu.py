@@ -1,0 +1,136 @@
+"""Decode (split-KV) on the GPU against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import assert_close
+from parameterized_local_linear_plx_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def plx():
+    from parameterized_local_linear_plx_b200 import build
+    build.build()
+    from parameterized_local_linear_plx_b200 import plx as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def run(plx, B, Hq, Hkv, S, d, seqlens="equal", seed=0, use_r=True, splits=0, r_scale=0.1, batches=None):
+    q, kc, vc, r, sl = inputs.decode_inputs(B, Hq, Hkv, S, d, seed=seed, seqlens=seqlens, r_scale=r_scale)
+    dev = "cuda"
+    out, lse = plx.plx_decode(q.to(dev), kc.to(dev), vc.to(dev), sl.to(dev), r.to(dev) if use_r else None,
+                              num_splits=splits)
+    torch.cuda.synchronize()
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    ro, rl = oracle.decode_effective(q, r if use_r else None, kc, vc, sl, batches=batches)
+    o, l = out.float().cpu().numpy(), lse.cpu().numpy()
+    if batches is not None:
+        o, l, ro, rl = o[batches], l[batches], ro[batches], rl[batches]
+    return o, l, ro, rl
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2), (16, 8), (8, 1), (24, 2)])
+def test_decode_parity_shapes(plx, d, Hq, Hkv):
+    o, l, ro, rl = run(plx, 3, Hq, Hkv, 200, d, seqlens=[200, 1, 130])
+    assert_close(o, ro, l, rl, f"d={d} Hq={Hq} Hkv={Hkv}")
+
+
+@pytest.mark.parametrize("S", [1, 2, 63, 64, 65, 127, 129, 1000])
+def test_decode_ragged_lengths(plx, S):
+    o, l, ro, rl = run(plx, 2, 4, 2, S, 128, seqlens=[S, max(1, S // 3)], seed=S)
+    assert_close(o, ro, l, rl, f"S={S}")
+
+
+def test_decode_empty_context(plx):
+    q, kc, vc, r, sl = inputs.decode_inputs(3, 4, 2, 256, 128, seed=3, seqlens=[0, 256, -5])
+    for splits in (1, 2, 0):
+        out, lse = plx.plx_decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda(), r.cuda(), num_splits=splits)
+        o, l = out.float().cpu().numpy(), lse.cpu().numpy()
+        assert (o[0] == 0).all() and (o[2] == 0).all()
+        assert np.isneginf(l[0]).all() and np.isneginf(l[2]).all()
+        ro, rl = oracle.decode_effective(q, r, kc, vc, sl)
+        assert_close(o, ro, l, rl, f"splits={splits}")
+
+
+def test_decode_seqlen_clamped_to_cache(plx):
+    q, kc, vc, r, _ = inputs.decode_inputs(2, 4, 2, 96, 64, seed=4)
+    sl = torch.tensor([500, 96], dtype=torch.int32)
+    out, lse = plx.plx_decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda(), r.cuda())
+    ro, rl = oracle.decode_effective(q, r, kc, vc, torch.tensor([96, 96]))
+    assert_close(out, ro, lse, rl)
+
+
+def test_decode_split_invariance(plx):
+    q, kc, vc, r, sl = inputs.decode_inputs(4, 16, 8, 2048, 128, seed=5, seqlens="ragged")
+    args = (q.cuda(), kc.cuda(), vc.cuda(), sl.cuda(), r.cuda())
+    ref_o, ref_l = plx.plx_decode(*args, num_splits=1)
+    ro, rl = oracle.decode_effective(q, r, kc, vc, sl)
+    assert_close(ref_o, ro, ref_l, rl, "splits=1")
+    for s in (2, 3, 7, 16, 0):
+        o, l = plx.plx_decode(*args, num_splits=s)
+        assert_close(o, ro, l, rl, f"splits={s}")
+        # different splits differ only by rounding
+        assert (o.float() - ref_o.float()).abs().max().item() <= 1e-2
+
+
+def test_decode_r_none_equals_r_zero_and_softmax(plx):
+    q, kc, vc, r, sl = inputs.decode_inputs(2, 8, 4, 300, 128, seed=6, seqlens=[300, 123])
+    a = plx.plx_decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda(), None)
+    b = plx.plx_decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda(), torch.zeros_like(r).cuda())
+    assert torch.equal(a[0], b[0])
+    assert torch.allclose(a[1], b[1], rtol=0, atol=0)
+    # rho = 0 is softmax attention: compare with torch SDPA in fp64 on the host
+    qq = q.double()[:, :, None]
+    for bb, n in enumerate([300, 123]):
+        kk = kc.double()[bb:bb + 1, :, :n].repeat_interleave(2, 1)
+        vv = vc.double()[bb:bb + 1, :, :n].repeat_interleave(2, 1)
+        ref = torch.nn.functional.scaled_dot_product_attention(qq[bb:bb + 1], kk, vv)[0, :, 0]
+        assert (a[0][bb].double().cpu() - ref).abs().max().item() < 1e-2
+
+
+def test_decode_stress_inputs(plx):
+    """Peaked scores, correlated values (large covariance) and a large probe."""
+    B, Hq, Hkv, S, d = 2, 4, 2, 512, 128
+    q, kc, vc, r, sl = inputs.decode_inputs(B, Hq, Hkv, S, d, seed=7, r_scale=1.0, seqlens=[512, 400])
+    q = (q.float() * 4).bfloat16()
+    g = torch.Generator().manual_seed(8)
+    W = torch.randn(d, d, generator=g) / d ** 0.5
+    vc = (kc.float() @ W + 0.1 * torch.randn(kc.shape, generator=g)).bfloat16()
+    out, lse = plx.plx_decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda(), r.cuda())
+    ro, rl = oracle.decode_effective(q, r, kc, vc, sl)
+    assert_close(out, ro, lse, rl, "stress", scale_abs=True)
+
+
+@pytest.mark.parametrize("B", [1, 16, 64])
+def test_decode_qwen3_layer_full_size(plx, B):
+    """B in {1, 16, 64}, context 4096, Hq=16, Hkv=8, d=128, equal seqlens; the
+    same launch configuration (automatic split count) the benchmark times."""
+    o, l, ro, rl = run(plx, B, 16, 8, 4096, 128, seqlens="equal", seed=0)
+    assert_close(o, ro, l, rl, f"B={B}")
+
+
+def test_decode_sweep_point_ragged(plx):
+    """A decode-sweep point with ragged seqlens in [ctx/2, ctx], sampled batches."""
+    B, ctx = 256, 1024
+    q, kc, vc, r, sl = inputs.decode_inputs(B, 16, 8, ctx, 128, seed=9, seqlens="ragged", device="cuda")
+    out, lse = plx.plx_decode(q, kc, vc, sl, r)
+    pick = [0, 1, 77, 128, 255]
+    qc, kcc, vcc, rc, slc = (t[pick].cpu() for t in (q, kc, vc, r, sl))
+    ro, rl = oracle.decode_effective(qc, rc, kcc, vcc, slc)
+    assert_close(out[pick], ro, lse[pick], rl, "sweep point")
+
+
+def test_decode_timeout_path_reports_and_recovers(plx):
+    """A bounded wait that nothing completes: the kernel records a timeout,
+    returns, and the context stays usable."""
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    assert plx.plx_selftest_wait_timeout(2_000_000) == plx.PLX_OK  # ~1 ms
+    assert plx.plx_check_device_status() == plx.PLX_ERR_DEVICE_TIMEOUT
+    assert plx.plx_check_device_status() == plx.PLX_OK  # cleared
+    o, l, ro, rl = run(plx, 2, 4, 2, 128, 128, seed=11)
+    assert_close(o, ro, l, rl, "after timeout")
