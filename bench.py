@@ -105,56 +105,98 @@ def load_traffic(kernel_key):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples every 200 ms while timing."""
+    """SM clock and clock-event (throttle) reasons sampled while timing.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Polls NVML (the library nvidia-smi reads) from a thread every ~2 ms, so
+    even a short timed region gets samples; falls back to `nvidia-smi -lms 50`.
+    """
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, cuda_index):
+        self.cuda_index = cuda_index
+        self.gpu = str(cuda_index)  # nvidia-smi -i: the device UUID when known
+        self.uuid = None
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(cuda_index).uuid)
+            self.uuid = u if u.startswith("GPU-") else "GPU-" + u
+            self.gpu = self.uuid
+        except Exception:
+            pass
+        self.samples = []  # (sm_mhz, max_mhz, reasons_mask)
+        self._stop = None
+        self._thread = None
+        self._proc = None
+
+    def _poll_nvml(self, handle, nvml):
+        import time as _t
+        while not self._stop.is_set():
+            try:
+                sm = nvml.nvmlDeviceGetClockInfo(handle, nvml.NVML_CLOCK_SM)
+                mx = nvml.nvmlDeviceGetMaxClockInfo(handle, nvml.NVML_CLOCK_SM)
+                try:
+                    rs = nvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                except Exception:
+                    rs = nvml.nvmlDeviceGetCurrentClocksThrottleReasons(handle)
+                self.samples.append((float(sm), float(mx), int(rs)))
+            except Exception:
+                pass
+            _t.sleep(0.002)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml as nvml
+            nvml.nvmlInit()
+            # NVML numbers GPUs ignoring CUDA_VISIBLE_DEVICES: find ours by UUID
+            handle = (nvml.nvmlDeviceGetHandleByUUID(self.uuid.encode()) if self.uuid
+                      else nvml.nvmlDeviceGetHandleByIndex(self.cuda_index))
+            self._stop = threading.Event()
+            self._thread = threading.Thread(target=self._poll_nvml, args=(handle, nvml), daemon=True)
+            self._thread.start()
         except Exception:
-            self.proc = None
+            self._thread = None
+            try:
+                self._proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=clocks.sm,clocks.max.sm,"
+                     "clocks_event_reasons.active", "--format=csv,noheader,nounits", "-lms", "50"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except Exception:
+                self._proc = None
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                out, _ = self._proc.communicate(timeout=5)
             except Exception:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+                self._proc.kill()
+                out, _ = self._proc.communicate()
+            for ln in out.splitlines():
+                parts = [x.strip() for x in ln.split(",")]
+                try:
+                    self.samples.append((float(parts[0]), float(parts[1]), int(parts[2], 16)))
+                except Exception:
+                    continue
         return False
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for _, _, mask in self.samples:
+            for bit, name in self.REASONS.items():
+                if mask & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": max(s[1] for s in self.samples), "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": "nvml" if self._thread is not None else "nvidia-smi"}
 
 
 # ------------------------------------------------------------------ distributed
@@ -200,14 +242,15 @@ def cpu_threads():
 
 def oracle_decode_sample(q, r, kc, vc, sl, budget_s=10.0, max_entries=None):
     """Run the oracle's effective-weight decode on batch entries one at a time
-    until ~budget_s of CPU time is used.  Returns (entries, seconds, bytes)."""
+    (cycling over them) until ~budget_s of wall time is used or max_entries
+    are done.  Returns (entries, seconds, bytes)."""
     import oracle
     B, Hq, d = q.shape
     Hkv = kc.shape[1]
     done, t0, nbytes = 0, time.perf_counter(), 0
-    limit = max_entries or B
+    limit = max_entries or 1 << 30
     while done < limit:
-        b = done
+        b = done % B  # cycle over the entries until the budget is used
         oracle.decode_effective(q[b:b + 1], r[b:b + 1], kc[b:b + 1], vc[b:b + 1], sl[b:b + 1])
         nbytes += decode_bytes(1, Hq, Hkv, d, sl[b:b + 1].tolist())
         done += 1
@@ -346,11 +389,11 @@ def run_gpu(args, world, rank, local):
     # ---- CPU baseline: the oracle on this host, rank 0, N=1 only
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        qh, kh, vh, rh, slh = (t[:8].cpu() for t in (q, kc, vc, r, sl))
+        qh, kh, vh, rh, slh = (t.cpu() for t in (q, kc, vc, r, sl))
         n, secs, nb = oracle_decode_sample(qh, rh, kh, vh, slh, budget_s=10.0)
         cpu = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"{n} of {DEC['B']} batch entries of the decode step (all {DEC['Hq']} heads, "
-                         f"{DEC['S']} keys), effective-weight fp64 form, {secs:.1f} s"}
+               "sample": f"{n} (b) entries of the B={DEC['B']} decode step, cycling (each: all {DEC['Hq']} "
+                         f"heads x {DEC['S']} keys), effective-weight fp64 form, {secs:.1f} s"}
 
     clocks = clk.summary()
     if rank == 0:
@@ -359,10 +402,12 @@ def run_gpu(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {
-                "workload": "decode: Qwen3-0.6B-shaped layer B=64 ctx=4096 (equal seqlens) Hq=16 Hkv=8 d=128 "
-                            "bf16 KV cache; prefill: B=8 N=4096 Hq=16 Hkv=8 d=128 causal bf16, out+lse",
+                "workload": f"decode: Qwen3-0.6B-shaped layer B={DEC['B']} ctx={DEC['S']} (equal seqlens) "
+                            f"Hq=16 Hkv=8 d=128 bf16 KV cache; prefill: B={PRE['B']} N={PRE['N']} Hq=16 Hkv=8 "
+                            "d=128 causal bf16, out+lse",
                 "decode_splits": n_splits,
-                "l2": "inputs larger than L2 (decode KV 1.07 GB, prefill 0.54 GB per step)",
+                "l2": f"inputs larger than L2 (decode {d_bytes / 1e9:.2f} GB, prefill "
+                      f"{prefill_bytes(**PRE) / 1e9:.2f} GB per step; L2 126 MB)",
                 "parallelism": f"replicas x{world}, no collective on the data path",
             },
             "decode": {"gbs": value, "us_per_step": dec_avg * 1e3, "bytes_per_step": d_bytes,
@@ -493,15 +538,20 @@ def run_compute_matched(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["plx", "reference"], default="plx")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--small", action="store_true",
+                    help="profiling-size workload: decode B=16, prefill B=2 (both still larger than L2)")
     ap.add_argument("--sweep", action="store_true", help="decode sweep lines instead of the bench line")
     ap.add_argument("--compute-matched", action="store_true", help="compute-matched decode comparison")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.small:
+        DEC["B"] = 16
+        PRE["B"] = 2
     world, rank, local = dist_setup()
     if args.gpus != world and world > 1:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")

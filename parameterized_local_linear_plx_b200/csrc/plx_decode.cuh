@@ -38,7 +38,7 @@ struct DecodeCfg {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kStages = D == 128 ? 3 : 6;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-  static constexpr int kPartialFloats = 2 * D + 4;             // m, l, c, pad, O1[D], O2[D]
+  static constexpr int kPartialFloats = 2 * D + 4;             // m, l, c, e, O1[D], O2[D]
 };
 
 struct DecodeParams {
@@ -48,6 +48,7 @@ struct DecodeParams {
   __nv_bfloat16* out;       // [B, Hq, D]
   float* lse;               // [B, Hq] or nullptr
   float* ws;                // [B, Hq, splits, 2D+4] or nullptr when splits == 1
+                            //   per row: m (log2 units), l, c, e (sum of unrounded p), O1[D], O2[D]
   int B, Hq, Hkv, S_max, G, n_hgroups, splits, chunk;
   float scale_log2;         // scale * log2(e)
 };
@@ -173,6 +174,7 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
   for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
   float m_run = -INFINITY, l_run = 0.f, c_run = 0.f;  // l, c: this thread's column share
+  float e_run = 0.f;  // sum of unrounded p, for lse only
 
   // ldmatrix row addresses (relative to a K or V tile) for this lane.
   const int mi = lane >> 3, ri = lane & 7;
@@ -220,15 +222,21 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
     for (int i = 0; i < 4; ++i) pr[i] = ex2(x[i] - m_use);
     const float sv[4] = {acc[0][2], acc[0][3], acc[1][2], acc[1][3]};  // rho.k, same keys
-    float psum = 0.f, csum = 0.f, ps[4];
+    float ps[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ps[i] = HAS_R ? pr[i] * sv[i] : 0.f;
-      psum += pr[i];
-      csum += ps[i];
-    }
+    for (int i = 0; i < 4; ++i) ps[i] = HAS_R ? pr[i] * sv[i] : 0.f;
+    // stacked A operand of the value MMA: rows g = P, rows g+8 = P*S (bf16)
+    uint32_t pa[4];
+    pa[0] = pack_bf16(pr[0], pr[1]);
+    pa[1] = pack_bf16(ps[0], ps[1]);
+    pa[2] = pack_bf16(pr[2], pr[3]);
+    pa[3] = pack_bf16(ps[2], ps[3]);
+    // l and c from the rounded values the MMA consumes: effective weights sum to one
+    const float psum = bf16_lo(pa[0]) + bf16_hi(pa[0]) + bf16_lo(pa[2]) + bf16_hi(pa[2]);
+    const float csum = bf16_lo(pa[1]) + bf16_hi(pa[1]) + bf16_lo(pa[3]) + bf16_hi(pa[3]);
     l_run = l_run * alpha + psum;
     c_run = c_run * alpha + csum;
+    e_run = e_run * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
     m_run = m_new;
     if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
@@ -238,11 +246,6 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     }
 
     // ---- value product with the stacked [P ; P*S] operand
-    uint32_t pa[4];
-    pa[0] = pack_bf16(pr[0], pr[1]);
-    pa[1] = pack_bf16(ps[0], ps[1]);
-    pa[2] = pack_bf16(pr[2], pr[3]);
-    pa[3] = pack_bf16(ps[2], ps[3]);
 #pragma unroll
     for (int jp = 0; jp < D / 16; ++jp) {
       const int chunk = (2 * jp + (mi >> 1)) & 7;
@@ -261,20 +264,22 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
   c_run += __shfl_xor_sync(0xffffffffu, c_run, 1);
   c_run += __shfl_xor_sync(0xffffffffu, c_run, 2);
+  e_run += __shfl_xor_sync(0xffffffffu, e_run, 1);
+  e_run += __shfl_xor_sync(0xffffffffu, e_run, 2);
   asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumerWarps * 32) : "memory");
 
-  constexpr int kRowF = 2 * D + 3;  // m, l, c, O1[D], O2[D]
+  constexpr int kRowF = 2 * D + 4;  // m, l, c, e, O1[D], O2[D]
   float* red = reinterpret_cast<float*>(smem);
   {
     float* mine = red + (warp * 8 + gr) * kRowF;
-    if (qc == 0) { mine[0] = m_run; mine[1] = l_run; mine[2] = c_run; }
+    if (qc == 0) { mine[0] = m_run; mine[1] = l_run; mine[2] = c_run; mine[3] = e_run; }
 #pragma unroll
     for (int j = 0; j < D / 8; ++j) {
       const int dd = j * 8 + qc * 2;
-      mine[3 + dd] = o[j][0];
-      mine[3 + dd + 1] = o[j][1];
-      mine[3 + D + dd] = o[j][2];
-      mine[3 + D + dd + 1] = o[j][3];
+      mine[4 + dd] = o[j][0];
+      mine[4 + dd + 1] = o[j][1];
+      mine[4 + D + dd] = o[j][2];
+      mine[4 + D + dd + 1] = o[j][3];
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumerWarps * 32) : "memory");
@@ -286,15 +291,16 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
     for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, red[(w * 8 + hh) * kRowF]);
     const float Mu = M == -INFINITY ? 0.f : M;
-    float L = 0.f, C = 0.f, O1 = 0.f, O2 = 0.f;
+    float L = 0.f, C = 0.f, E = 0.f, O1 = 0.f, O2 = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecConsumerWarps; ++w) {
       const float* rw = red + (w * 8 + hh) * kRowF;
       const float beta = ex2(rw[0] - Mu);
       L += beta * rw[1];
       C += beta * rw[2];
-      O1 += beta * rw[3 + dd];
-      O2 += beta * rw[3 + D + dd];
+      E += beta * rw[3];
+      O1 += beta * rw[4 + dd];
+      O2 += beta * rw[4 + D + dd];
     }
     const size_t row = static_cast<size_t>(b) * p.Hq + h0 + hh;
     if (p.splits == 1) {
@@ -305,10 +311,10 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
         res = o1 - (O2 * inv - (C * inv) * o1);
       }
       p.out[row * D + dd] = __float2bfloat16(res);
-      if (dd == 0 && p.lse) p.lse[row] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+      if (dd == 0 && p.lse) p.lse[row] = E > 0.f ? (M + __log2f(E)) * kLn2 : -INFINITY;
     } else {
       float* ws = p.ws + (row * p.splits + split) * Cfg::kPartialFloats;
-      if (dd == 0) { ws[0] = M; ws[1] = L; ws[2] = C; ws[3] = 0.f; }
+      if (dd == 0) { ws[0] = M; ws[1] = L; ws[2] = C; ws[3] = E; }
       ws[4 + dd] = O1;
       ws[4 + D + dd] = O2;
     }
@@ -327,12 +333,13 @@ plx_decode_combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restric
   float M = -INFINITY;
   for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldg(base + s * PF));
   const float Mu = M == -INFINITY ? 0.f : M;
-  float L = 0.f, C = 0.f, O1 = 0.f, O2 = 0.f;
+  float L = 0.f, C = 0.f, E = 0.f, O1 = 0.f, O2 = 0.f;
   for (int s = 0; s < splits; ++s) {
     const float* ps = base + s * PF;
     const float beta = ex2(__ldg(ps) - Mu);
     L += beta * __ldg(ps + 1);
     C += beta * __ldg(ps + 2);
+    E += beta * __ldg(ps + 3);
     O1 += beta * __ldg(ps + 4 + dd);
     O2 += beta * __ldg(ps + 4 + D + dd);
   }
@@ -343,7 +350,7 @@ plx_decode_combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restric
     res = o1 - (O2 * inv - (C * inv) * o1);
   }
   out[row * D + dd] = __float2bfloat16(res);
-  if (dd == 0 && lse) lse[row] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+  if (dd == 0 && lse) lse[row] = E > 0.f ? (M + __log2f(E)) * kLn2 : -INFINITY;
 }
 
 }  // namespace plx

@@ -276,6 +276,7 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const int q_hi = q_lo + 8;
     float m_lo = -INFINITY, m_hi = -INFINITY;
     float l_lo = 0.f, l_hi = 0.f, c_lo = 0.f, c_hi = 0.f;  // this thread's column share
+    float e_lo = 0.f, e_hi = 0.f;  // sum of unrounded p, for lse only
 
     for (int j = 0; j < nkv; ++j) {
       // warp-uniform: the .sync.aligned tensor-memory accesses below need every lane
@@ -293,9 +294,8 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 
       // register i: half h = i/32, rep g = (i%32)/4, e = i%4;
       // key = 64h + 8g + 2*c4 + (e&1); row lo for e < 2, row hi for e >= 2.
-      float x[64];
-#pragma unroll
-      for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(ra[i]) * p.scale_log2;
+      // Masked scores become -inf in place; the max is taken on raw q.k and
+      // scaled afterwards (scale_log2 > 0), and the scale folds into exp2's FMA.
       const int kbase = j * kFwdBN;
       const bool need_mask = (p.causal && kbase + kFwdBN - 1 > q0) || (kbase + kFwdBN > p.N);
       if (need_mask) {
@@ -304,25 +304,26 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           const int key = kbase + 64 * (i >> 5) + 8 * ((i & 31) >> 2) + 2 * c4 + (i & 1);
           const int q = (i & 2) ? q_hi : q_lo;
           const bool valid = key < p.N && (!p.causal || key <= q);
-          x[i] = valid ? x[i] : -INFINITY;
+          if (!valid) ra[i] = 0xFF800000u;  // -inf
         }
       }
       float mx_lo = -INFINITY, mx_hi = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 64; i += 4) {
-        mx_lo = fmaxf(mx_lo, fmaxf(x[i], x[i + 1]));
-        mx_hi = fmaxf(mx_hi, fmaxf(x[i + 2], x[i + 3]));
+        mx_lo = fmaxf(mx_lo, fmaxf(__uint_as_float(ra[i]), __uint_as_float(ra[i + 1])));
+        mx_hi = fmaxf(mx_hi, fmaxf(__uint_as_float(ra[i + 2]), __uint_as_float(ra[i + 3])));
       }
       mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
       mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
-      mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
-      mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
+      mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2)) * p.scale_log2;
+      mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2)) * p.scale_log2;
       const bool grow = mx_lo > m_lo + kRescaleThreshold || mx_hi > m_hi + kRescaleThreshold;
       if (__any_sync(0xffffffffu, grow)) {
         const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
         const float al_lo = mn_lo == -INFINITY ? 1.f : ex2(m_lo - mn_lo);
         const float al_hi = mn_hi == -INFINITY ? 1.f : ex2(m_hi - mn_hi);
         l_lo *= al_lo; c_lo *= al_lo; l_hi *= al_hi; c_hi *= al_hi;
+        e_lo *= al_lo; e_hi *= al_hi;
         m_lo = mn_lo; m_hi = mn_hi;
         if (j > 0) {
           // O rows of this warp: O1 at the a lanes, O2 at the s lanes; PV(j-1)
@@ -346,17 +347,19 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       }
       const float mu_lo = m_lo == -INFINITY ? 0.f : m_lo;
       const float mu_hi = m_hi == -INFINITY ? 0.f : m_hi;
-      float sl = 0.f, sh = 0.f, cl = 0.f, ch_ = 0.f;
+      float xl = 0.f, xh = 0.f;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        const float pv = ex2(x[i] - ((i & 2) ? mu_hi : mu_lo));
+        const float pv = ex2(fmaf(__uint_as_float(ra[i]), p.scale_log2, (i & 2) ? -mu_hi : -mu_lo));
         const float sv = HAS_R ? __uint_as_float(rs[i]) : 0.f;
-        const float psv = pv * sv;
-        if (i & 2) { sh += pv; ch_ += psv; } else { sl += pv; cl += psv; }
+        if (i & 2) xh += pv; else xl += pv;
         ra[i] = __float_as_uint(pv);
-        rs[i] = __float_as_uint(psv);
+        rs[i] = __float_as_uint(pv * sv);
       }
-      l_lo += sl; l_hi += sh; c_lo += cl; c_hi += ch_;
+      e_lo += xl; e_hi += xh;
+      // l and c are summed from the bf16-rounded P and P*S that the value MMA
+      // consumes, so the output's effective weights sum to exactly one.
+      float sl = 0.f, sh = 0.f, cl = 0.f, ch_ = 0.f;
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t pp[16], pq[16];
@@ -367,10 +370,15 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           pp[2 * gg + 1] = pack_bf16(__uint_as_float(ra[i + 2]), __uint_as_float(ra[i + 3]));
           pq[2 * gg] = pack_bf16(__uint_as_float(rs[i]), __uint_as_float(rs[i + 1]));
           pq[2 * gg + 1] = pack_bf16(__uint_as_float(rs[i + 2]), __uint_as_float(rs[i + 3]));
+          sl += bf16_lo(pp[2 * gg]) + bf16_hi(pp[2 * gg]);
+          sh += bf16_lo(pp[2 * gg + 1]) + bf16_hi(pp[2 * gg + 1]);
+          cl += bf16_lo(pq[2 * gg]) + bf16_hi(pq[2 * gg]);
+          ch_ += bf16_lo(pq[2 * gg + 1]) + bf16_hi(pq[2 * gg + 1]);
         }
         tc::st_16x128b_x8(ta + 32 * hf, pp);
         tc::st_16x128b_x8(ts + 32 * hf, pq);
       }
+      l_lo += sl; l_hi += sh; c_lo += cl; c_hi += ch_;
       tc::wait_st();
       tc::fence_before_sync();
       mbar_arrive(smem_u32(&p_ready[t]));
@@ -387,6 +395,10 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       c_lo += __shfl_xor_sync(0xffffffffu, c_lo, 2);
       c_hi += __shfl_xor_sync(0xffffffffu, c_hi, 1);
       c_hi += __shfl_xor_sync(0xffffffffu, c_hi, 2);
+      e_lo += __shfl_xor_sync(0xffffffffu, e_lo, 1);
+      e_lo += __shfl_xor_sync(0xffffffffu, e_lo, 2);
+      e_hi += __shfl_xor_sync(0xffffffffu, e_hi, 1);
+      e_hi += __shfl_xor_sync(0xffffffffu, e_hi, 2);
       const float inv_lo = l_lo > 0.f ? 1.f / l_lo : 0.f;
       const float inv_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
       const float sb_lo = c_lo * inv_lo, sb_hi = c_hi * inv_hi;  // s_bar = c / l
@@ -416,8 +428,8 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         }
       }
       if (p.lse && c4 == 0) {
-        if (q_lo < p.N) p.lse[plane * p.N + q_lo] = l_lo > 0.f ? (m_lo + __log2f(l_lo)) * kLn2 : -INFINITY;
-        if (q_hi < p.N) p.lse[plane * p.N + q_hi] = l_hi > 0.f ? (m_hi + __log2f(l_hi)) * kLn2 : -INFINITY;
+        if (q_lo < p.N) p.lse[plane * p.N + q_lo] = e_lo > 0.f ? (m_lo + __log2f(e_lo)) * kLn2 : -INFINITY;
+        if (q_hi < p.N) p.lse[plane * p.N + q_hi] = e_hi > 0.f ? (m_hi + __log2f(e_hi)) * kLn2 : -INFINITY;
       }
     }
   }

@@ -152,6 +152,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// The two bf16 halves of a packed word as fp32 (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
 // Hardware base-2 exponential (MUFU); exp2(-inf) = 0.
 __device__ __forceinline__ float ex2(float x) {
   float y;
