@@ -36,7 +36,8 @@
  *   - lse may be NULL (not written).
  *   - The caller owns every buffer.  The library allocates no device or
  *     host memory; it keeps one device word that records a bounded-wait
- *     timeout (see plx_check_device_status).
+ *     timeout (see plx_check_device_status) and one fixed scratch array for
+ *     plx_decode_noalloc.
  *   - stream is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     asynchronous on it.  Argument errors are returned synchronously
  *     before anything is launched; launch failures return PLX_ERR_CUDA.
@@ -130,6 +131,46 @@ int plx_decode(const void* q, const void* r, const void* kcache, const void* vca
                const int32_t* seqlens, void* out, float* lse,
                int B, int Hq, int Hkv, int S_max, int d, float scale, int num_splits,
                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * PLX_NOALLOC_SCRATCH_BYTES -- size of the library's fixed device scratch
+ * array used by plx_decode_noalloc (16 MiB, held on every GPU that loads the
+ * library until the process exits).
+ */
+#define PLX_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
+ * plx_decode_noalloc -- plx_decode for callers that cannot allocate device
+ * memory.  Some callers have no way to call cudaMalloc, or must not: a
+ * plugin inside another runtime that owns all device memory and hands the
+ * plugin only its input and output buffers, or a latency-critical serving
+ * loop whose host forbids device allocation after start-up (an allocation
+ * can synchronise the device or fail under memory pressure).  This entry
+ * point needs no workspace argument:
+ * the split partial states live in a fixed device array inside the library
+ * (PLX_NOALLOC_SCRATCH_BYTES).  The paper has no counterpart to this call; it
+ * is a convenience of this library.
+ *
+ * Arguments, layouts and results are those of plx_decode (without
+ * workspace / workspace_bytes); num_splits = 0 picks the automatic count.
+ *   - The caller still owns and passes every input and output buffer.
+ *   - Returns PLX_ERR_WORKSPACE, before launching anything, when the partial
+ *     states for these shapes and this split count would need more than
+ *     PLX_NOALLOC_SCRATCH_BYTES (plx_decode_workspace_size tells the need).
+ *   - The first call on a device looks up that device's address of the array
+ *     (cudaGetSymbolAddress, with the device current); make that first call
+ *     before any stream capture.  It allocates nothing, here or later.
+ *   - Every call, on every stream, shares the one array, and the array keeps
+ *     the contents of the last call.  Nothing in it needs to start at zero:
+ *     each call writes every partial it later reads.  Calls that overlap on
+ *     the GPU (different streams without ordering between them) race on the
+ *     array and give undefined results; order them, or use plx_decode with a
+ *     workspace per stream.
+ */
+int plx_decode_noalloc(const void* q, const void* r, const void* kcache, const void* vcache,
+                       const int32_t* seqlens, void* out, float* lse,
+                       int B, int Hq, int Hkv, int S_max, int d, float scale, int num_splits,
+                       void* stream);
 
 /*
  * plx_check_device_status -- synchronises `stream`, then reads and clears the

@@ -307,3 +307,39 @@ extern "C" int plx_selftest_wait_timeout(unsigned long long limit_cycles, void* 
       static_cast<long long>(limit_cycles));
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
+
+// ------------------------------------------------------------------ no-alloc decode
+// Scratch for plx_decode_noalloc: a fixed device array, zero-initialised at
+// module load and shared by every call.  In host code the symbol is only a
+// stand-in; its device address is looked up once per device.
+static __device__ __align__(256) unsigned char g_plx_noalloc_scratch[PLX_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+}  // namespace
+
+extern "C" int plx_decode_noalloc(const void* q, const void* r, const void* kcache, const void* vcache,
+                                  const int32_t* seqlens, void* out, float* lse, int B, int Hq, int Hkv,
+                                  int S_max, int d, float scale, int num_splits, void* stream) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || num_splits < 0) return PLX_ERR_SHAPE;
+  if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
+  if (Hq % Hkv) return PLX_ERR_GQA;
+  const size_t need = plx_decode_workspace_size(B, Hq, Hkv, S_max, d, num_splits);
+  if (need > PLX_NOALLOC_SCRATCH_BYTES) return PLX_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PLX_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_plx_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+        return PLX_ERR_CUDA;
+      g_noalloc_ptr[dev] = ptr;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return plx_decode(q, r, kcache, vcache, seqlens, out, lse, B, Hq, Hkv, S_max, d, scale, num_splits,
+                    scratch, PLX_NOALLOC_SCRATCH_BYTES, stream);
+}

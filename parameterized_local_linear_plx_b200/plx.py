@@ -39,6 +39,8 @@ _lib.plx_decode_workspace_size.restype = _SZ
 _lib.plx_decode_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I]
 _lib.plx_decode.restype = _I
 _lib.plx_decode.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P]
+_lib.plx_decode_noalloc.restype = _I
+_lib.plx_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]
 _lib.plx_check_device_status.restype = _I
 _lib.plx_check_device_status.argtypes = [_P]
 _lib.plx_selftest_wait_timeout.restype = _I
@@ -163,6 +165,36 @@ def plx_decode(q, kcache, vcache, seqlens, r=None, scale=None, num_splits=0, out
                          _stream(stream))
     if st != PLX_OK:
         raise PlxError(st, "plx_decode")
+    return out, lse
+
+
+PLX_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def plx_decode_noalloc(q, kcache, vcache, seqlens, r=None, scale=None, num_splits=0, out=None, lse=None,
+                       return_lse=True, stream=None):
+    """plx_decode without a workspace: for callers that cannot allocate device
+    memory.  The partial states go to the library's fixed device scratch array
+    (PLX_NOALLOC_SCRATCH_BYTES), shared by every call; calls that overlap on
+    the GPU race on it.  out / lse are allocated here only when not given."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(kcache, "kcache", torch.bfloat16, 4)
+    _check(vcache, "vcache", torch.bfloat16, 4)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    if r is not None:
+        _check(r, "r", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    Hkv, S_max = kcache.shape[1], kcache.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    st = _lib.plx_decode_noalloc(_ptr(q), _ptr(r), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(out),
+                                 _ptr(lse), B, Hq, Hkv, S_max, d, float(scale), int(num_splits), _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_decode_noalloc")
     return out, lse
 
 
