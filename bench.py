@@ -79,13 +79,19 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash():
+KERNEL_SOURCES = {
+    "prefill": ("plx_fwd.cuh", "plx_tcgen05.cuh", "plx_ptx.cuh"),
+    "decode": ("plx_decode.cuh", "plx_ptx.cuh"),
+}
+
+
+def source_hash(kernel_key):
+    """Hash of the source files that make up one kernel."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "parameterized_local_linear_plx_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    for name in KERNEL_SOURCES[kernel_key]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -99,7 +105,7 @@ def load_traffic(kernel_key):
     except Exception:
         return None
     e = t.get(kernel_key)
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash(kernel_key):
         return None
     return e.get("dram_bytes_per_launch")
 
