@@ -38,7 +38,7 @@ struct DecodeCfg {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kStages = D == 128 ? 3 : 6;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-  static constexpr int kPartialFloats = 2 * D + 4;             // m, l, c, e, O1[D], O2[D]
+  static constexpr int kPartialFloats = 2 * D + 4;             // m, l, c, pad, O1[D], O2[D]
 };
 
 struct DecodeParams {
@@ -48,7 +48,7 @@ struct DecodeParams {
   __nv_bfloat16* out;       // [B, Hq, D]
   float* lse;               // [B, Hq] or nullptr
   float* ws;                // [B, Hq, splits, 2D+4] or nullptr when splits == 1
-                            //   per row: m (log2 units), l, c, e (sum of unrounded p), O1[D], O2[D]
+                            //   per row: m (log2 units), l, c, pad, O1[D], O2[D]
   int B, Hq, Hkv, S_max, G, n_hgroups, splits, chunk;
   float scale_log2;         // scale * log2(e)
 };
@@ -173,8 +173,9 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
   float o[D / 8][4];
 #pragma unroll
   for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f, c_run = 0.f;  // l, c: this thread's column share
-  float e_run = 0.f;  // sum of unrounded p, for lse only
+  // this thread's column share: l = sum p (fp32, also gives lse), c = sum of
+  // the bf16-rounded p*s the value MMA consumes (so that O2 and c agree)
+  float m_run = -INFINITY, l_run = 0.f, c_run = 0.f;
 
   // ldmatrix row addresses (relative to a K or V tile) for this lane.
   const int mi = lane >> 3, ri = lane & 7;
@@ -231,12 +232,10 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     pa[1] = pack_bf16(ps[0], ps[1]);
     pa[2] = pack_bf16(pr[2], pr[3]);
     pa[3] = pack_bf16(ps[2], ps[3]);
-    // l and c from the rounded values the MMA consumes: effective weights sum to one
-    const float psum = bf16_lo(pa[0]) + bf16_hi(pa[0]) + bf16_lo(pa[2]) + bf16_hi(pa[2]);
-    const float csum = bf16_lo(pa[1]) + bf16_hi(pa[1]) + bf16_lo(pa[3]) + bf16_hi(pa[3]);
+    const float psum = (pr[0] + pr[1]) + (pr[2] + pr[3]);
+    const float csum = (bf16_lo(pa[1]) + bf16_hi(pa[1])) + (bf16_lo(pa[3]) + bf16_hi(pa[3]));
     l_run = l_run * alpha + psum;
     c_run = c_run * alpha + csum;
-    e_run = e_run * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
     m_run = m_new;
     if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
@@ -264,15 +263,13 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
   c_run += __shfl_xor_sync(0xffffffffu, c_run, 1);
   c_run += __shfl_xor_sync(0xffffffffu, c_run, 2);
-  e_run += __shfl_xor_sync(0xffffffffu, e_run, 1);
-  e_run += __shfl_xor_sync(0xffffffffu, e_run, 2);
   asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumerWarps * 32) : "memory");
 
-  constexpr int kRowF = 2 * D + 4;  // m, l, c, e, O1[D], O2[D]
+  constexpr int kRowF = 2 * D + 4;  // m, l, c, pad, O1[D], O2[D]
   float* red = reinterpret_cast<float*>(smem);
   {
     float* mine = red + (warp * 8 + gr) * kRowF;
-    if (qc == 0) { mine[0] = m_run; mine[1] = l_run; mine[2] = c_run; mine[3] = e_run; }
+    if (qc == 0) { mine[0] = m_run; mine[1] = l_run; mine[2] = c_run; mine[3] = 0.f; }
 #pragma unroll
     for (int j = 0; j < D / 8; ++j) {
       const int dd = j * 8 + qc * 2;
@@ -291,14 +288,13 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
     for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, red[(w * 8 + hh) * kRowF]);
     const float Mu = M == -INFINITY ? 0.f : M;
-    float L = 0.f, C = 0.f, E = 0.f, O1 = 0.f, O2 = 0.f;
+    float L = 0.f, C = 0.f, O1 = 0.f, O2 = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecConsumerWarps; ++w) {
       const float* rw = red + (w * 8 + hh) * kRowF;
       const float beta = ex2(rw[0] - Mu);
       L += beta * rw[1];
       C += beta * rw[2];
-      E += beta * rw[3];
       O1 += beta * rw[4 + dd];
       O2 += beta * rw[4 + D + dd];
     }
@@ -311,10 +307,10 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
         res = o1 - (O2 * inv - (C * inv) * o1);
       }
       p.out[row * D + dd] = __float2bfloat16(res);
-      if (dd == 0 && p.lse) p.lse[row] = E > 0.f ? (M + __log2f(E)) * kLn2 : -INFINITY;
+      if (dd == 0 && p.lse) p.lse[row] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
     } else {
       float* ws = p.ws + (row * p.splits + split) * Cfg::kPartialFloats;
-      if (dd == 0) { ws[0] = M; ws[1] = L; ws[2] = C; ws[3] = E; }
+      if (dd == 0) { ws[0] = M; ws[1] = L; ws[2] = C; ws[3] = 0.f; }
       ws[4 + dd] = O1;
       ws[4 + D + dd] = O2;
     }
@@ -333,13 +329,12 @@ plx_decode_combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restric
   float M = -INFINITY;
   for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldg(base + s * PF));
   const float Mu = M == -INFINITY ? 0.f : M;
-  float L = 0.f, C = 0.f, E = 0.f, O1 = 0.f, O2 = 0.f;
+  float L = 0.f, C = 0.f, O1 = 0.f, O2 = 0.f;
   for (int s = 0; s < splits; ++s) {
     const float* ps = base + s * PF;
     const float beta = ex2(__ldg(ps) - Mu);
     L += beta * __ldg(ps + 1);
     C += beta * __ldg(ps + 2);
-    E += beta * __ldg(ps + 3);
     O1 += beta * __ldg(ps + 4 + dd);
     O2 += beta * __ldg(ps + 4 + D + dd);
   }
@@ -350,7 +345,7 @@ plx_decode_combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restric
     res = o1 - (O2 * inv - (C * inv) * o1);
   }
   out[row * D + dd] = __float2bfloat16(res);
-  if (dd == 0 && lse) lse[row] = E > 0.f ? (M + __log2f(E)) * kLn2 : -INFINITY;
+  if (dd == 0 && lse) lse[row] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
 }
 
 }  // namespace plx

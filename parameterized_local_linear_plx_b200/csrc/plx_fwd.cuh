@@ -26,7 +26,8 @@
 //     warp 8: TMA loads (Q/R once, K/V ring); warp 9: TMEM allocation and
 //     the single thread that issues every MMA.  The MMA order
 //     PV0(j), S0(j+1), PV1(j), S1(j+1) lets each softmax overlap the other
-//     tile's MMAs.
+//     tile's MMAs, and each softmax hands over P in two 64-key halves so the
+//     first half of its value MMA runs while it computes the second.
 //   * The running max is updated lazily: O is rescaled in tensor memory only
 //     when a row max grows by more than 2^8 (so p <= 256 before the final
 //     normalisation, which bf16 P holds without loss of relative precision).
@@ -86,8 +87,8 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   uint64_t* v_full = k_empty + NS;      // [NS]
   uint64_t* v_empty = v_full + NS;      // [NS]
   uint64_t* s_full = v_empty + NS;      // [2]
-  uint64_t* p_ready = s_full + 2;       // [2]
-  uint64_t* o_done = p_ready + 2;       // [2]
+  uint64_t* p_ready = s_full + 2;       // [2 tiles][2 halves]
+  uint64_t* o_done = p_ready + 4;       // [2]
   uint64_t* fin = o_done + 2;           // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
 
@@ -111,9 +112,9 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   if (threadIdx.x == 0) {
     // every barrier takes one arrival (+ TMA bytes / tcgen05.commit), except
     // p_ready, which all 128 threads of a softmax warpgroup arrive on
-    for (int i = 0; i < 2 + 4 * NS + 7; ++i) {
+    for (int i = 0; i < 2 + 4 * NS + 9; ++i) {
       uint64_t* bp = &bars[i];
-      mbar_init(smem_u32(bp), (bp == &p_ready[0] || bp == &p_ready[1]) ? 128u : 1u);
+      mbar_init(smem_u32(bp), (bp >= &p_ready[0] && bp <= &p_ready[3]) ? 128u : 1u);
     }
     fence_barrier_init();
   }
@@ -215,13 +216,17 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         }
         tc::commit(smem_u32(&s_full[t]));
       };
-      auto issue_pv = [&](int t, int j) {
+      // value product for keys 64h..64h+63 of tile t once that half of P is ready
+      auto issue_pv = [&](int t, int j, int h) -> bool {
+        if (!mbar_wait(smem_u32(&p_ready[2 * t + h]), j & 1, kErrFwdMma)) return false;
+        tc::fence_after_sync();
         const uint32_t b0 = v_base + (j % NS) * Cfg::kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < kFwdBN / 16; ++kk)
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
           tc::mma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
                      tc::smem_desc_sw128(b0 + kk * 2048, Cfg::kBlock, 1024), idesc_o,
                      (j > 0 || kk > 0) ? 1u : 0u);
+        return true;
       };
 
       ok = mbar_wait(smem_u32(&qr_full[0]), 0, kErrFwdMma) && mbar_wait(smem_u32(&qr_full[1]), 0, kErrFwdMma) &&
@@ -234,19 +239,15 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       }
       for (int j = 0; j < nkv && ok; ++j) {
         const int s = j % NS;
-        if (!mbar_wait(smem_u32(&v_full[s]), (j / NS) & 1, kErrFwdMma) ||
-            !mbar_wait(smem_u32(&p_ready[0]), j & 1, kErrFwdMma)) { ok = false; break; }
-        tc::fence_after_sync();
-        issue_pv(0, j);
+        if (!mbar_wait(smem_u32(&v_full[s]), (j / NS) & 1, kErrFwdMma) || !issue_pv(0, j, 0) ||
+            !issue_pv(0, j, 1)) { ok = false; break; }
         const bool more = j + 1 < nkv;
         if (more) {
           if (!mbar_wait(smem_u32(&k_full[(j + 1) % NS]), ((j + 1) / NS) & 1, kErrFwdMma)) { ok = false; break; }
           tc::fence_after_sync();
           issue_s(0, j + 1);
         }
-        if (!mbar_wait(smem_u32(&p_ready[1]), j & 1, kErrFwdMma)) { ok = false; break; }
-        tc::fence_after_sync();
-        issue_pv(1, j);
+        if (!issue_pv(1, j, 0) || !issue_pv(1, j, 1)) { ok = false; break; }
         tc::commit(smem_u32(&v_empty[s]));
         if (more) {
           issue_s(1, j + 1);
@@ -275,8 +276,9 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const int q_lo = q0 + 16 * wq + (lane >> 2);
     const int q_hi = q_lo + 8;
     float m_lo = -INFINITY, m_hi = -INFINITY;
-    float l_lo = 0.f, l_hi = 0.f, c_lo = 0.f, c_hi = 0.f;  // this thread's column share
-    float e_lo = 0.f, e_hi = 0.f;  // sum of unrounded p, for lse only
+    // this thread's column share: l = sum p (fp32, also gives lse), c = sum of
+    // the bf16-rounded p*s the value MMA consumes (so that O2 and c agree)
+    float l_lo = 0.f, l_hi = 0.f, c_lo = 0.f, c_hi = 0.f;
 
     for (int j = 0; j < nkv; ++j) {
       // warp-uniform: the .sync.aligned tensor-memory accesses below need every lane
@@ -323,7 +325,6 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         const float al_lo = mn_lo == -INFINITY ? 1.f : ex2(m_lo - mn_lo);
         const float al_hi = mn_hi == -INFINITY ? 1.f : ex2(m_hi - mn_hi);
         l_lo *= al_lo; c_lo *= al_lo; l_hi *= al_hi; c_hi *= al_hi;
-        e_lo *= al_lo; e_hi *= al_hi;
         m_lo = mn_lo; m_hi = mn_hi;
         if (j > 0) {
           // O rows of this warp: O1 at the a lanes, O2 at the s lanes; PV(j-1)
@@ -347,41 +348,47 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       }
       const float mu_lo = m_lo == -INFINITY ? 0.f : m_lo;
       const float mu_hi = m_hi == -INFINITY ? 0.f : m_hi;
-      float xl = 0.f, xh = 0.f;
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float pv = ex2(fmaf(__uint_as_float(ra[i]), p.scale_log2, (i & 2) ? -mu_hi : -mu_lo));
-        const float sv = HAS_R ? __uint_as_float(rs[i]) : 0.f;
-        if (i & 2) xh += pv; else xl += pv;
-        ra[i] = __float_as_uint(pv);
-        rs[i] = __float_as_uint(pv * sv);
-      }
-      e_lo += xl; e_hi += xh;
-      // l and c are summed from the bf16-rounded P and P*S that the value MMA
-      // consumes, so the output's effective weights sum to exactly one.
-      float sl = 0.f, sh = 0.f, cl = 0.f, ch_ = 0.f;
+      // p = 2^(a*scale*log2e - m) with the scale folded into one packed FMA per
+      // row pair; l from fp32 p, c from the rounded p*s.
+      const uint64_t sl2 = f2(p.scale_log2, p.scale_log2);
+      const uint64_t nmu_lo = f2(-mu_lo, -mu_lo), nmu_hi = f2(-mu_hi, -mu_hi);
+      uint64_t ls_lo = 0, ls_hi = 0, cs_lo = 0, cs_hi = 0;  // packed partial sums (0 bits = +0.0f)
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t pp[16], pq[16];
 #pragma unroll
         for (int gg = 0; gg < 8; ++gg) {
           const int i = 32 * hf + 4 * gg;
-          pp[2 * gg] = pack_bf16(__uint_as_float(ra[i]), __uint_as_float(ra[i + 1]));
-          pp[2 * gg + 1] = pack_bf16(__uint_as_float(ra[i + 2]), __uint_as_float(ra[i + 3]));
-          pq[2 * gg] = pack_bf16(__uint_as_float(rs[i]), __uint_as_float(rs[i + 1]));
-          pq[2 * gg + 1] = pack_bf16(__uint_as_float(rs[i + 2]), __uint_as_float(rs[i + 3]));
-          sl += bf16_lo(pp[2 * gg]) + bf16_hi(pp[2 * gg]);
-          sh += bf16_lo(pp[2 * gg + 1]) + bf16_hi(pp[2 * gg + 1]);
-          cl += bf16_lo(pq[2 * gg]) + bf16_hi(pq[2 * gg]);
-          ch_ += bf16_lo(pq[2 * gg + 1]) + bf16_hi(pq[2 * gg + 1]);
+          const uint64_t xl = f2_fma(f2(__uint_as_float(ra[i]), __uint_as_float(ra[i + 1])), sl2, nmu_lo);
+          const uint64_t xh = f2_fma(f2(__uint_as_float(ra[i + 2]), __uint_as_float(ra[i + 3])), sl2, nmu_hi);
+          const uint64_t pl = f2(ex2(f2_lo(xl)), ex2(f2_hi(xl)));
+          const uint64_t ph = f2(ex2(f2_lo(xh)), ex2(f2_hi(xh)));
+          ls_lo = f2_add(ls_lo, pl);
+          ls_hi = f2_add(ls_hi, ph);
+          pp[2 * gg] = pack_bf16(f2_lo(pl), f2_hi(pl));
+          pp[2 * gg + 1] = pack_bf16(f2_lo(ph), f2_hi(ph));
+          if (HAS_R) {
+            const uint64_t sl = f2_mul(pl, f2(__uint_as_float(rs[i]), __uint_as_float(rs[i + 1])));
+            const uint64_t sh = f2_mul(ph, f2(__uint_as_float(rs[i + 2]), __uint_as_float(rs[i + 3])));
+            const uint32_t wl = pack_bf16(f2_lo(sl), f2_hi(sl));
+            const uint32_t wh = pack_bf16(f2_lo(sh), f2_hi(sh));
+            pq[2 * gg] = wl;
+            pq[2 * gg + 1] = wh;
+            cs_lo = f2_add(cs_lo, f2(bf16_lo(wl), bf16_hi(wl)));
+            cs_hi = f2_add(cs_hi, f2(bf16_lo(wh), bf16_hi(wh)));
+          }
         }
         tc::st_16x128b_x8(ta + 32 * hf, pp);
-        tc::st_16x128b_x8(ts + 32 * hf, pq);
+        // rho = 0: the probe rows of S are exact zeros, which read as bf16 zeros
+        if (HAS_R) tc::st_16x128b_x8(ts + 32 * hf, pq);
+        tc::wait_st();
+        tc::fence_before_sync();
+        mbar_arrive(smem_u32(&p_ready[2 * t + hf]));
       }
-      l_lo += sl; l_hi += sh; c_lo += cl; c_hi += ch_;
-      tc::wait_st();
-      tc::fence_before_sync();
-      mbar_arrive(smem_u32(&p_ready[t]));
+      l_lo += f2_lo(ls_lo) + f2_hi(ls_lo);
+      l_hi += f2_lo(ls_hi) + f2_hi(ls_hi);
+      c_lo += f2_lo(cs_lo) + f2_hi(cs_lo);
+      c_hi += f2_lo(cs_hi) + f2_hi(cs_hi);
     }
 
     const bool fin_ok = ok && mbar_wait(smem_u32(&o_done[t]), 0, kErrFwdSoftmax);
@@ -395,10 +402,6 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       c_lo += __shfl_xor_sync(0xffffffffu, c_lo, 2);
       c_hi += __shfl_xor_sync(0xffffffffu, c_hi, 1);
       c_hi += __shfl_xor_sync(0xffffffffu, c_hi, 2);
-      e_lo += __shfl_xor_sync(0xffffffffu, e_lo, 1);
-      e_lo += __shfl_xor_sync(0xffffffffu, e_lo, 2);
-      e_hi += __shfl_xor_sync(0xffffffffu, e_hi, 1);
-      e_hi += __shfl_xor_sync(0xffffffffu, e_hi, 2);
       const float inv_lo = l_lo > 0.f ? 1.f / l_lo : 0.f;
       const float inv_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
       const float sb_lo = c_lo * inv_lo, sb_hi = c_hi * inv_hi;  // s_bar = c / l
@@ -428,8 +431,8 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         }
       }
       if (p.lse && c4 == 0) {
-        if (q_lo < p.N) p.lse[plane * p.N + q_lo] = e_lo > 0.f ? (m_lo + __log2f(e_lo)) * kLn2 : -INFINITY;
-        if (q_hi < p.N) p.lse[plane * p.N + q_hi] = e_hi > 0.f ? (m_hi + __log2f(e_hi)) * kLn2 : -INFINITY;
+        if (q_lo < p.N) p.lse[plane * p.N + q_lo] = l_lo > 0.f ? (m_lo + __log2f(l_lo)) * kLn2 : -INFINITY;
+        if (q_hi < p.N) p.lse[plane * p.N + q_hi] = l_hi > 0.f ? (m_hi + __log2f(l_hi)) * kLn2 : -INFINITY;
       }
     }
   }
