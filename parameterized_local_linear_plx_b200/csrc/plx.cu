@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/plx.h"
@@ -23,6 +24,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // ---------------------------------------------------------------- device checks
 int g_arch_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 not sm_100
+int g_sm_count[kMaxDevices];
 std::mutex g_mu;
 
 int check_arch(int* dev_out) {
@@ -35,6 +37,10 @@ int check_arch(int* dev_out) {
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
       return PLX_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+      return PLX_ERR_CUDA;
+    g_sm_count[dev] = sms;
     g_arch_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
   }
   return g_arch_ok[dev] == 1 ? PLX_OK : PLX_ERR_ARCH;
@@ -134,14 +140,14 @@ int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const plx::Decod
 
 template <int D, bool HAS_R>
 int launch_fwd(const CUtensorMap& qm, const CUtensorMap& rm, const CUtensorMap& km, const CUtensorMap& vm,
-               const plx::FwdParams& p, unsigned grid, cudaStream_t st) {
+               const CUtensorMap& om, const plx::FwdParams& p, unsigned grid, cudaStream_t st) {
   using Cfg = plx::FwdCfg<D>;
   static bool done[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
   auto kern = plx::plx_fwd_kernel<D, HAS_R>;
   if (ensure_smem(kern, Cfg::kSmemBytes, &done[dev]) != PLX_OK) return PLX_ERR_CUDA;
-  kern<<<grid, plx::kFwdThreads, Cfg::kSmemBytes, st>>>(qm, rm, km, vm, p);
+  kern<<<grid, plx::kFwdThreads, Cfg::kSmemBytes, st>>>(qm, rm, km, vm, om, p);
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
@@ -187,10 +193,10 @@ int plx_fwd(const void* q, const void* k, const void* v, const void* r, void* ou
   if (rc != PLX_OK) return rc;
   if ((rc = get_encoder()) != PLX_OK) return rc;
 
-  CUtensorMap qm, rm, km, vm;
+  CUtensorMap qm, rm, km, vm, om;
   const long long pq = static_cast<long long>(B) * Hq, pkv = static_cast<long long>(B) * Hkv;
   if (make_map_3d(&qm, q, d, N, pq, 16) != PLX_OK || make_map_3d(&km, k, d, N, pkv, plx::kFwdBN) != PLX_OK ||
-      make_map_3d(&vm, v, d, N, pkv, plx::kFwdBN) != PLX_OK)
+      make_map_3d(&vm, v, d, N, pkv, plx::kFwdBN) != PLX_OK || make_map_3d(&om, out, d, N, pq, 16) != PLX_OK)
     return PLX_ERR_CUDA;
   if (r) {
     if (make_map_3d(&rm, r, d, N, pq, 16) != PLX_OK) return PLX_ERR_CUDA;
@@ -202,12 +208,15 @@ int plx_fwd(const void* q, const void* k, const void* v, const void* r, void* ou
   p.lse = lse;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.G = G;
   p.pair_heads = pair_heads; p.n_pairs = n_pairs; p.n_qblocks = n_qblocks;
+  p.num_units = static_cast<int>(grid);
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * plx::kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const unsigned g = static_cast<unsigned>(grid);
-  if (d == 128) return r ? launch_fwd<128, true>(qm, rm, km, vm, p, g, st) : launch_fwd<128, false>(qm, rm, km, vm, p, g, st);
-  return r ? launch_fwd<64, true>(qm, rm, km, vm, p, g, st) : launch_fwd<64, false>(qm, rm, km, vm, p, g, st);
+  // persistent: one CTA per SM (the kernel's shared memory allows no more)
+  const unsigned g = static_cast<unsigned>(std::min<long long>(grid, g_sm_count[dev]));
+  if (d == 128)
+    return r ? launch_fwd<128, true>(qm, rm, km, vm, om, p, g, st) : launch_fwd<128, false>(qm, rm, km, vm, om, p, g, st);
+  return r ? launch_fwd<64, true>(qm, rm, km, vm, om, p, g, st) : launch_fwd<64, false>(qm, rm, km, vm, om, p, g, st);
 }
 
 int plx_decode_num_splits(int B, int Hq, int Hkv, int S_max, int d) {

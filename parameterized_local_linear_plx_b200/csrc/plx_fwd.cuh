@@ -24,10 +24,20 @@
 //     of one head.  Tensor memory: [S0 | O0 | S1 | O1], 128 columns each.
 //   * Warps 0-3 and 4-7: softmax + epilogue of tile 0 and tile 1;
 //     warp 8: TMA loads (Q/R once, K/V ring); warp 9: TMEM allocation and
-//     the single thread that issues every MMA.  The MMA order
-//     PV0(j), S0(j+1), PV1(j), S1(j+1) lets each softmax overlap the other
-//     tile's MMAs, and each softmax hands over P in two 64-key halves so the
-//     first half of its value MMA runs while it computes the second.
+//     the single thread that issues every MMA, in the order
+//     PV0(j), S0(j+1), PV1(j), S1(j+1): each tile's next scores come right
+//     after its value MMA, so each softmax overlaps the other tile's MMAs.
+//     One M=128 N=128 MMA takes ~64 tensor cycles and a thread needs a large
+//     part of that to issue one, so descriptors are precomputed and each MMA
+//     only adds a constant to the start-address field.  Each softmax hands
+//     over P in two 64-key halves so the first half of its value MMA runs
+//     while it computes the second.
+//   * Persistent: one CTA per SM walks the work units (tile pairs, longest
+//     causal rows first) in steps of the grid size.  The K/V ring and every
+//     barrier phase carry on across units; the load warp fetches the next
+//     unit's Q/R as soon as the last score MMA of the current unit has been
+//     issued, the next unit's score MMAs overlap this unit's epilogue, and
+//     its first value MMA waits only until the epilogue has read O.
 //   * The running max is updated lazily: O is rescaled in tensor memory only
 //     when a row max grows by more than 2^8 (so p <= 256 before the final
 //     normalisation, which bf16 P holds without loss of relative precision).
@@ -55,7 +65,9 @@ struct FwdCfg {
   static constexpr int kOffQR = 0;
   static constexpr int kOffK = 2 * kQRBytes;
   static constexpr int kOffV = kOffK + kStages * kKVBytes;
-  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+  static constexpr int kOffOut = kOffV + kStages * kKVBytes;     // bf16 output staging for TMA stores
+  static constexpr int kOutWarpBytes = kCB * 16 * 128;              // 16 rows per softmax warp
+  static constexpr int kOffBar = kOffOut + 8 * kOutWarpBytes;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
   static constexpr uint32_t kTmemCols = 512;
 };
@@ -67,6 +79,7 @@ struct FwdParams {
   int pair_heads;      // 1: tiles are heads (2p, 2p+1) at rows 64*qb; 0: rows 128*qb (+64) of head p
   int n_pairs;         // Hq / 2 or Hq
   int n_qblocks;       // ceil(N/64) or ceil(N/128)
+  int num_units;       // B * n_pairs * n_qblocks
   int causal;
   float scale_log2;    // scale * log2(e)
 };
@@ -75,46 +88,57 @@ template <int D, bool HAS_R>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap rmap,
                const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-               const FwdParams p) {
+               const __grid_constant__ CUtensorMap omap, const FwdParams p) {
   using Cfg = FwdCfg<D>;
   constexpr int NS = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
   uint64_t* qr_full = bars;             // [2]
-  uint64_t* k_full = bars + 2;          // [NS]
+  uint64_t* qr_empty = bars + 2;        // [1] last score MMA of a unit issued and done
+  uint64_t* k_full = bars + 3;          // [NS]
   uint64_t* k_empty = k_full + NS;      // [NS]
   uint64_t* v_full = k_empty + NS;      // [NS]
   uint64_t* v_empty = v_full + NS;      // [NS]
   uint64_t* s_full = v_empty + NS;      // [2]
   uint64_t* p_ready = s_full + 2;       // [2 tiles][2 halves]
   uint64_t* o_done = p_ready + 4;       // [2]
-  uint64_t* fin = o_done + 2;           // [1]
+  uint64_t* o_free = o_done + 2;        // [2] epilogue has read O (128 arrivals)
+  uint64_t* fin = o_free + 2;           // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: longest causal rows first
-  const int per = p.B * p.n_pairs;
-  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) / per;
-  const int rem = static_cast<int>(blockIdx.x) % per;
-  const int b = rem / p.n_pairs;
-  const int hp = rem % p.n_pairs;
-  // tile t in {0, 1}: query head head_of(t), first query row row0_of(t)
-  auto head_of = [&](int t) { return p.pair_heads ? 2 * hp + t : hp; };
-  auto row0_of = [&](int t) { return p.pair_heads ? qb * kFwdBM : (2 * qb + t) * kFwdBM; };
-  const int g = head_of(0) / p.G;
-  const int qmax = min(p.N - 1, row0_of(1) + kFwdBM - 1);
-  const int nkv_all = (p.N + kFwdBN - 1) / kFwdBN;
-  const int nkv = p.causal ? min(nkv_all, qmax / kFwdBN + 1) : nkv_all;
+  // ---- work units: index u -> (b, head pair / head, query block), longest
+  // causal rows first; CTA c takes u = c, c + gridDim.x, ...
+  struct Unit {
+    int b, hp, qb, nkv;
+  };
+  auto unit_of = [&](int u) {
+    Unit w;
+    const int per = p.B * p.n_pairs;
+    w.qb = p.n_qblocks - 1 - u / per;
+    const int rem = u % per;
+    w.b = rem / p.n_pairs;
+    w.hp = rem % p.n_pairs;
+    const int last_row = p.pair_heads ? w.qb * kFwdBM + kFwdBM - 1 : (2 * w.qb + 2) * kFwdBM - 1;
+    const int qmax = min(p.N - 1, last_row);
+    const int nkv_all = (p.N + kFwdBN - 1) / kFwdBN;
+    w.nkv = p.causal ? min(nkv_all, qmax / kFwdBN + 1) : nkv_all;
+    return w;
+  };
+  // tile t in {0, 1} of a unit: query head and first query row
+  auto head_of = [&](const Unit& w, int t) { return p.pair_heads ? 2 * w.hp + t : w.hp; };
+  auto row0_of = [&](const Unit& w, int t) { return p.pair_heads ? w.qb * kFwdBM : (2 * w.qb + t) * kFwdBM; };
 
   if (threadIdx.x == 0) {
-    // every barrier takes one arrival (+ TMA bytes / tcgen05.commit), except
-    // p_ready, which all 128 threads of a softmax warpgroup arrive on
-    for (int i = 0; i < 2 + 4 * NS + 9; ++i) {
+    // arrivals per phase: p_ready and o_free get all 128 threads of a
+    // softmax warpgroup; every other barrier one arrival (+ TMA bytes / a commit)
+    for (int i = 0; i < 3 + 4 * NS + 11; ++i) {
       uint64_t* bp = &bars[i];
-      mbar_init(smem_u32(bp), (bp >= &p_ready[0] && bp <= &p_ready[3]) ? 128u : 1u);
+      const bool wg = (bp >= &p_ready[0] && bp <= &p_ready[3]) || bp == &o_free[0] || bp == &o_free[1];
+      mbar_init(smem_u32(bp), wg ? 128u : 1u);
     }
     fence_barrier_init();
   }
@@ -149,47 +173,56 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       if (HAS_R) tma_prefetch_desc(&rmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      for (int t = 0; t < 2; ++t) {
-        const uint32_t fb = smem_u32(&qr_full[t]);
-        mbar_arrive_expect_tx(fb, HAS_R ? Cfg::kQRBytes : Cfg::kQRBytes / 2);
-        const uint32_t base = smem_u32(smem + Cfg::kOffQR + t * Cfg::kQRBytes);
-        const int plane = b * p.Hq + head_of(t);
-#pragma unroll
-        for (int w = 0; w < 4; ++w)
-#pragma unroll
-          for (int cb = 0; cb < Cfg::kCB; ++cb) {
-            const uint32_t dst = base + cb * Cfg::kBlock + (32 * w) * 128;
-            tma_load_3d(&qmap, dst, fb, cb * 64, row0_of(t) + 16 * w, plane);
-            if (HAS_R) tma_load_3d(&rmap, dst + 16 * 128, fb, cb * 64, row0_of(t) + 16 * w, plane);
-          }
-      }
-      const int plane_kv = b * p.Hkv + g;
+      int kv = 0;        // K/V tiles issued so far: ring stage kv % NS, phase (kv / NS) & 1
+      int n_unit = 0;    // units whose Q/R were issued
       int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int s = j % NS;
-        if (j >= NS && !mbar_wait(smem_u32(&k_empty[s]), ((j / NS) - 1) & 1, kErrFwdLoad)) { ok = false; break; }
-        {
-          const uint32_t fb = smem_u32(&k_full[s]);
-          mbar_arrive_expect_tx(fb, Cfg::kKVBytes);
-          const uint32_t dst = smem_u32(smem + Cfg::kOffK + s * Cfg::kKVBytes);
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++n_unit) {
+        const Unit w = unit_of(u);
+        // the previous unit's last score MMA must have read Q/R
+        if (n_unit > 0 && !mbar_wait(smem_u32(qr_empty), (n_unit - 1) & 1, kErrFwdLoad)) { ok = false; break; }
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t fb = smem_u32(&qr_full[t]);
+          mbar_arrive_expect_tx(fb, HAS_R ? Cfg::kQRBytes : Cfg::kQRBytes / 2);
+          const uint32_t base = smem_u32(smem + Cfg::kOffQR + t * Cfg::kQRBytes);
+          const int plane = w.b * p.Hq + head_of(w, t);
+          const int row0 = row0_of(w, t);
 #pragma unroll
-          for (int cb = 0; cb < Cfg::kCB; ++cb)
-            tma_load_3d(&kmap, dst + cb * Cfg::kBlock, fb, cb * 64, j * kFwdBN, plane_kv);
-          issued_k = j + 1;
+          for (int wq = 0; wq < 4; ++wq)
+#pragma unroll
+            for (int cb = 0; cb < Cfg::kCB; ++cb) {
+              const uint32_t dst = base + cb * Cfg::kBlock + (32 * wq) * 128;
+              tma_load_3d(&qmap, dst, fb, cb * 64, row0 + 16 * wq, plane);
+              if (HAS_R) tma_load_3d(&rmap, dst + 16 * 128, fb, cb * 64, row0 + 16 * wq, plane);
+            }
         }
-        if (j >= NS && !mbar_wait(smem_u32(&v_empty[s]), ((j / NS) - 1) & 1, kErrFwdLoad)) { ok = false; break; }
-        {
-          const uint32_t fb = smem_u32(&v_full[s]);
-          mbar_arrive_expect_tx(fb, Cfg::kKVBytes);
-          const uint32_t dst = smem_u32(smem + Cfg::kOffV + s * Cfg::kKVBytes);
+        const int plane_kv = w.b * p.Hkv + head_of(w, 0) / p.G;
+        for (int j = 0; j < w.nkv; ++j, ++kv) {
+          const int s = kv % NS;
+          if (kv >= NS && !mbar_wait(smem_u32(&k_empty[s]), ((kv / NS) - 1) & 1, kErrFwdLoad)) { ok = false; break; }
+          {
+            const uint32_t fb = smem_u32(&k_full[s]);
+            mbar_arrive_expect_tx(fb, Cfg::kKVBytes);
+            const uint32_t dst = smem_u32(smem + Cfg::kOffK + s * Cfg::kKVBytes);
 #pragma unroll
-          for (int cb = 0; cb < Cfg::kCB; ++cb)
-            tma_load_3d(&vmap, dst + cb * Cfg::kBlock, fb, cb * 64, j * kFwdBN, plane_kv);
-          issued_v = j + 1;
+            for (int cb = 0; cb < Cfg::kCB; ++cb)
+              tma_load_3d(&kmap, dst + cb * Cfg::kBlock, fb, cb * 64, j * kFwdBN, plane_kv);
+            issued_k = kv + 1;
+          }
+          if (kv >= NS && !mbar_wait(smem_u32(&v_empty[s]), ((kv / NS) - 1) & 1, kErrFwdLoad)) { ok = false; break; }
+          {
+            const uint32_t fb = smem_u32(&v_full[s]);
+            mbar_arrive_expect_tx(fb, Cfg::kKVBytes);
+            const uint32_t dst = smem_u32(smem + Cfg::kOffV + s * Cfg::kKVBytes);
+#pragma unroll
+            for (int cb = 0; cb < Cfg::kCB; ++cb)
+              tma_load_3d(&vmap, dst + cb * Cfg::kBlock, fb, cb * 64, j * kFwdBN, plane_kv);
+            issued_v = kv + 1;
+          }
         }
       }
       if (!ok) {  // let every issued load land before the CTA can exit
-        for (int t = 0; t < 2; ++t) mbar_wait(smem_u32(&qr_full[t]), 0, kErrFwdDrain);
+        if (n_unit > 0)
+          for (int t = 0; t < 2; ++t) mbar_wait(smem_u32(&qr_full[t]), (n_unit - 1) & 1, kErrFwdDrain);
         for (int j = max(0, issued_k - NS); j < issued_k; ++j)
           mbar_wait(smem_u32(&k_full[j % NS]), (j / NS) & 1, kErrFwdDrain);
         for (int j = max(0, issued_v - NS); j < issued_v; ++j)
@@ -201,61 +234,82 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     if (lane == 0) {
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kFwdBN, 0, 0);  // [Q;R] x K^T, both K-major
       constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, 0, 1);       // [P;PS] x V, V MN-major
-      const uint32_t qr_base = smem_u32(smem + Cfg::kOffQR);
-      const uint32_t k_base = smem_u32(smem + Cfg::kOffK);
-      const uint32_t v_base = smem_u32(smem + Cfg::kOffV);
+      constexpr uint64_t kStageStep = Cfg::kKVBytes >> 4;                  // descriptor units
+      constexpr uint64_t kTileStep = Cfg::kQRBytes >> 4;
+      // base descriptors; each MMA adds a constant to the start-address field
+      const uint64_t d_qr = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffQR), 16, 1024);
+      const uint64_t d_k = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffK), 16, 1024);
+      const uint64_t d_v = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffV), Cfg::kBlock, 1024);
 
-      auto issue_s = [&](int t, int j) {
-        const uint32_t a0 = qr_base + t * Cfg::kQRBytes;
-        const uint32_t b0 = k_base + (j % NS) * Cfg::kKVBytes;
+      // S_t = [Q;R]_t K^T of the K/V tile in ring stage s, into tile t's score columns
+      auto issue_s = [&](int t, int s) {
+        const uint64_t da = d_qr + t * kTileStep;
+        const uint64_t db = d_k + s * kStageStep;
+        const uint32_t dst = tmem + col_s(t);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * Cfg::kBlock + (ks & 3) * 32;
-          tc::mma_ss(tmem + col_s(t), tc::smem_desc_sw128(a0 + off, 16, 1024),
-                     tc::smem_desc_sw128(b0 + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+          const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
+          tc::mma_ss(dst, da + koff, db + koff, idesc_s, ks > 0 ? 1u : 0u);
         }
         tc::commit(smem_u32(&s_full[t]));
       };
-      // value product for keys 64h..64h+63 of tile t once that half of P is ready
-      auto issue_pv = [&](int t, int j, int h) -> bool {
-        if (!mbar_wait(smem_u32(&p_ready[2 * t + h]), j & 1, kErrFwdMma)) return false;
+      // O_t (+)= [P;PS]_t V for keys 64h..64h+63 of global tile g, once that half of P is ready
+      auto issue_pv = [&](int t, int g, int h, bool first) -> bool {
+        if (!mbar_wait(smem_u32(&p_ready[2 * t + h]), g & 1, kErrFwdMma)) return false;
         tc::fence_after_sync();
-        const uint32_t b0 = v_base + (j % NS) * Cfg::kKVBytes;
+        const uint64_t db = d_v + (g % NS) * kStageStep;
+        const uint32_t a = tmem + col_s(t), dst = tmem + col_o(t);
 #pragma unroll
-        for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
-          tc::mma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
-                     tc::smem_desc_sw128(b0 + kk * 2048, Cfg::kBlock, 1024), idesc_o,
-                     (j > 0 || kk > 0) ? 1u : 0u);
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * h + k4;
+          tc::mma_ts(dst, a + kk * 8, db + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
+                     (!first || kk > 0) ? 1u : 0u);
+        }
         return true;
       };
 
-      ok = mbar_wait(smem_u32(&qr_full[0]), 0, kErrFwdMma) && mbar_wait(smem_u32(&qr_full[1]), 0, kErrFwdMma) &&
-           mbar_wait(smem_u32(&k_full[0]), 0, kErrFwdMma);
-      if (ok) {
+      int kv = 0;       // global K/V tile index of the current unit's first tile
+      int n_unit = 0;
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++n_unit) {
+        const Unit w = unit_of(u);
+        const uint32_t uph = n_unit & 1;
+        ok = mbar_wait(smem_u32(&qr_full[0]), uph, kErrFwdMma) && mbar_wait(smem_u32(&qr_full[1]), uph, kErrFwdMma) &&
+             mbar_wait(smem_u32(&k_full[kv % NS]), (kv / NS) & 1, kErrFwdMma);
+        if (!ok) break;
         tc::fence_after_sync();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        tc::commit(smem_u32(&k_empty[0]));
-      }
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int s = j % NS;
-        if (!mbar_wait(smem_u32(&v_full[s]), (j / NS) & 1, kErrFwdMma) || !issue_pv(0, j, 0) ||
-            !issue_pv(0, j, 1)) { ok = false; break; }
-        const bool more = j + 1 < nkv;
-        if (more) {
-          if (!mbar_wait(smem_u32(&k_full[(j + 1) % NS]), ((j + 1) / NS) & 1, kErrFwdMma)) { ok = false; break; }
-          tc::fence_after_sync();
-          issue_s(0, j + 1);
+        // The previous unit's PV(last) precede these in issue order, so they
+        // overwrite its last P only after it was read.
+        issue_s(0, kv % NS);
+        issue_s(1, kv % NS);
+        tc::commit(smem_u32(&k_empty[kv % NS]));
+        if (w.nkv == 1) tc::commit(smem_u32(qr_empty));
+        for (int j = 0; j < w.nkv && ok; ++j) {
+          const int g = kv + j;
+          const int s = g % NS;
+          const bool more = j + 1 < w.nkv;
+          if (!mbar_wait(smem_u32(&v_full[s]), (g / NS) & 1, kErrFwdMma)) { ok = false; break; }
+          // a unit's first PV overwrites O: the previous unit's epilogue must have read it
+          if (j == 0 && n_unit > 0 && !mbar_wait(smem_u32(&o_free[0]), (n_unit - 1) & 1, kErrFwdMma)) { ok = false; break; }
+          if (!issue_pv(0, g, 0, j == 0) || !issue_pv(0, g, 1, j == 0)) { ok = false; break; }
+          if (more) {
+            // S0 of the next tile follows PV0 in issue order: it overwrites P0 only after it was read
+            if (!mbar_wait(smem_u32(&k_full[(g + 1) % NS]), ((g + 1) / NS) & 1, kErrFwdMma)) { ok = false; break; }
+            tc::fence_after_sync();
+            issue_s(0, (g + 1) % NS);
+          }
+          if (j == 0 && n_unit > 0 && !mbar_wait(smem_u32(&o_free[1]), (n_unit - 1) & 1, kErrFwdMma)) { ok = false; break; }
+          if (!issue_pv(1, g, 0, j == 0) || !issue_pv(1, g, 1, j == 0)) { ok = false; break; }
+          tc::commit(smem_u32(&v_empty[s]));
+          if (more) {
+            issue_s(1, (g + 1) % NS);
+            tc::commit(smem_u32(&k_empty[(g + 1) % NS]));
+            if (j + 2 == w.nkv) tc::commit(smem_u32(qr_empty));  // last score MMAs of the unit
+          } else {
+            tc::commit(smem_u32(&o_done[0]));
+            tc::commit(smem_u32(&o_done[1]));
+          }
         }
-        if (!issue_pv(1, j, 0) || !issue_pv(1, j, 1)) { ok = false; break; }
-        tc::commit(smem_u32(&v_empty[s]));
-        if (more) {
-          issue_s(1, j + 1);
-          tc::commit(smem_u32(&k_empty[(j + 1) % NS]));
-        } else {
-          tc::commit(smem_u32(&o_done[0]));
-          tc::commit(smem_u32(&o_done[1]));
-        }
+        kv += w.nkv;
       }
       // Every MMA issued must be complete before tensor memory is released.
       tc::commit(smem_u32(&fin[0]));
@@ -272,127 +326,136 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const uint32_t ts = tmem + lane_s + col_s(t);
     const uint32_t to1 = tmem + lane_a + col_o(t);
     const uint32_t to2 = tmem + lane_s + col_o(t);
-    const int q0 = row0_of(t);
-    const int q_lo = q0 + 16 * wq + (lane >> 2);
-    const int q_hi = q_lo + 8;
-    float m_lo = -INFINITY, m_hi = -INFINITY;
-    // this thread's column share: l = sum p (fp32, also gives lse), c = sum of
-    // the bf16-rounded p*s the value MMA consumes (so that O2 and c agree)
-    float l_lo = 0.f, l_hi = 0.f, c_lo = 0.f, c_hi = 0.f;
+    int kv = 0, n_unit = 0;
+    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++n_unit) {
+      const Unit w = unit_of(u);
+      const int q0 = row0_of(w, t);
+      const int q_lo = q0 + 16 * wq + (lane >> 2);
+      const int q_hi = q_lo + 8;
+      float m_lo = -INFINITY, m_hi = -INFINITY;
+      // this thread's column share: l = sum p (fp32, also gives lse), c = sum of
+      // the bf16-rounded p*s the value MMA consumes (so that O2 and c agree)
+      float l_lo = 0.f, l_hi = 0.f, c_lo = 0.f, c_hi = 0.f;
 
-    for (int j = 0; j < nkv; ++j) {
-      // warp-uniform: the .sync.aligned tensor-memory accesses below need every lane
-      const bool landed = mbar_wait(smem_u32(&s_full[t]), j & 1, kErrFwdSoftmax);
-      if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
-      tc::fence_after_sync();
-      uint32_t ra[64], rs[64];
-      tc::ld_16x256b_x8(ta, *reinterpret_cast<uint32_t(*)[32]>(&ra[0]));
-      tc::ld_16x256b_x8(ta + 64, *reinterpret_cast<uint32_t(*)[32]>(&ra[32]));
-      if (HAS_R) {
-        tc::ld_16x256b_x8(ts, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
-        tc::ld_16x256b_x8(ts + 64, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
-      }
-      tc::wait_ld();
-
-      // register i: half h = i/32, rep g = (i%32)/4, e = i%4;
-      // key = 64h + 8g + 2*c4 + (e&1); row lo for e < 2, row hi for e >= 2.
-      // Masked scores become -inf in place; the max is taken on raw q.k and
-      // scaled afterwards (scale_log2 > 0), and the scale folds into exp2's FMA.
-      const int kbase = j * kFwdBN;
-      const bool need_mask = (p.causal && kbase + kFwdBN - 1 > q0) || (kbase + kFwdBN > p.N);
-      if (need_mask) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const int key = kbase + 64 * (i >> 5) + 8 * ((i & 31) >> 2) + 2 * c4 + (i & 1);
-          const int q = (i & 2) ? q_hi : q_lo;
-          const bool valid = key < p.N && (!p.causal || key <= q);
-          if (!valid) ra[i] = 0xFF800000u;  // -inf
+      for (int j = 0; j < w.nkv; ++j) {
+        const int g = kv + j;
+        // warp-uniform: the .sync.aligned tensor-memory accesses below need every lane
+        const bool landed = mbar_wait(smem_u32(&s_full[t]), g & 1, kErrFwdSoftmax);
+        if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
+        tc::fence_after_sync();
+        uint32_t ra[64], rs[64];
+        tc::ld_16x256b_x8(ta, *reinterpret_cast<uint32_t(*)[32]>(&ra[0]));
+        tc::ld_16x256b_x8(ta + 64, *reinterpret_cast<uint32_t(*)[32]>(&ra[32]));
+        if (HAS_R) {
+          tc::ld_16x256b_x8(ts, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
+          tc::ld_16x256b_x8(ts + 64, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
         }
-      }
-      float mx_lo = -INFINITY, mx_hi = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 64; i += 4) {
-        mx_lo = fmaxf(mx_lo, fmaxf(__uint_as_float(ra[i]), __uint_as_float(ra[i + 1])));
-        mx_hi = fmaxf(mx_hi, fmaxf(__uint_as_float(ra[i + 2]), __uint_as_float(ra[i + 3])));
-      }
-      mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
-      mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
-      mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2)) * p.scale_log2;
-      mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2)) * p.scale_log2;
-      const bool grow = mx_lo > m_lo + kRescaleThreshold || mx_hi > m_hi + kRescaleThreshold;
-      if (__any_sync(0xffffffffu, grow)) {
-        const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
-        const float al_lo = mn_lo == -INFINITY ? 1.f : ex2(m_lo - mn_lo);
-        const float al_hi = mn_hi == -INFINITY ? 1.f : ex2(m_hi - mn_hi);
-        l_lo *= al_lo; c_lo *= al_lo; l_hi *= al_hi; c_hi *= al_hi;
-        m_lo = mn_lo; m_hi = mn_hi;
-        if (j > 0) {
-          // O rows of this warp: O1 at the a lanes, O2 at the s lanes; PV(j-1)
-          // has completed (it precedes S(j) in the MMA stream).
-#pragma unroll 1
-          for (int ch = 0; ch < D / 16; ++ch) {
-            uint32_t o1[8], o2[8];
-            tc::ld_16x256b_x2(to1 + 16 * ch, o1);
-            tc::ld_16x256b_x2(to2 + 16 * ch, o2);
-            tc::wait_ld();
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float al = (i & 2) ? al_hi : al_lo;
-              o1[i] = __float_as_uint(__uint_as_float(o1[i]) * al);
-              o2[i] = __float_as_uint(__uint_as_float(o2[i]) * al);
+        tc::wait_ld();
+        // register i: half h = i/32, rep g = (i%32)/4, e = i%4;
+        // key = 64h + 8g + 2*c4 + (e&1); row lo for e < 2, row hi for e >= 2.
+        // Masked scores become -inf in place; the max is taken on raw q.k and
+        // scaled afterwards (scale_log2 > 0), and the scale folds into exp2's FMA.
+        const int kbase = j * kFwdBN;
+        const bool need_mask = (p.causal && kbase + kFwdBN - 1 > q0) || (kbase + kFwdBN > p.N);
+        if (need_mask) {
+  #pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const int key = kbase + 64 * (i >> 5) + 8 * ((i & 31) >> 2) + 2 * c4 + (i & 1);
+            const int q = (i & 2) ? q_hi : q_lo;
+            const bool valid = key < p.N && (!p.causal || key <= q);
+            if (!valid) ra[i] = 0xFF800000u;  // -inf
+          }
+        }
+        // row maxima with four running maxima per row (short dependency chains)
+        float tl[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float th[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  #pragma unroll
+        for (int gg = 0; gg < 16; ++gg) {
+          tl[gg & 3] = fmaxf(tl[gg & 3], fmaxf(__uint_as_float(ra[4 * gg]), __uint_as_float(ra[4 * gg + 1])));
+          th[gg & 3] = fmaxf(th[gg & 3], fmaxf(__uint_as_float(ra[4 * gg + 2]), __uint_as_float(ra[4 * gg + 3])));
+        }
+        float mx_lo = fmaxf(fmaxf(tl[0], tl[1]), fmaxf(tl[2], tl[3]));
+        float mx_hi = fmaxf(fmaxf(th[0], th[1]), fmaxf(th[2], th[3]));
+        mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
+        mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
+        mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2)) * p.scale_log2;
+        mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2)) * p.scale_log2;
+        const bool grow = mx_lo > m_lo + kRescaleThreshold || mx_hi > m_hi + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, grow)) {
+          const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
+          const float al_lo = mn_lo == -INFINITY ? 1.f : ex2(m_lo - mn_lo);
+          const float al_hi = mn_hi == -INFINITY ? 1.f : ex2(m_hi - mn_hi);
+          l_lo *= al_lo; c_lo *= al_lo; l_hi *= al_hi; c_hi *= al_hi;
+          m_lo = mn_lo; m_hi = mn_hi;
+          if (j > 0) {  // the unit's first PV starts O from zero
+            // O rows of this warp: O1 at the a lanes, O2 at the s lanes; PV(j-1)
+            // has completed (it precedes S(j) in the MMA stream).
+  #pragma unroll 1
+            for (int ch = 0; ch < D / 16; ++ch) {
+              uint32_t o1[8], o2[8];
+              tc::ld_16x256b_x2(to1 + 16 * ch, o1);
+              tc::ld_16x256b_x2(to2 + 16 * ch, o2);
+              tc::wait_ld();
+  #pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float al = (i & 2) ? al_hi : al_lo;
+                o1[i] = __float_as_uint(__uint_as_float(o1[i]) * al);
+                o2[i] = __float_as_uint(__uint_as_float(o2[i]) * al);
+              }
+              tc::st_16x256b_x2(to1 + 16 * ch, o1);
+              tc::st_16x256b_x2(to2 + 16 * ch, o2);
             }
-            tc::st_16x256b_x2(to1 + 16 * ch, o1);
-            tc::st_16x256b_x2(to2 + 16 * ch, o2);
           }
         }
-      }
-      const float mu_lo = m_lo == -INFINITY ? 0.f : m_lo;
-      const float mu_hi = m_hi == -INFINITY ? 0.f : m_hi;
-      // p = 2^(a*scale*log2e - m) with the scale folded into one packed FMA per
-      // row pair; l from fp32 p, c from the rounded p*s.
-      const uint64_t sl2 = f2(p.scale_log2, p.scale_log2);
-      const uint64_t nmu_lo = f2(-mu_lo, -mu_lo), nmu_hi = f2(-mu_hi, -mu_hi);
-      uint64_t ls_lo = 0, ls_hi = 0, cs_lo = 0, cs_hi = 0;  // packed partial sums (0 bits = +0.0f)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t pp[16], pq[16];
-#pragma unroll
-        for (int gg = 0; gg < 8; ++gg) {
-          const int i = 32 * hf + 4 * gg;
-          const uint64_t xl = f2_fma(f2(__uint_as_float(ra[i]), __uint_as_float(ra[i + 1])), sl2, nmu_lo);
-          const uint64_t xh = f2_fma(f2(__uint_as_float(ra[i + 2]), __uint_as_float(ra[i + 3])), sl2, nmu_hi);
-          const uint64_t pl = f2(ex2(f2_lo(xl)), ex2(f2_hi(xl)));
-          const uint64_t ph = f2(ex2(f2_lo(xh)), ex2(f2_hi(xh)));
-          ls_lo = f2_add(ls_lo, pl);
-          ls_hi = f2_add(ls_hi, ph);
-          pp[2 * gg] = pack_bf16(f2_lo(pl), f2_hi(pl));
-          pp[2 * gg + 1] = pack_bf16(f2_lo(ph), f2_hi(ph));
-          if (HAS_R) {
-            const uint64_t sl = f2_mul(pl, f2(__uint_as_float(rs[i]), __uint_as_float(rs[i + 1])));
-            const uint64_t sh = f2_mul(ph, f2(__uint_as_float(rs[i + 2]), __uint_as_float(rs[i + 3])));
-            const uint32_t wl = pack_bf16(f2_lo(sl), f2_hi(sl));
-            const uint32_t wh = pack_bf16(f2_lo(sh), f2_hi(sh));
-            pq[2 * gg] = wl;
-            pq[2 * gg + 1] = wh;
-            cs_lo = f2_add(cs_lo, f2(bf16_lo(wl), bf16_hi(wl)));
-            cs_hi = f2_add(cs_hi, f2(bf16_lo(wh), bf16_hi(wh)));
+        const float mu_lo = m_lo == -INFINITY ? 0.f : m_lo;
+        const float mu_hi = m_hi == -INFINITY ? 0.f : m_hi;
+        // p = 2^(a*scale*log2e - m) with the scale folded into one packed FMA per
+        // row pair; l from fp32 p, c from the rounded p*s.
+        const uint64_t sl2 = f2(p.scale_log2, p.scale_log2);
+        const uint64_t nmu_lo = f2(-mu_lo, -mu_lo), nmu_hi = f2(-mu_hi, -mu_hi);
+        uint64_t ls_lo = 0, ls_hi = 0, cs_lo = 0, cs_hi = 0;  // packed partial sums (0 bits = +0.0f)
+  #pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pp[16], pq[16];
+  #pragma unroll
+          for (int gg = 0; gg < 8; ++gg) {
+            const int i = 32 * hf + 4 * gg;
+            const uint64_t xl = f2_fma(f2(__uint_as_float(ra[i]), __uint_as_float(ra[i + 1])), sl2, nmu_lo);
+            const uint64_t xh = f2_fma(f2(__uint_as_float(ra[i + 2]), __uint_as_float(ra[i + 3])), sl2, nmu_hi);
+            const uint64_t pl = f2(ex2(f2_lo(xl)), ex2(f2_hi(xl)));
+            const uint64_t ph = f2(ex2(f2_lo(xh)), ex2(f2_hi(xh)));
+            ls_lo = f2_add(ls_lo, pl);
+            ls_hi = f2_add(ls_hi, ph);
+            pp[2 * gg] = pack_bf16(f2_lo(pl), f2_hi(pl));
+            pp[2 * gg + 1] = pack_bf16(f2_lo(ph), f2_hi(ph));
+            if (HAS_R) {
+              const uint64_t sl = f2_mul(pl, f2(__uint_as_float(rs[i]), __uint_as_float(rs[i + 1])));
+              const uint64_t sh = f2_mul(ph, f2(__uint_as_float(rs[i + 2]), __uint_as_float(rs[i + 3])));
+              const uint32_t wl = pack_bf16(f2_lo(sl), f2_hi(sl));
+              const uint32_t wh = pack_bf16(f2_lo(sh), f2_hi(sh));
+              pq[2 * gg] = wl;
+              pq[2 * gg + 1] = wh;
+              cs_lo = f2_add(cs_lo, f2(bf16_lo(wl), bf16_hi(wl)));
+              cs_hi = f2_add(cs_hi, f2(bf16_lo(wh), bf16_hi(wh)));
+            }
           }
+          tc::st_16x128b_x8(ta + 32 * hf, pp);
+          // rho = 0: the probe rows of S are exact zeros, which read as bf16 zeros
+          if (HAS_R) tc::st_16x128b_x8(ts + 32 * hf, pq);
+          tc::wait_st();
+          tc::fence_before_sync();
+          mbar_arrive(smem_u32(&p_ready[2 * t + hf]));
         }
-        tc::st_16x128b_x8(ta + 32 * hf, pp);
-        // rho = 0: the probe rows of S are exact zeros, which read as bf16 zeros
-        if (HAS_R) tc::st_16x128b_x8(ts + 32 * hf, pq);
-        tc::wait_st();
-        tc::fence_before_sync();
-        mbar_arrive(smem_u32(&p_ready[2 * t + hf]));
+        l_lo += f2_lo(ls_lo) + f2_hi(ls_lo);
+        l_hi += f2_lo(ls_hi) + f2_hi(ls_hi);
+        c_lo += f2_lo(cs_lo) + f2_hi(cs_lo);
+        c_hi += f2_lo(cs_hi) + f2_hi(cs_hi);
       }
-      l_lo += f2_lo(ls_lo) + f2_hi(ls_lo);
-      l_hi += f2_lo(ls_hi) + f2_hi(ls_hi);
-      c_lo += f2_lo(cs_lo) + f2_hi(cs_lo);
-      c_hi += f2_lo(cs_hi) + f2_hi(cs_hi);
-    }
+      if (!ok) break;
 
-    const bool fin_ok = ok && mbar_wait(smem_u32(&o_done[t]), 0, kErrFwdSoftmax);
-    if (__all_sync(0xffffffffu, fin_ok)) {
+      // ---- epilogue: out = O1/l - (O2/l - (c/l)(O1/l)), lse = m + log2(l) (in ln units)
+      const bool done = mbar_wait(smem_u32(&o_done[t]), n_unit & 1, kErrFwdSoftmax);
+      if (!__all_sync(0xffffffffu, done)) { ok = false; break; }
       tc::fence_after_sync();
       l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
       l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
@@ -405,9 +468,13 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const float inv_lo = l_lo > 0.f ? 1.f / l_lo : 0.f;
       const float inv_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
       const float sb_lo = c_lo * inv_lo, sb_hi = c_hi * inv_hi;  // s_bar = c / l
-      const size_t plane = static_cast<size_t>(b) * p.Hq + head_of(t);
-      __nv_bfloat16* out_lo = p.out + (plane * p.N + (q_lo < p.N ? q_lo : 0)) * D;
-      __nv_bfloat16* out_hi = p.out + (plane * p.N + (q_hi < p.N ? q_hi : 0)) * D;
+      const size_t plane = static_cast<size_t>(w.b) * p.Hq + head_of(w, t);
+      // This warp's 16 output rows are staged in shared memory in the 128-byte
+      // swizzled layout of the output tensor map and written by one TMA store.
+      const uint32_t stage = smem_u32(smem + Cfg::kOffOut) + (t * 4 + wq) * Cfg::kOutWarpBytes;
+      if (lane == 0) bulk_wait_read();  // the previous unit's store has read the staging block
+      __syncwarp();
+      const int r_lo = lane >> 2, r_hi = r_lo + 8;  // rows of this warp's 16
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t o1[16], o2[16];
@@ -426,17 +493,34 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             const float a2 = __uint_as_float(o2[4 * gg + e]) * inv;  // O2 / l
             r[e] = a1 - (a2 - sb * a1);
           }
-          if (q_lo < p.N) *reinterpret_cast<uint32_t*>(out_lo + dcol) = pack_bf16(r[0], r[1]);
-          if (q_hi < p.N) *reinterpret_cast<uint32_t*>(out_hi + dcol) = pack_bf16(r[2], r[3]);
+          const int cb = dcol >> 6, chunk = (dcol & 63) >> 3;
+          const uint32_t blk = stage + cb * 2048 + 4 * c4;
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(blk + r_lo * 128 + ((chunk ^ (r_lo & 7)) << 4)),
+                       "r"(pack_bf16(r[0], r[1])) : "memory");
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(blk + r_hi * 128 + ((chunk ^ (r_hi & 7)) << 4)),
+                       "r"(pack_bf16(r[2], r[3])) : "memory");
         }
       }
+      // O has been read: the next unit's first value MMA may overwrite it
+      tc::fence_before_sync();
+      mbar_arrive(smem_u32(&o_free[t]));
       if (p.lse && c4 == 0) {
         if (q_lo < p.N) p.lse[plane * p.N + q_lo] = l_lo > 0.f ? (m_lo + __log2f(l_lo)) * kLn2 : -INFINITY;
         if (q_hi < p.N) p.lse[plane * p.N + q_hi] = l_hi > 0.f ? (m_hi + __log2f(l_hi)) * kLn2 : -INFINITY;
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int row0 = q0 + 16 * wq;
+      if (lane == 0 && row0 < p.N) {
+#pragma unroll
+        for (int cb = 0; cb < Cfg::kCB; ++cb) tma_store_3d(&omap, stage + cb * 2048, cb * 64, row0, static_cast<int>(plane));
+        bulk_commit();
+      }
+      kv += w.nkv;
     }
   }
 
+  if (warp < kFwdTmaWarp && lane == 0) bulk_wait_all();  // output stores complete before exit
   tc::fence_before_sync();
   __syncthreads();
   if (warp == kFwdMmaWarp) {
