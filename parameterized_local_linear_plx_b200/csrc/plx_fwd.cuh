@@ -24,7 +24,9 @@
 //     of one head.  Tensor memory: [S0 | O0 | S1 | O1], 128 columns each.
 //   * Warps 0-3 and 4-7: softmax + epilogue of tile 0 and tile 1;
 //     warp 8: TMA loads (Q/R once, K/V ring); warp 9: TMEM allocation and
-//     the single thread that issues every MMA, in the order
+//     the single thread that issues every MMA (warps 10-11 only complete the
+//     third warpgroup, so that setmaxnreg can move registers from it to the
+//     softmax warps), in the order
 //     PV0(j), S0(j+1), PV1(j), S1(j+1): each tile's next scores come right
 //     after its value MMA, so each softmax overlaps the other tile's MMAs.
 //     One M=128 N=128 MMA takes ~64 tensor cycles and a thread needs a large
@@ -50,7 +52,11 @@ namespace plx {
 
 constexpr int kFwdBM = 64;        // queries per tile (128 stacked rows with their probes)
 constexpr int kFwdBN = 128;       // keys per K/V tile
-constexpr int kFwdThreads = 320;  // 8 softmax warps + TMA warp + MMA warp
+constexpr int kFwdThreads = 384;  // 8 softmax warps, TMA warp, MMA warp, 2 idle warps (3 warpgroups)
+// registers per thread after setmaxnreg: the two softmax warpgroups gain
+// what the load/MMA warpgroup gives up (3 x 128 x 168 = 2 x 128 x 200 + 128 x 104)
+constexpr int kFwdRegsSoftmax = 200;
+constexpr int kFwdRegsOther = 104;
 constexpr int kFwdTmaWarp = 8;
 constexpr int kFwdMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -166,6 +172,9 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   auto col_o = [](int t) { return static_cast<uint32_t>(256 * t + 128); };
   bool ok = true;
 
+  if (warp >= kFwdTmaWarp) {
+    // warpgroup 2 (load, MMA and two idle warps) gives registers to the softmax warpgroups
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kFwdRegsOther));
   if (warp == kFwdTmaWarp) {
     // ================================================================ TMA producer
     if (lane == 0) {
@@ -315,7 +324,15 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       tc::commit(smem_u32(&fin[0]));
       mbar_wait(smem_u32(&fin[0]), 0, kErrFwdMma);
     }
+  }
+    tc::fence_before_sync();
+    asm volatile("bar.sync 1, %0;" ::"n"(kFwdThreads) : "memory");  // every role is done
+    if (warp == kFwdMmaWarp) {
+      tc::fence_after_sync();
+      tc::tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kFwdRegsSoftmax));
     // ================================================================ softmax + epilogue
     const int t = warp >> 2;     // query tile
     const int wq = warp & 3;     // TMEM lane quadrant
@@ -358,7 +375,7 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         const int kbase = j * kFwdBN;
         const bool need_mask = (p.causal && kbase + kFwdBN - 1 > q0) || (kbase + kFwdBN > p.N);
         if (need_mask) {
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < 64; ++i) {
             const int key = kbase + 64 * (i >> 5) + 8 * ((i & 31) >> 2) + 2 * c4 + (i & 1);
             const int q = (i & 2) ? q_hi : q_lo;
@@ -366,16 +383,16 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             if (!valid) ra[i] = 0xFF800000u;  // -inf
           }
         }
-        // row maxima with four running maxima per row (short dependency chains)
+        // row maxima: four running three-input maxima per row (short chains)
         float tl[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         float th[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-  #pragma unroll
+#pragma unroll
         for (int gg = 0; gg < 16; ++gg) {
-          tl[gg & 3] = fmaxf(tl[gg & 3], fmaxf(__uint_as_float(ra[4 * gg]), __uint_as_float(ra[4 * gg + 1])));
-          th[gg & 3] = fmaxf(th[gg & 3], fmaxf(__uint_as_float(ra[4 * gg + 2]), __uint_as_float(ra[4 * gg + 3])));
+          tl[gg & 3] = fmax3(tl[gg & 3], __uint_as_float(ra[4 * gg]), __uint_as_float(ra[4 * gg + 1]));
+          th[gg & 3] = fmax3(th[gg & 3], __uint_as_float(ra[4 * gg + 2]), __uint_as_float(ra[4 * gg + 3]));
         }
-        float mx_lo = fmaxf(fmaxf(tl[0], tl[1]), fmaxf(tl[2], tl[3]));
-        float mx_hi = fmaxf(fmaxf(th[0], th[1]), fmaxf(th[2], th[3]));
+        float mx_lo = fmaxf(fmax3(tl[0], tl[1], tl[2]), tl[3]);
+        float mx_hi = fmaxf(fmax3(th[0], th[1], th[2]), th[3]);
         mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
         mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
         mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2)) * p.scale_log2;
@@ -390,13 +407,13 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           if (j > 0) {  // the unit's first PV starts O from zero
             // O rows of this warp: O1 at the a lanes, O2 at the s lanes; PV(j-1)
             // has completed (it precedes S(j) in the MMA stream).
-  #pragma unroll 1
+#pragma unroll 1
             for (int ch = 0; ch < D / 16; ++ch) {
               uint32_t o1[8], o2[8];
               tc::ld_16x256b_x2(to1 + 16 * ch, o1);
               tc::ld_16x256b_x2(to2 + 16 * ch, o2);
               tc::wait_ld();
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 8; ++i) {
                 const float al = (i & 2) ? al_hi : al_lo;
                 o1[i] = __float_as_uint(__uint_as_float(o1[i]) * al);
@@ -414,10 +431,10 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         const uint64_t sl2 = f2(p.scale_log2, p.scale_log2);
         const uint64_t nmu_lo = f2(-mu_lo, -mu_lo), nmu_hi = f2(-mu_hi, -mu_hi);
         uint64_t ls_lo = 0, ls_hi = 0, cs_lo = 0, cs_hi = 0;  // packed partial sums (0 bits = +0.0f)
-  #pragma unroll
+#pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           uint32_t pp[16], pq[16];
-  #pragma unroll
+#pragma unroll
           for (int gg = 0; gg < 8; ++gg) {
             const int i = 32 * hf + 4 * gg;
             const uint64_t xl = f2_fma(f2(__uint_as_float(ra[i]), __uint_as_float(ra[i + 1])), sl2, nmu_lo);
@@ -518,14 +535,9 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       }
       kv += w.nkv;
     }
-  }
-
-  if (warp < kFwdTmaWarp && lane == 0) bulk_wait_all();  // output stores complete before exit
-  tc::fence_before_sync();
-  __syncthreads();
-  if (warp == kFwdMmaWarp) {
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, Cfg::kTmemCols);
+    if (lane == 0) bulk_wait_all();  // output stores complete before exit
+    tc::fence_before_sync();
+    asm volatile("bar.sync 1, %0;" ::"n"(kFwdThreads) : "memory");  // every role is done
   }
 }
 
