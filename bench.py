@@ -421,8 +421,9 @@ def run_gpu(args, world, rank, local):
             "prefill": {"tflops": prefill_tflops, "ms_per_step": pre_avg, "flops_per_step": p_flops,
                         "gbs_io": world * prefill_bytes(**PRE) / (pre_avg * 1e-3) / 1e9,
                         "roofline": roof_pre},
-            "roofline": roof_dec,
-            "roofline_prefill": roof_pre,
+            # the dominant kernel of the step by time is the prefill kernel
+            "roofline": roof_pre,
+            "roofline_decode": roof_dec,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,

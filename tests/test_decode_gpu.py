@@ -134,3 +134,25 @@ def test_decode_timeout_path_reports_and_recovers(plx):
     assert plx.plx_check_device_status() == plx.PLX_OK  # cleared
     o, l, ro, rl = run(plx, 2, 4, 2, 128, 128, seed=11)
     assert_close(o, ro, l, rl, "after timeout")
+
+
+def test_decode_largest_sweep_point(plx):
+    """The largest decode-sweep point kept under the 150 GB cap: B=1024,
+    context 32768 (137 GB of bf16 KV), ragged seqlens in [ctx/2, ctx], in the
+    automatic split configuration the sweep times; sampled batch entries
+    (first, last, random) against the oracle."""
+    B, ctx = 1024, 32768
+    free, _ = torch.cuda.mem_get_info()
+    need = 2 * B * 8 * ctx * 128 * 2
+    if free < need + (8 << 30):
+        pytest.skip(f"needs {need / 1e9:.0f} GB of free device memory, {free / 1e9:.0f} GB free")
+    q, kc, vc, r, sl = inputs.decode_inputs(B, 16, 8, ctx, 128, seed=10, seqlens="ragged", device="cuda")
+    out, lse = plx.plx_decode(q, kc, vc, sl, r)
+    torch.cuda.synchronize()
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    pick = [0, 1, 511, 777, 1023]
+    qc, kcc, vcc, rc, slc = (t[pick].cpu() for t in (q, kc, vc, r, sl))
+    ro, rl = oracle.decode_effective(qc, rc, kcc, vcc, slc)
+    assert_close(out[pick], ro, lse[pick], rl, "largest sweep point")
+    del q, kc, vc, r, sl
+    torch.cuda.empty_cache()
