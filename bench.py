@@ -265,6 +265,17 @@ def oracle_decode_sample(q, r, kc, vc, sl, budget_s=10.0, max_entries=None):
     return done, time.perf_counter() - t0, nbytes
 
 
+def bench_config(world):
+    """The `config` object of the JSON line, identical in both arms."""
+    return {
+        "workload": f"decode: Qwen3-0.6B-shaped layer B={DEC['B']} ctx={DEC['S']} (equal seqlens) Hq=16 Hkv=8 "
+                    f"d=128 bf16 KV cache; prefill: B={PRE['B']} N={PRE['N']} Hq=16 Hkv=8 d=128 causal bf16, out+lse",
+        "l2": f"inputs larger than L2 (decode {decode_bytes(DEC['B'], DEC['Hq'], DEC['Hkv'], DEC['d'], [DEC['S']] * DEC['B']) / 1e9:.2f} GB, "
+              f"prefill {prefill_bytes(**PRE) / 1e9:.2f} GB per step; L2 126 MB)",
+        "parallelism": f"replicas x{world}, no collective on the data path",
+    }
+
+
 def run_reference(args, world, rank):
     """--impl reference: the fp64 CPU oracle on a bounded sample per step."""
     if rank != 0:
@@ -287,11 +298,10 @@ def run_reference(args, world, rank):
         "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": "decode: Qwen3-0.6B-shaped layer B=64 ctx=4096 Hq=16 Hkv=8 d=128 bf16 KV cache, "
-                               "equal seqlens (oracle: 2 of the 64 batch entries per step)"},
+        "config": bench_config(world),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
-                         "sample": f"{per_step} batch entries x {DEC['Hq']} heads x {DEC['S']} keys per step, "
-                                   "effective-weight fp64 form"},
+                         "sample": f"decode only: {per_step} of the {DEC['B']} batch entries (x {DEC['Hq']} heads x "
+                                   f"{DEC['S']} keys) per step, effective-weight fp64 form"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -407,16 +417,8 @@ def run_gpu(args, world, rank, local):
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {
-                "workload": f"decode: Qwen3-0.6B-shaped layer B={DEC['B']} ctx={DEC['S']} (equal seqlens) "
-                            f"Hq=16 Hkv=8 d=128 bf16 KV cache; prefill: B={PRE['B']} N={PRE['N']} Hq=16 Hkv=8 "
-                            "d=128 causal bf16, out+lse",
-                "decode_splits": n_splits,
-                "l2": f"inputs larger than L2 (decode {d_bytes / 1e9:.2f} GB, prefill "
-                      f"{prefill_bytes(**PRE) / 1e9:.2f} GB per step; L2 126 MB)",
-                "parallelism": f"replicas x{world}, no collective on the data path",
-            },
-            "decode": {"gbs": value, "us_per_step": dec_avg * 1e3, "bytes_per_step": d_bytes,
+            "config": bench_config(world),
+            "decode": {"gbs": value, "us_per_step": dec_avg * 1e3, "bytes_per_step": d_bytes, "splits": n_splits,
                        "tflops": world * d_flops / (dec_avg * 1e-3) / 1e12},
             "prefill": {"tflops": prefill_tflops, "ms_per_step": pre_avg, "flops_per_step": p_flops,
                         "gbs_io": world * prefill_bytes(**PRE) / (pre_avg * 1e-3) / 1e9,
@@ -436,25 +438,32 @@ def run_gpu(args, world, rank, local):
 def run_e2e(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes):
     """Decode measured through plx_decode with the step's inputs (q, r,
     seqlens) copied from pinned host memory and its result (out, lse) read
-    back, all inside the timed region.  The KV cache is the engine's resident
-    state and is not re-sent each step."""
+    back, all inside the timed region.  The inputs travel packed in one
+    buffer and the results in another (one H2D and one D2H copy per step);
+    the KV cache is the engine's resident state and is not re-sent."""
     import torch
-    hq = q.cpu().pin_memory()
-    hr = r.cpu().pin_memory()
-    hsl = sl.cpu().pin_memory()
-    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    hlse = torch.empty(q.shape[:2], dtype=torch.float32).pin_memory()
-    dq, dr, dsl = torch.empty_like(q), torch.empty_like(r), torch.empty_like(sl)
-    h2d = hq.numel() * 2 + hr.numel() * 2 + hsl.numel() * 4
-    d2h = hout.numel() * 2 + hlse.numel() * 4
+    B, Hq, d = q.shape
+    nq, nsl = q.numel() * 2, sl.numel() * 4
+    nout, nlse = q.numel() * 2, B * Hq * 4
+    h_in = torch.empty(2 * nq + nsl, dtype=torch.uint8).pin_memory()
+    h_in[:nq].view(torch.bfloat16).view(q.shape).copy_(q.cpu())
+    h_in[nq:2 * nq].view(torch.bfloat16).view(q.shape).copy_(r.cpu())
+    h_in[2 * nq:].view(torch.int32).copy_(sl.cpu())
+    d_in = torch.empty_like(h_in, device=dev)
+    dq = d_in[:nq].view(torch.bfloat16).view(q.shape)
+    dr = d_in[nq:2 * nq].view(torch.bfloat16).view(q.shape)
+    dsl = d_in[2 * nq:].view(torch.int32)
+    d_res = torch.empty(nout + nlse, dtype=torch.uint8, device=dev)
+    dout = d_res[:nout].view(torch.bfloat16).view(q.shape)
+    dlse = d_res[nout:].view(torch.float32).view(B, Hq)
+    h_res = torch.empty(nout + nlse, dtype=torch.uint8).pin_memory()
+    ws = torch.empty(max(16, plx.plx_decode_workspace_size(B, Hq, kc.shape[1], kc.shape[2], d, 0)),
+                     dtype=torch.uint8, device=dev)
 
     def one():
-        dq.copy_(hq, non_blocking=True)
-        dr.copy_(hr, non_blocking=True)
-        dsl.copy_(hsl, non_blocking=True)
-        o, l = plx.plx_decode(dq, kc, vc, dsl, dr, stream=stream)
-        hout.copy_(o, non_blocking=True)
-        hlse.copy_(l, non_blocking=True)
+        d_in.copy_(h_in, non_blocking=True)
+        plx.plx_decode(dq, kc, vc, dsl, dr, out=dout, lse=dlse, workspace=ws, stream=stream)
+        h_res.copy_(d_res, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
         one()
@@ -467,8 +476,8 @@ def run_e2e(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes):
     t1.record(stream)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
-    return {"value": world * d_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "us_per_step": ms * 1e3}
+    return {"value": world * d_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h_in.numel(),
+            "d2h_bytes_per_step": h_res.numel(), "us_per_step": ms * 1e3}
 
 
 # ------------------------------------------------------------------ extra reports
