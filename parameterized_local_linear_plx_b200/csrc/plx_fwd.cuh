@@ -363,11 +363,13 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         uint32_t ra[64], rs[64];
         tc::ld_16x256b_x8(ta, *reinterpret_cast<uint32_t(*)[32]>(&ra[0]));
         tc::ld_16x256b_x8(ta + 64, *reinterpret_cast<uint32_t(*)[32]>(&ra[32]));
+        tc::wait_ld();
+        // the probe scores are needed only after the row max: their load
+        // overlaps the max reduction (the next wait::ld collects it)
         if (HAS_R) {
           tc::ld_16x256b_x8(ts, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
           tc::ld_16x256b_x8(ts + 64, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
         }
-        tc::wait_ld();
         // register i: half h = i/32, rep g = (i%32)/4, e = i%4;
         // key = 64h + 8g + 2*c4 + (e&1); row lo for e < 2, row hi for e >= 2.
         // Masked scores become -inf in place; the max is taken on raw q.k and
@@ -424,6 +426,7 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             }
           }
         }
+        if (HAS_R) tc::wait_ld();
         const float mu_lo = m_lo == -INFINITY ? 0.f : m_lo;
         const float mu_hi = m_hi == -INFINITY ? 0.f : m_hi;
         // p = 2^(a*scale*log2e - m) with the scale folded into one packed FMA per
