@@ -93,6 +93,69 @@ int plx_fwd(const void* q, const void* k, const void* v, const void* r,
             void* stream);
 
 /*
+ * plx_fwd_train -- plx_fwd for training: the same outputs, plus two per-row
+ * values that plx_bwd needs.
+ *
+ *   obar [B, Hq, N, d] bf16   o_bar_i = sum_j w_ij v_j, the softmax-attention
+ *                             output inside the Parallax output equation
+ *   sbar [B, Hq, N]    fp32   s_bar_i = sum_j w_ij (rho_i . k_j); may be NULL
+ *                             only when r is NULL (then s_bar = 0)
+ *   lse must not be NULL here.
+ *
+ * Both are exact by-products of the streamed form (O1 / l and c / l).  The
+ * pages give the forward only; keeping them is this library's choice, so that
+ * the backward needs no extra pass over the keys.  Returns PLX_ERR_NULL when
+ * lse or obar is NULL, or sbar is NULL with r non-NULL; otherwise as plx_fwd.
+ */
+int plx_fwd_train(const void* q, const void* k, const void* v, const void* r,
+                  void* out, float* lse, void* obar, float* sbar,
+                  int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                  void* stream);
+
+/*
+ * plx_bwd_workspace_size -- bytes of device workspace plx_bwd needs: two fp32
+ * values per query row (g_bar and Dd below), each array padded to 256 bytes.
+ * 0 for invalid sizes.
+ */
+size_t plx_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
+
+/*
+ * plx_bwd -- gradients of the loss sum_i dout_i . out_i with respect to q, k,
+ * v and rho, for the forward of plx_fwd_train with the same arguments.
+ *
+ * The pages define the forward only (gist.science, section "Method: Parallax
+ * / Core mechanism").  Written with effective weights
+ * w_hat_ij = w_ij (1 - s_ij + s_bar_i), s_ij = rho_i . k_j, its gradient is
+ *   g_ij = dout_i . v_j, g_bar_i = dout_i . obar_i, Dd_i = dout_i . out_i + s_bar_i g_bar_i
+ *   dv_j = sum_i w_hat_ij dout_i
+ *   dS_ij = w_ij (g_bar_i - g_ij),  dA_ij = w_ij (g_ij (1 - s_ij + s_bar_i) + s_ij g_bar_i - Dd_i)
+ *   dq_i = scale sum_j dA_ij k_j,  dr_i = sum_j dS_ij k_j,
+ *   dk_j = sum_i scale dA_ij q_i + dS_ij rho_i
+ * with w_ij = exp(scale q_i . k_j - lse_i).
+ *
+ *   q, r [B, Hq, N, d] bf16; k, v [B, Hkv, N, d] bf16   forward inputs (r NULL: rho = 0)
+ *   out, obar [B, Hq, N, d] bf16; lse, sbar [B, Hq, N] fp32   from plx_fwd_train
+ *                                                    (sbar ignored when r is NULL)
+ *   dout [B, Hq, N, d] bf16                          gradient of the loss w.r.t. out
+ *   dq, dr [B, Hq, N, d] bf16; dk, dv [B, Hkv, N, d] bf16   written (dr may be NULL;
+ *                                                    with r NULL it is the gradient at rho = 0)
+ *   workspace: at least plx_bwd_workspace_size(...) bytes, 16-byte aligned;
+ *   its contents are overwritten.
+ *
+ * Runs three kernels on `stream`: a per-row reduction, a query-side kernel
+ * (dq, dr) and a key-side kernel (dk, dv), both on tcgen05 tensor cores.  The
+ * outputs are written, not accumulated; dk and dv sum over the query heads
+ * of each KV group.  Requirements and errors as plx_fwd, plus
+ * PLX_ERR_WORKSPACE for a missing or small workspace.
+ */
+int plx_bwd(const void* q, const void* k, const void* v, const void* r,
+            const void* out, const void* dout, const float* lse,
+            const void* obar, const float* sbar,
+            void* dq, void* dk, void* dv, void* dr,
+            int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * plx_decode_num_splits -- the split count plx_decode uses when passed
  * num_splits = 0 (a function of the shapes only; >= 1).
  */

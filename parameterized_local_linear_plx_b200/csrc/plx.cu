@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/plx.h"
+#include "plx_bwd.cuh"
 #include "plx_decode.cuh"
 #include "plx_fwd.cuh"
 
@@ -138,17 +139,47 @@ int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const plx::Decod
   return PLX_OK;
 }
 
-template <int D, bool HAS_R>
+template <int D, bool HAS_R, bool SAVE_AUX>
 int launch_fwd(const CUtensorMap& qm, const CUtensorMap& rm, const CUtensorMap& km, const CUtensorMap& vm,
-               const CUtensorMap& om, const plx::FwdParams& p, unsigned grid, cudaStream_t st) {
+               const CUtensorMap& om, const CUtensorMap& am, const plx::FwdParams& p, unsigned grid,
+               cudaStream_t st) {
   using Cfg = plx::FwdCfg<D>;
   static bool done[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  auto kern = plx::plx_fwd_kernel<D, HAS_R>;
+  auto kern = plx::plx_fwd_kernel<D, HAS_R, SAVE_AUX>;
   if (ensure_smem(kern, Cfg::kSmemBytes, &done[dev]) != PLX_OK) return PLX_ERR_CUDA;
-  kern<<<grid, plx::kFwdThreads, Cfg::kSmemBytes, st>>>(qm, rm, km, vm, om, p);
+  kern<<<grid, plx::kFwdThreads, Cfg::kSmemBytes, st>>>(qm, rm, km, vm, om, am, p);
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
+template <int D, bool HAS_R>
+int launch_bwd(const CUtensorMap& qm, const CUtensorMap& rm, const CUtensorMap& om, const CUtensorMap& km,
+               const CUtensorMap& vm, const plx::BwdParams& p, const void* dout, const void* out,
+               const void* obar, float* gbar, float* dd, cudaStream_t st) {
+  using QCfg = plx::BwdQCfg<D>;
+  using KVCfg = plx::BwdKVCfg<D>;
+  static bool done_q[kMaxDevices], done_kv[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const long long rows = static_cast<long long>(p.B) * p.Hq * p.N;
+  plx::plx_bwd_pre_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out),
+      static_cast<const __nv_bfloat16*>(obar), p.sbar, gbar, dd, rows);
+  if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+  auto kq = plx::plx_bwd_q_kernel<D, HAS_R>;
+  if (ensure_smem(kq, QCfg::kSmemBytes, &done_q[dev]) != PLX_OK) return PLX_ERR_CUDA;
+  kq<<<static_cast<unsigned>(p.B * p.Hq * p.n_qtiles), plx::kBwdThreads, QCfg::kSmemBytes, st>>>(qm, rm, om, km, vm, p);
+  if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+  auto kkv = plx::plx_bwd_kv_kernel<D, HAS_R>;
+  if (ensure_smem(kkv, KVCfg::kSmemBytes, &done_kv[dev]) != PLX_OK) return PLX_ERR_CUDA;
+  kkv<<<static_cast<unsigned>(p.B * p.Hkv * p.n_ktiles), plx::kBwdThreads, KVCfg::kSmemBytes, st>>>(qm, rm, om, km, vm, p);
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
+size_t bwd_workspace_bytes(int B, int Hq, int N) {
+  const size_t rows = static_cast<size_t>(B) * Hq * N;
+  return 2 * ((rows * sizeof(float) + 255) / 256 * 256);
 }
 
 }  // namespace
@@ -173,15 +204,23 @@ const char* plx_status_string(int status) {
   }
 }
 
-int plx_fwd(const void* q, const void* k, const void* v, const void* r, void* out, float* lse, int B,
-            int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// plx_fwd and plx_fwd_train: obar / sbar non-NULL selects the training kernel.
+int fwd_common(const void* q, const void* k, const void* v, const void* r, void* out, float* lse,
+               void* obar, float* sbar, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+               void* stream) {
   if (!q || !k || !v || !out) return PLX_ERR_NULL;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return PLX_ERR_SHAPE;
   if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
   if (Hq % Hkv) return PLX_ERR_GQA;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (r && !aligned16(r)) || !aligned16(out) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (obar && !aligned16(obar)) ||
+      (sbar && (reinterpret_cast<uintptr_t>(sbar) & 3u)))
     return PLX_ERR_ALIGN;
+  const bool train = obar != nullptr;
   const int G = Hq / Hkv;
   const int pair_heads = (G % 2 == 0) ? 1 : 0;
   const int n_pairs = pair_heads ? Hq / 2 : Hq;
@@ -193,7 +232,7 @@ int plx_fwd(const void* q, const void* k, const void* v, const void* r, void* ou
   if (rc != PLX_OK) return rc;
   if ((rc = get_encoder()) != PLX_OK) return rc;
 
-  CUtensorMap qm, rm, km, vm, om;
+  CUtensorMap qm, rm, km, vm, om, am;
   const long long pq = static_cast<long long>(B) * Hq, pkv = static_cast<long long>(B) * Hkv;
   if (make_map_3d(&qm, q, d, N, pq, 16) != PLX_OK || make_map_3d(&km, k, d, N, pkv, plx::kFwdBN) != PLX_OK ||
       make_map_3d(&vm, v, d, N, pkv, plx::kFwdBN) != PLX_OK || make_map_3d(&om, out, d, N, pq, 16) != PLX_OK)
@@ -203,9 +242,15 @@ int plx_fwd(const void* q, const void* k, const void* v, const void* r, void* ou
   } else {
     rm = qm;  // unused
   }
+  if (train) {
+    if (make_map_3d(&am, obar, d, N, pq, 16) != PLX_OK) return PLX_ERR_CUDA;
+  } else {
+    am = om;  // unused
+  }
   plx::FwdParams p;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
+  p.sbar = sbar;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.G = G;
   p.pair_heads = pair_heads; p.n_pairs = n_pairs; p.n_qblocks = n_qblocks;
   p.num_units = static_cast<int>(grid);
@@ -214,9 +259,93 @@ int plx_fwd(const void* q, const void* k, const void* v, const void* r, void* ou
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // persistent: one CTA per SM (the kernel's shared memory allows no more)
   const unsigned g = static_cast<unsigned>(std::min<long long>(grid, g_sm_count[dev]));
+  if (train) {
+    if (d == 128)
+      return r ? launch_fwd<128, true, true>(qm, rm, km, vm, om, am, p, g, st)
+               : launch_fwd<128, false, true>(qm, rm, km, vm, om, am, p, g, st);
+    return r ? launch_fwd<64, true, true>(qm, rm, km, vm, om, am, p, g, st)
+             : launch_fwd<64, false, true>(qm, rm, km, vm, om, am, p, g, st);
+  }
   if (d == 128)
-    return r ? launch_fwd<128, true>(qm, rm, km, vm, om, p, g, st) : launch_fwd<128, false>(qm, rm, km, vm, om, p, g, st);
-  return r ? launch_fwd<64, true>(qm, rm, km, vm, om, p, g, st) : launch_fwd<64, false>(qm, rm, km, vm, om, p, g, st);
+    return r ? launch_fwd<128, true, false>(qm, rm, km, vm, om, am, p, g, st)
+             : launch_fwd<128, false, false>(qm, rm, km, vm, om, am, p, g, st);
+  return r ? launch_fwd<64, true, false>(qm, rm, km, vm, om, am, p, g, st)
+           : launch_fwd<64, false, false>(qm, rm, km, vm, om, am, p, g, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int plx_fwd(const void* q, const void* k, const void* v, const void* r, void* out, float* lse, int B,
+            int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  return fwd_common(q, k, v, r, out, lse, nullptr, nullptr, B, Hq, Hkv, N, d, causal, scale, stream);
+}
+
+int plx_fwd_train(const void* q, const void* k, const void* v, const void* r, void* out, float* lse,
+                  void* obar, float* sbar, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                  void* stream) {
+  if (!lse || !obar || (r && !sbar)) return PLX_ERR_NULL;
+  return fwd_common(q, k, v, r, out, lse, obar, sbar, B, Hq, Hkv, N, d, causal, scale, stream);
+}
+
+size_t plx_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv || (d != 64 && d != 128)) return 0;
+  return bwd_workspace_bytes(B, Hq, N);
+}
+
+int plx_bwd(const void* q, const void* k, const void* v, const void* r, const void* out, const void* dout,
+            const float* lse, const void* obar, const float* sbar, void* dq, void* dk, void* dv, void* dr,
+            int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* workspace,
+            size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out || !dout || !lse || !obar || !dq || !dk || !dv || (r && !sbar)) return PLX_ERR_NULL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return PLX_ERR_SHAPE;
+  if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
+  if (Hq % Hkv) return PLX_ERR_GQA;
+  const void* p16[] = {q, k, v, r, out, dout, obar, dq, dk, dv, dr, workspace};
+  for (const void* ptr : p16)
+    if (ptr && !aligned16(ptr)) return PLX_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (sbar && (reinterpret_cast<uintptr_t>(sbar) & 3u)))
+    return PLX_ERR_ALIGN;
+  const size_t need = bwd_workspace_bytes(B, Hq, N);
+  if (!workspace || workspace_bytes < need) return PLX_ERR_WORKSPACE;
+  const int n_qtiles = (N + plx::kBwdBM - 1) / plx::kBwdBM;
+  const int n_ktiles = (N + plx::kBwdBN - 1) / plx::kBwdBN;
+  if (static_cast<long long>(B) * Hq * n_qtiles > 0x7fffffffLL) return PLX_ERR_SHAPE;
+  int dev = 0;
+  int rc = check_arch(&dev);
+  if (rc != PLX_OK) return rc;
+  if ((rc = get_encoder()) != PLX_OK) return rc;
+  CUtensorMap qm, rm, om, km, vm;
+  const long long pq = static_cast<long long>(B) * Hq, pkv = static_cast<long long>(B) * Hkv;
+  if (make_map_3d(&qm, q, d, N, pq, 16) != PLX_OK || make_map_3d(&om, dout, d, N, pq, 16) != PLX_OK ||
+      make_map_3d(&km, k, d, N, pkv, plx::kBwdBN) != PLX_OK || make_map_3d(&vm, v, d, N, pkv, plx::kBwdBN) != PLX_OK)
+    return PLX_ERR_CUDA;
+  if (r) {
+    if (make_map_3d(&rm, r, d, N, pq, 16) != PLX_OK) return PLX_ERR_CUDA;
+  } else {
+    rm = qm;  // unused
+  }
+  const size_t half = need / 2;
+  float* gbar = static_cast<float*>(workspace);
+  float* dd = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
+  plx::BwdParams p;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dr = static_cast<__nv_bfloat16*>(dr);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.lse = lse; p.gbar = gbar; p.dd = dd; p.sbar = r ? sbar : nullptr;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.G = Hq / Hkv;
+  p.n_qtiles = n_qtiles; p.n_ktiles = n_ktiles;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.scale_log2 = scale * plx::kLog2e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return r ? launch_bwd<128, true>(qm, rm, om, km, vm, p, dout, out, obar, gbar, dd, st)
+             : launch_bwd<128, false>(qm, rm, om, km, vm, p, dout, out, obar, gbar, dd, st);
+  return r ? launch_bwd<64, true>(qm, rm, om, km, vm, p, dout, out, obar, gbar, dd, st)
+           : launch_bwd<64, false>(qm, rm, om, km, vm, p, dout, out, obar, gbar, dd, st);
 }
 
 int plx_decode_num_splits(int B, int Hq, int Hkv, int S_max, int d) {

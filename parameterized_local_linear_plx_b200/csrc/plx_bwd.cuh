@@ -1,0 +1,659 @@
+// plx_bwd.cuh -- gradients of the Parallax attention forward on sm_100a.
+//
+// The forward is that of gist.science, "Technical overview: Parallax -
+// parameterized local linear attention for language modeling", section
+// "Method: Parallax / Core mechanism" (o = o_SA - Sigma_KV rho, eta = 0), in
+// its effective-weight form o_i = sum_j w_hat_ij v_j with
+// w_hat_ij = w_ij (1 - s_ij + s_bar_i), s_ij = rho_i . k_j.  The pages give no
+// backward; the gradient of the loss sum_i dO_i . o_i is
+//
+//   g_ij  = dO_i . v_j,   g_bar_i = dO_i . o_bar_i,   Dd_i = dO_i . o_i + s_bar_i g_bar_i
+//   dV_j  = sum_i w_hat_ij dO_i
+//   dS_ij = w_ij (g_bar_i - g_ij)
+//   dA_ij = w_ij (g_ij (1 - s_ij + s_bar_i) + s_ij g_bar_i - Dd_i)
+//   dQ_i  = scale sum_j dA_ij k_j,   dR_i = sum_j dS_ij k_j
+//   dK_j  = sum_i (scale dA_ij) q_i + dS_ij rho_i
+//
+// with w_ij = exp(scale q_i . k_j - lse_i) recomputed from the forward's lse,
+// and o_bar, s_bar kept by the training forward.
+//
+// Kernels:
+//   * plx_bwd_pre_kernel: one warp per query row: g_bar and Dd.
+//   * plx_bwd_q_kernel (dQ, dR): one CTA per 64-query tile, with the stacked
+//     [Q;R] operand of the forward (rows 32w..32w+15: queries 16w..16w+15; rows
+//     32w+16..32w+31: their probes).  Per 128-key tile: S = [Q;R] K^T and
+//     G = [dO;0] V^T (dO in the query slots of a second stacked operand and
+//     zeros in the probe slots, so g lands in the query lanes beside a), then
+//     the element-wise warps write [scale dA ; dS] in bf16 over S and one MMA
+//     [scale dA ; dS] K accumulates [dQ ; dR] in tensor memory.
+//   * plx_bwd_kv_kernel (dK, dV): one CTA per 128-key tile, keys as the MMA
+//     rows.  For each 64-query tile of each query head of the KV group:
+//     [A^T | S^T] = K [Q;R]^T and G^T = V dO^T; per (key, query) the
+//     element-wise warps write W_hat^T, scale dA^T and dS^T in bf16; then
+//     dV += W_hat^T dO and dK += [scale dA^T | dS^T] [Q;R] (the stacked tile is
+//     the K-major B of the first product and the MN-major B of the last).
+//     Each CTA owns its output rows: no atomics anywhere.
+//   * In both: warps 0-3 element-wise (warp w reads TMEM lanes 32w..32w+31),
+//     warp 4 issues the TMA loads, warp 5 allocates tensor memory and one of
+//     its threads issues every MMA.  Every wait is bounded (device error word).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "plx_ptx.cuh"
+#include "plx_tcgen05.cuh"
+
+namespace plx {
+
+constexpr int kBwdBM = 64;        // queries per tile (128 stacked rows with their probes)
+constexpr int kBwdBN = 128;       // keys per tile
+constexpr int kBwdThreads = 192;  // 4 element-wise warps, TMA warp, MMA warp
+constexpr int kBwdTmaWarp = 4;
+constexpr int kBwdMmaWarp = 5;
+constexpr int kBwdStages = 2;
+
+struct BwdParams {
+  __nv_bfloat16* dq;  // [B, Hq, N, D]
+  __nv_bfloat16* dr;  // [B, Hq, N, D] or nullptr
+  __nv_bfloat16* dk;  // [B, Hkv, N, D]
+  __nv_bfloat16* dv;  // [B, Hkv, N, D]
+  const float* lse;   // [B, Hq, N]
+  const float* gbar;  // [B, Hq, N]  dO . o_bar
+  const float* dd;    // [B, Hq, N]  dO . o + s_bar g_bar
+  const float* sbar;  // [B, Hq, N] or nullptr (rho = 0)
+  int B, Hq, Hkv, N, G;
+  int n_qtiles;  // ceil(N / 64)
+  int n_ktiles;  // ceil(N / 128)
+  int causal;
+  float scale, scale_log2;
+};
+
+// ---------------------------------------------------------------- preprocess
+// g_bar = dO . o_bar and Dd = dO . o + s_bar g_bar for every query row (one
+// warp per row; lane l reads the 32-bit words l, l + 32, ... of the row).
+template <int D>
+__global__ void __launch_bounds__(256) plx_bwd_pre_kernel(const __nv_bfloat16* __restrict__ dout,
+                                                          const __nv_bfloat16* __restrict__ out,
+                                                          const __nv_bfloat16* __restrict__ obar,
+                                                          const float* __restrict__ sbar, float* __restrict__ gbar,
+                                                          float* __restrict__ dd, long long rows) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint32_t* pd = reinterpret_cast<const uint32_t*>(dout + row * D);
+  const uint32_t* po = reinterpret_cast<const uint32_t*>(out + row * D);
+  const uint32_t* pb = reinterpret_cast<const uint32_t*>(obar + row * D);
+  float go = 0.f, gb = 0.f;
+#pragma unroll
+  for (int i = 0; i < D / 64; ++i) {
+    const uint32_t a = __ldg(pd + 32 * i + lane), o = __ldg(po + 32 * i + lane), b = __ldg(pb + 32 * i + lane);
+    go = fmaf(bf16_lo(a), bf16_lo(o), go);
+    go = fmaf(bf16_hi(a), bf16_hi(o), go);
+    gb = fmaf(bf16_lo(a), bf16_lo(b), gb);
+    gb = fmaf(bf16_hi(a), bf16_hi(b), gb);
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) {
+    go += __shfl_xor_sync(0xffffffffu, go, m);
+    gb += __shfl_xor_sync(0xffffffffu, gb, m);
+  }
+  if (lane == 0) {
+    const float sb = sbar ? sbar[row] : 0.f;
+    gbar[row] = gb;
+    dd[row] = go + sb * gb;
+  }
+}
+
+// ---------------------------------------------------------------- dQ, dR
+template <int D>
+struct BwdQCfg {
+  static constexpr int kCB = D / 64;              // 128-byte column blocks per row
+  static constexpr int kBlock = 128 * 128;        // one [128 rows x 128 B] block
+  static constexpr int kTileBytes = kCB * kBlock;  // a 128-row tile
+  static constexpr int kOffQR = 0;
+  static constexpr int kOffDO = kTileBytes;        // [dO ; 0] stacked like [Q ; R]
+  static constexpr int kOffK = 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kBwdStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kBwdStages * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  // tensor memory: S [0,128), G [128,256), [dQ ; dR] [256, 256 + D)
+  static constexpr uint32_t kColS = 0, kColG = 128, kColAcc = 256, kTmemCols = 512;
+};
+
+template <int D, bool HAS_R>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap rmap,
+                 const __grid_constant__ CUtensorMap omap, const __grid_constant__ CUtensorMap kmap,
+                 const __grid_constant__ CUtensorMap vmap, const BwdParams p) {
+  using Cfg = BwdQCfg<D>;
+  constexpr int NS = kBwdStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* q_full = bars;              // [1] [Q;R] and [dO;0] landed
+  uint64_t* kv_full = bars + 1;         // [NS]
+  uint64_t* kv_empty = kv_full + NS;    // [NS]
+  uint64_t* s_full = kv_empty + NS;     // [1] S and G of the current key tile are in TMEM
+  uint64_t* p_ready = s_full + 1;       // [1] [dA ; dS] written (128 arrivals)
+  uint64_t* o_done = p_ready + 1;       // [1] every MMA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int per = p.B * p.Hq;
+  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) / per;  // longest causal rows first
+  const int bh = static_cast<int>(blockIdx.x) % per;                   // b * Hq + h
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int q0 = qt * kBwdBM;
+  const int plane_kv = b * p.Hkv + h / p.G;
+  const int qmax = min(p.N - 1, q0 + kBwdBM - 1);
+  const int nkv = p.causal ? qmax / kBwdBN + 1 : p.n_ktiles;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(smem_u32(&kv_full[s]), 1);
+      mbar_init(smem_u32(&kv_empty[s]), 1);
+    }
+    mbar_init(smem_u32(s_full), 1);
+    mbar_init(smem_u32(p_ready), 128);
+    mbar_init(smem_u32(o_done), 1);
+    fence_barrier_init();
+  }
+  {
+    // zero the probe slots of [dO ; 0] (and of [Q ; R] when rho = 0): TMA writes only the other rows
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    const int n_tiles = HAS_R ? 1 : 2;
+    for (int i = threadIdx.x; i < n_tiles * Cfg::kCB * 4 * 16 * 8; i += kBwdThreads) {
+      const int c16 = i & 7, row = (i >> 3) & 15, w = (i >> 7) & 3, cb = (i >> 9) % Cfg::kCB,
+                t = (i >> 9) / Cfg::kCB;
+      const int base = (HAS_R || t == 1) ? Cfg::kOffDO : Cfg::kOffQR;
+      uint8_t* dst = smem + base + cb * Cfg::kBlock + (32 * w + 16 + row) * 128 + c16 * 16;
+      *reinterpret_cast<uint4*>(dst) = z;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == kBwdMmaWarp) {
+    tc::tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == kBwdTmaWarp) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      const int plane = bh;
+      {
+        const uint32_t fb = smem_u32(q_full);
+        mbar_arrive_expect_tx(fb, (HAS_R ? 3 : 2) * Cfg::kTileBytes / 2);
+#pragma unroll
+        for (int wq = 0; wq < 4; ++wq)
+#pragma unroll
+          for (int cb = 0; cb < Cfg::kCB; ++cb) {
+            const uint32_t off = cb * Cfg::kBlock + (32 * wq) * 128;
+            tma_load_3d(&qmap, smem_u32(smem + Cfg::kOffQR + off), fb, cb * 64, q0 + 16 * wq, plane);
+            if (HAS_R) tma_load_3d(&rmap, smem_u32(smem + Cfg::kOffQR + off + 16 * 128), fb, cb * 64, q0 + 16 * wq, plane);
+            tma_load_3d(&omap, smem_u32(smem + Cfg::kOffDO + off), fb, cb * 64, q0 + 16 * wq, plane);
+          }
+      }
+      int issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(smem_u32(&kv_empty[s]), ((j / NS) - 1) & 1, kErrBwdLoad)) { ok = false; break; }
+        const uint32_t fb = smem_u32(&kv_full[s]);
+        mbar_arrive_expect_tx(fb, 2 * Cfg::kTileBytes);
+#pragma unroll
+        for (int cb = 0; cb < Cfg::kCB; ++cb) {
+          tma_load_3d(&kmap, smem_u32(smem + Cfg::kOffK + s * Cfg::kTileBytes + cb * Cfg::kBlock), fb, cb * 64,
+                      j * kBwdBN, plane_kv);
+          tma_load_3d(&vmap, smem_u32(smem + Cfg::kOffV + s * Cfg::kTileBytes + cb * Cfg::kBlock), fb, cb * 64,
+                      j * kBwdBN, plane_kv);
+        }
+        issued = j + 1;
+      }
+      if (!ok) {  // let every issued load land before the CTA can exit
+        mbar_wait(smem_u32(q_full), 0, kErrBwdDrain);
+        for (int j = max(0, issued - NS); j < issued; ++j) mbar_wait(smem_u32(&kv_full[j % NS]), (j / NS) & 1, kErrBwdDrain);
+      }
+    }
+  } else if (warp == kBwdMmaWarp) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kBwdBN, 0, 0);  // [X;Y] x Z^T, both K-major
+      constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, 0, 1);       // [dA;dS] x K, K MN-major
+      constexpr uint64_t kStageStep = Cfg::kTileBytes >> 4;
+      const uint64_t d_qr = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffQR), 16, 1024);
+      const uint64_t d_do = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffDO), 16, 1024);
+      const uint64_t d_k = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffK), 16, 1024);
+      const uint64_t d_v = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffV), 16, 1024);
+      const uint64_t d_kmn = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffK), Cfg::kBlock, 1024);
+      ok = mbar_wait(smem_u32(q_full), 0, kErrBwdMma);
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int s = j % NS;
+        if (!mbar_wait(smem_u32(&kv_full[s]), (j / NS) & 1, kErrBwdMma)) { ok = false; break; }
+        tc::fence_after_sync();
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
+          tc::mma_ss(tmem + Cfg::kColS, d_qr + koff, d_k + s * kStageStep + koff, idesc_s, ks > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
+          tc::mma_ss(tmem + Cfg::kColG, d_do + koff, d_v + s * kStageStep + koff, idesc_s, ks > 0 ? 1u : 0u);
+        }
+        tc::commit(smem_u32(s_full));
+        if (!mbar_wait(smem_u32(p_ready), j & 1, kErrBwdMma)) { ok = false; break; }
+        tc::fence_after_sync();
+        // [dQ ; dR] += [scale dA ; dS] K: A = the bf16 pairs over S (128 keys = 64 columns)
+#pragma unroll
+        for (int kk = 0; kk < kBwdBN / 16; ++kk)
+          tc::mma_ts(tmem + Cfg::kColAcc, tmem + Cfg::kColS + 8 * kk,
+                     d_kmn + s * kStageStep + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+        tc::commit(smem_u32(&kv_empty[s]));
+      }
+      tc::commit(smem_u32(o_done));  // also on abort: every issued MMA completes before dealloc
+      mbar_wait(smem_u32(o_done), 0, kErrBwdMma);
+    }
+  } else {
+    // ================================================================ element-wise + epilogue
+    const int wq = warp;
+    const int c4 = lane & 3;
+    const int r_lo = lane >> 2;
+    const uint32_t lane_a = static_cast<uint32_t>(32 * wq) << 16;
+    const uint32_t lane_s = static_cast<uint32_t>(32 * wq + 16) << 16;
+    const uint32_t ta = tmem + lane_a + Cfg::kColS, ts = tmem + lane_s + Cfg::kColS;
+    const uint32_t tg = tmem + lane_a + Cfg::kColG;
+    const int q_lo = q0 + 16 * wq + r_lo, q_hi = q_lo + 8;
+    const size_t rb = static_cast<size_t>(bh) * p.N;
+    // per-row statistics (rows past N: lse = +inf gives w = 0)
+    float l2_lo = INFINITY, l2_hi = INFINITY, sb_lo = 0.f, sb_hi = 0.f, gb_lo = 0.f, gb_hi = 0.f, dd_lo = 0.f,
+          dd_hi = 0.f;
+    if (q_lo < p.N) {
+      l2_lo = p.lse[rb + q_lo] * kLog2e;
+      gb_lo = p.gbar[rb + q_lo];
+      dd_lo = p.dd[rb + q_lo];
+      if (HAS_R) sb_lo = p.sbar[rb + q_lo];
+    }
+    if (q_hi < p.N) {
+      l2_hi = p.lse[rb + q_hi] * kLog2e;
+      gb_hi = p.gbar[rb + q_hi];
+      dd_hi = p.dd[rb + q_hi];
+      if (HAS_R) sb_hi = p.sbar[rb + q_hi];
+    }
+    for (int j = 0; j < nkv; ++j) {
+      const bool landed = mbar_wait(smem_u32(s_full), j & 1, kErrBwdElem);
+      if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
+      tc::fence_after_sync();
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t ra[32], rs[32], rg[32];
+        tc::ld_16x256b_x8(ta + 64 * hf, ra);
+        tc::ld_16x256b_x8(ts + 64 * hf, rs);
+        tc::ld_16x256b_x8(tg + 64 * hf, rg);
+        tc::wait_ld();
+        // register i: rep gg = i/4, e = i%4; key = 128j + 64hf + 8gg + 2c4 + (e&1);
+        // row lo for e < 2, row hi for e >= 2
+        uint32_t pa[16], pd[16];
+#pragma unroll
+        for (int gg = 0; gg < 8; ++gg) {
+          float da[4], ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * gg + e;
+            const int key = j * kBwdBN + 64 * hf + 8 * gg + 2 * c4 + (e & 1);
+            const bool hi = (e & 2) != 0;
+            const int q = hi ? q_hi : q_lo;
+            const bool valid = key < p.N && (!p.causal || key <= q);
+            const float a = __uint_as_float(ra[i]), s = __uint_as_float(rs[i]), g = __uint_as_float(rg[i]);
+            const float w = valid ? ex2(fmaf(a, p.scale_log2, -(hi ? l2_hi : l2_lo))) : 0.f;
+            const float sb = hi ? sb_hi : sb_lo, gb = hi ? gb_hi : gb_lo, d2 = hi ? dd_hi : dd_lo;
+            ds[e] = w * (gb - g);
+            da[e] = p.scale * w * (fmaf(g, 1.f - s + sb, s * gb) - d2);
+          }
+          pa[2 * gg] = pack_bf16(da[0], da[1]);
+          pa[2 * gg + 1] = pack_bf16(da[2], da[3]);
+          pd[2 * gg] = pack_bf16(ds[0], ds[1]);
+          pd[2 * gg + 1] = pack_bf16(ds[2], ds[3]);
+        }
+        // bf16 pairs over the fp32 columns this thread has already read
+        // (half hf writes columns 32hf..32hf+31, inside the half-0 range)
+        tc::st_16x128b_x8(ta + 32 * hf, pa);
+        tc::st_16x128b_x8(ts + 32 * hf, pd);
+      }
+      tc::wait_st();
+      tc::fence_before_sync();
+      mbar_arrive(smem_u32(p_ready));
+    }
+    if (ok) {
+      const bool done = mbar_wait(smem_u32(o_done), 0, kErrBwdElem);
+      if (__all_sync(0xffffffffu, done)) {
+        tc::fence_after_sync();
+        const uint32_t t1 = tmem + lane_a + Cfg::kColAcc, t2 = tmem + lane_s + Cfg::kColAcc;
+        __nv_bfloat16* dq_row_lo = p.dq + (rb + q_lo) * D;
+        __nv_bfloat16* dq_row_hi = p.dq + (rb + q_hi) * D;
+        __nv_bfloat16* dr_row_lo = p.dr ? p.dr + (rb + q_lo) * D : nullptr;
+        __nv_bfloat16* dr_row_hi = p.dr ? p.dr + (rb + q_hi) * D : nullptr;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t o1[16], o2[16];
+          tc::ld_16x256b_x4(t1 + 32 * ch, o1);
+          tc::ld_16x256b_x4(t2 + 32 * ch, o2);
+          tc::wait_ld();
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg) {
+            const int col = 32 * ch + 8 * gg + 2 * c4;
+            if (q_lo < p.N) {
+              *reinterpret_cast<uint32_t*>(dq_row_lo + col) =
+                  pack_bf16(__uint_as_float(o1[4 * gg]), __uint_as_float(o1[4 * gg + 1]));
+              if (dr_row_lo)
+                *reinterpret_cast<uint32_t*>(dr_row_lo + col) =
+                    pack_bf16(__uint_as_float(o2[4 * gg]), __uint_as_float(o2[4 * gg + 1]));
+            }
+            if (q_hi < p.N) {
+              *reinterpret_cast<uint32_t*>(dq_row_hi + col) =
+                  pack_bf16(__uint_as_float(o1[4 * gg + 2]), __uint_as_float(o1[4 * gg + 3]));
+              if (dr_row_hi)
+                *reinterpret_cast<uint32_t*>(dr_row_hi + col) =
+                    pack_bf16(__uint_as_float(o2[4 * gg + 2]), __uint_as_float(o2[4 * gg + 3]));
+            }
+          }
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- dK, dV
+template <int D>
+struct BwdKVCfg {
+  static constexpr int kCB = D / 64;
+  static constexpr int kBlock = 128 * 128;        // [128 rows x 128 B]
+  static constexpr int kDOBlock = 64 * 128;       // [64 rows x 128 B]
+  static constexpr int kTileBytes = kCB * kBlock;  // K, V, [Q;R]
+  static constexpr int kDOBytes = kCB * kDOBlock;  // dO (64 rows)
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTileBytes;
+  static constexpr int kOffQR = 2 * kTileBytes;
+  static constexpr int kOffDO = kOffQR + kBwdStages * kTileBytes;
+  static constexpr int kOffStat = kOffDO + kBwdStages * kDOBytes;  // per warp: float4 per query of the tile
+  static constexpr int kOffBar = kOffStat + 4 * kBwdBM * 16;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  // tensor memory: [A^T | S^T] [0,128), G^T [128,192), W_hat^T [192,224), dK [256,256+D), dV [384 or 320, +D)
+  static constexpr uint32_t kColS = 0, kColG = 128, kColW = 192, kColDK = 256, kColDV = 256 + D;
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+template <int D, bool HAS_R>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap rmap,
+                  const __grid_constant__ CUtensorMap omap, const __grid_constant__ CUtensorMap kmap,
+                  const __grid_constant__ CUtensorMap vmap, const BwdParams p) {
+  using Cfg = BwdKVCfg<D>;
+  constexpr int NS = kBwdStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* kv_full = bars;             // [1] K and V of this CTA's key tile landed
+  uint64_t* q_full = bars + 1;          // [NS] [Q;R] and dO of a query tile landed
+  uint64_t* q_empty = q_full + NS;      // [NS]
+  uint64_t* s_full = q_empty + NS;      // [1] [A^T|S^T] and G^T in TMEM
+  uint64_t* p_ready = s_full + 1;       // [1] W_hat^T, dA^T, dS^T written (128 arrivals)
+  uint64_t* o_done = p_ready + 1;       // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int per = p.B * p.Hkv;
+  const int kt = static_cast<int>(blockIdx.x) / per;  // early key tiles see the most queries: first
+  const int bg = static_cast<int>(blockIdx.x) % per;  // b * Hkv + g
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int k0 = kt * kBwdBN;
+  const int qt0 = p.causal ? k0 / kBwdBM : 0;
+  const int n_qt = p.n_qtiles - qt0;
+  const int n_items = p.G * n_qt;  // (query head, query tile) pairs, head-major
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(kv_full), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(smem_u32(&q_full[s]), 1);
+      mbar_init(smem_u32(&q_empty[s]), 1);
+    }
+    mbar_init(smem_u32(s_full), 1);
+    mbar_init(smem_u32(p_ready), 128);
+    mbar_init(smem_u32(o_done), 1);
+    fence_barrier_init();
+  }
+  if (!HAS_R) {
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < NS * Cfg::kCB * 4 * 16 * 8; i += kBwdThreads) {
+      const int c16 = i & 7, row = (i >> 3) & 15, w = (i >> 7) & 3, cb = (i >> 9) % Cfg::kCB,
+                s = (i >> 9) / Cfg::kCB;
+      uint8_t* dst = smem + Cfg::kOffQR + s * Cfg::kTileBytes + cb * Cfg::kBlock + (32 * w + 16 + row) * 128 + c16 * 16;
+      *reinterpret_cast<uint4*>(dst) = z;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == kBwdMmaWarp) {
+    tc::tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == kBwdTmaWarp) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      {
+        const uint32_t fb = smem_u32(kv_full);
+        mbar_arrive_expect_tx(fb, 2 * Cfg::kTileBytes);
+#pragma unroll
+        for (int cb = 0; cb < Cfg::kCB; ++cb) {
+          tma_load_3d(&kmap, smem_u32(smem + Cfg::kOffK + cb * Cfg::kBlock), fb, cb * 64, k0, bg);
+          tma_load_3d(&vmap, smem_u32(smem + Cfg::kOffV + cb * Cfg::kBlock), fb, cb * 64, k0, bg);
+        }
+      }
+      int issued = 0;
+      for (int it = 0; it < n_items; ++it) {
+        const int s = it % NS;
+        if (it >= NS && !mbar_wait(smem_u32(&q_empty[s]), ((it / NS) - 1) & 1, kErrBwdLoad)) { ok = false; break; }
+        const int hq = g * p.G + it / n_qt;
+        const int q0 = (qt0 + it % n_qt) * kBwdBM;
+        const int plane = b * p.Hq + hq;
+        const uint32_t fb = smem_u32(&q_full[s]);
+        mbar_arrive_expect_tx(fb, (HAS_R ? 2 : 1) * Cfg::kTileBytes / 2 + Cfg::kDOBytes);
+        const uint32_t qr = smem_u32(smem + Cfg::kOffQR + s * Cfg::kTileBytes);
+        const uint32_t dob = smem_u32(smem + Cfg::kOffDO + s * Cfg::kDOBytes);
+#pragma unroll
+        for (int wq = 0; wq < 4; ++wq)
+#pragma unroll
+          for (int cb = 0; cb < Cfg::kCB; ++cb) {
+            const uint32_t dst = qr + cb * Cfg::kBlock + (32 * wq) * 128;
+            tma_load_3d(&qmap, dst, fb, cb * 64, q0 + 16 * wq, plane);
+            if (HAS_R) tma_load_3d(&rmap, dst + 16 * 128, fb, cb * 64, q0 + 16 * wq, plane);
+            tma_load_3d(&omap, dob + cb * Cfg::kDOBlock + (16 * wq) * 128, fb, cb * 64, q0 + 16 * wq, plane);
+          }
+        issued = it + 1;
+      }
+      if (!ok) {
+        mbar_wait(smem_u32(kv_full), 0, kErrBwdDrain);
+        for (int it = max(0, issued - NS); it < issued; ++it) mbar_wait(smem_u32(&q_full[it % NS]), (it / NS) & 1, kErrBwdDrain);
+      }
+    }
+  } else if (warp == kBwdMmaWarp) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, 0, 0);  // K [Q;R]^T
+      constexpr uint32_t idesc_g = tc::idesc_bf16_f32(128, kBwdBM, 0, 0);  // V dO^T
+      constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, 0, 1);   // X^T Y, Y MN-major
+      const uint64_t d_k = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffK), 16, 1024);
+      const uint64_t d_v = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffV), 16, 1024);
+      const uint64_t d_qr = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffQR), 16, 1024);
+      const uint64_t d_do = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffDO), 16, 1024);
+      const uint64_t d_qr_mn = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffQR), Cfg::kBlock, 1024);
+      const uint64_t d_do_mn = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffDO), Cfg::kDOBlock, 1024);
+      ok = mbar_wait(smem_u32(kv_full), 0, kErrBwdMma);
+      for (int it = 0; it < n_items && ok; ++it) {
+        const int s = it % NS;
+        if (!mbar_wait(smem_u32(&q_full[s]), (it / NS) & 1, kErrBwdMma)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint64_t qr_off = static_cast<uint64_t>(s) * (Cfg::kTileBytes >> 4);
+        const uint64_t do_off = static_cast<uint64_t>(s) * (Cfg::kDOBytes >> 4);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
+          tc::mma_ss(tmem + Cfg::kColS, d_k + koff, d_qr + qr_off + koff, idesc_s, ks > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t koff_a = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
+          const uint64_t koff_b = static_cast<uint64_t>(((ks >> 2) * Cfg::kDOBlock + (ks & 3) * 32) >> 4);
+          tc::mma_ss(tmem + Cfg::kColG, d_v + koff_a, d_do + do_off + koff_b, idesc_g, ks > 0 ? 1u : 0u);
+        }
+        tc::commit(smem_u32(s_full));
+        if (!mbar_wait(smem_u32(p_ready), it & 1, kErrBwdMma)) { ok = false; break; }
+        tc::fence_after_sync();
+        // dV += W_hat^T dO (K = 64 queries)
+#pragma unroll
+        for (int kk = 0; kk < kBwdBM / 16; ++kk)
+          tc::mma_ts(tmem + Cfg::kColDV, tmem + Cfg::kColW + 8 * kk,
+                     d_do_mn + do_off + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
+        // dK += [scale dA^T | dS^T] [Q ; R] (K = 128 stacked rows)
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          tc::mma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColS + 8 * kk,
+                     d_qr_mn + qr_off + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
+        tc::commit(smem_u32(&q_empty[s]));
+      }
+      tc::commit(smem_u32(o_done));
+      mbar_wait(smem_u32(o_done), 0, kErrBwdMma);
+    }
+  } else {
+    // ================================================================ element-wise + epilogue
+    // thread = key: TMEM lane 32 * warp + lane; columns are queries
+    const int wq = warp;
+    const int key = k0 + 32 * wq + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
+    const bool key_ok = key < p.N;
+    float4* stat = reinterpret_cast<float4*>(smem + Cfg::kOffStat) + wq * kBwdBM;  // this warp's copy
+    for (int it = 0; it < n_items; ++it) {
+      const int hq = g * p.G + it / n_qt;
+      const int q0 = (qt0 + it % n_qt) * kBwdBM;
+      const size_t rb = (static_cast<size_t>(b) * p.Hq + hq) * p.N;
+      // per-query statistics of this tile, one copy per warp (warp-level sync only)
+      __syncwarp();
+#pragma unroll
+      for (int u = 0; u < kBwdBM / 32; ++u) {
+        const int qi = lane + 32 * u;
+        const int q = q0 + qi;
+        float4 st4 = make_float4(INFINITY, 0.f, 0.f, 0.f);  // rows past N: w = 0
+        if (q < p.N) {
+          st4.x = p.lse[rb + q] * kLog2e;
+          st4.y = HAS_R ? p.sbar[rb + q] : 0.f;
+          st4.z = p.gbar[rb + q];
+          st4.w = p.dd[rb + q];
+        }
+        stat[qi] = st4;
+      }
+      __syncwarp();
+      const bool landed = mbar_wait(smem_u32(s_full), it & 1, kErrBwdElem);
+      if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
+      tc::fence_after_sync();
+      // 16 queries at a time: stacked columns 32w'..32w'+15 (q.k) and
+      // 32w'+16..32w'+31 (rho.k), G^T columns 16w'..16w'+15.  Outputs go to
+      // bf16 pair columns 16w'..16w'+15 of the score region (already read)
+      // and to W_hat^T pair columns 8w'..8w'+7.
+#pragma unroll 1
+      for (int wp = 0; wp < 4; ++wp) {
+        uint32_t ra[16], rs[16], rg[16];
+        tc::ld_32x32b_x16(tmem + lane_base + Cfg::kColS + 32 * wp, ra);
+        tc::ld_32x32b_x16(tmem + lane_base + Cfg::kColS + 32 * wp + 16, rs);
+        tc::ld_32x32b_x16(tmem + lane_base + Cfg::kColG + 16 * wp, rg);
+        tc::wait_ld();
+        uint32_t pw[8], pa[8], pd[8];
+#pragma unroll
+        for (int x = 0; x < 16; x += 2) {
+          float wh[2], da[2], ds[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int qi = 16 * wp + x + e;
+            const int q = q0 + qi;
+            const float4 st4 = stat[qi];
+            const bool valid = key_ok && (!p.causal || key <= q);
+            const float a = __uint_as_float(ra[x + e]), s = __uint_as_float(rs[x + e]), gv = __uint_as_float(rg[x + e]);
+            const float w = valid ? ex2(fmaf(a, p.scale_log2, -st4.x)) : 0.f;
+            const float f = 1.f - s + st4.y;
+            wh[e] = w * f;
+            ds[e] = w * (st4.z - gv);
+            da[e] = p.scale * w * (fmaf(gv, f, s * st4.z) - st4.w);
+          }
+          pw[x >> 1] = pack_bf16(wh[0], wh[1]);
+          pa[x >> 1] = pack_bf16(da[0], da[1]);
+          pd[x >> 1] = pack_bf16(ds[0], ds[1]);
+        }
+        tc::st_32x32b_x8(tmem + lane_base + Cfg::kColW + 8 * wp, pw);
+        tc::st_32x32b_x8(tmem + lane_base + Cfg::kColS + 16 * wp, pa);
+        tc::st_32x32b_x8(tmem + lane_base + Cfg::kColS + 16 * wp + 8, pd);
+      }
+      tc::wait_st();
+      tc::fence_before_sync();
+      mbar_arrive(smem_u32(p_ready));
+    }
+    if (ok) {
+      const bool done = mbar_wait(smem_u32(o_done), 0, kErrBwdElem);
+      if (__all_sync(0xffffffffu, done)) {
+        tc::fence_after_sync();
+        const size_t row = static_cast<size_t>(bg) * p.N + key;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t col = which == 0 ? Cfg::kColDK : Cfg::kColDV;
+          __nv_bfloat16* dst = (which == 0 ? p.dk : p.dv) + row * D;
+#pragma unroll
+          for (int ch = 0; ch < D / 16; ++ch) {
+            uint32_t v[16];
+            tc::ld_32x32b_x16(tmem + lane_base + col + 16 * ch, v);
+            tc::wait_ld();
+            if (key_ok) {
+              uint4 lo, hi;
+              lo.x = pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1]));
+              lo.y = pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3]));
+              lo.z = pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5]));
+              lo.w = pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7]));
+              hi.x = pack_bf16(__uint_as_float(v[8]), __uint_as_float(v[9]));
+              hi.y = pack_bf16(__uint_as_float(v[10]), __uint_as_float(v[11]));
+              hi.z = pack_bf16(__uint_as_float(v[12]), __uint_as_float(v[13]));
+              hi.w = pack_bf16(__uint_as_float(v[14]), __uint_as_float(v[15]));
+              *reinterpret_cast<uint4*>(dst + 16 * ch) = lo;
+              *reinterpret_cast<uint4*>(dst + 16 * ch + 8) = hi;
+            }
+          }
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace plx

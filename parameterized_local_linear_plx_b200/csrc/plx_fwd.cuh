@@ -88,13 +88,15 @@ struct FwdParams {
   int num_units;       // B * n_pairs * n_qblocks
   int causal;
   float scale_log2;    // scale * log2(e)
+  float* sbar;         // [B, Hq, N] s_bar = c / l (training forward only)
 };
 
-template <int D, bool HAS_R>
+template <int D, bool HAS_R, bool SAVE_AUX>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap rmap,
                const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-               const __grid_constant__ CUtensorMap omap, const FwdParams p) {
+               const __grid_constant__ CUtensorMap omap, const __grid_constant__ CUtensorMap amap,
+               const FwdParams p) {
   using Cfg = FwdCfg<D>;
   constexpr int NS = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -521,9 +523,11 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                        "r"(pack_bf16(r[2], r[3])) : "memory");
         }
       }
-      // O has been read: the next unit's first value MMA may overwrite it
-      tc::fence_before_sync();
-      mbar_arrive(smem_u32(&o_free[t]));
+      if (!SAVE_AUX) {
+        // O has been read: the next unit's first value MMA may overwrite it
+        tc::fence_before_sync();
+        mbar_arrive(smem_u32(&o_free[t]));
+      }
       if (p.lse && c4 == 0) {
         if (q_lo < p.N) p.lse[plane * p.N + q_lo] = l_lo > 0.f ? (m_lo + __log2f(l_lo)) * kLn2 : -INFINITY;
         if (q_hi < p.N) p.lse[plane * p.N + q_hi] = l_hi > 0.f ? (m_hi + __log2f(l_hi)) * kLn2 : -INFINITY;
@@ -535,6 +539,44 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 #pragma unroll
         for (int cb = 0; cb < Cfg::kCB; ++cb) tma_store_3d(&omap, stage + cb * 2048, cb * 64, row0, static_cast<int>(plane));
         bulk_commit();
+      }
+      if (SAVE_AUX) {
+        // Training forward: keep s_bar = c / l and o_bar = O1 / l (the softmax
+        // output) for the backward.  o_bar goes through the same staging
+        // block once the output store has read it.
+        if (p.sbar && c4 == 0) {
+          if (q_lo < p.N) p.sbar[plane * p.N + q_lo] = sb_lo;
+          if (q_hi < p.N) p.sbar[plane * p.N + q_hi] = sb_hi;
+        }
+        if (lane == 0) bulk_wait_read();
+        __syncwarp();
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t o1[16];
+          tc::ld_16x256b_x4(to1 + 32 * ch, o1);
+          tc::wait_ld();
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg) {
+            const int dcol = 32 * ch + 8 * gg + 2 * c4;
+            const int cb = dcol >> 6, chunk = (dcol & 63) >> 3;
+            const uint32_t blk = stage + cb * 2048 + 4 * c4;
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(blk + r_lo * 128 + ((chunk ^ (r_lo & 7)) << 4)),
+                         "r"(pack_bf16(__uint_as_float(o1[4 * gg]) * inv_lo, __uint_as_float(o1[4 * gg + 1]) * inv_lo))
+                         : "memory");
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(blk + r_hi * 128 + ((chunk ^ (r_hi & 7)) << 4)),
+                         "r"(pack_bf16(__uint_as_float(o1[4 * gg + 2]) * inv_hi, __uint_as_float(o1[4 * gg + 3]) * inv_hi))
+                         : "memory");
+          }
+        }
+        tc::fence_before_sync();
+        mbar_arrive(smem_u32(&o_free[t]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < p.N) {
+#pragma unroll
+          for (int cb = 0; cb < Cfg::kCB; ++cb) tma_store_3d(&amap, stage + cb * 2048, cb * 64, row0, static_cast<int>(plane));
+          bulk_commit();
+        }
       }
       kv += w.nkv;
     }

@@ -30,6 +30,10 @@ enum : unsigned {
   kErrFwdMma = 0x202u,        // prefill MMA warp
   kErrFwdSoftmax = 0x203u,    // prefill softmax warps
   kErrFwdDrain = 0x204u,      // prefill load warp draining after an abort
+  kErrBwdLoad = 0x301u,       // backward load warp
+  kErrBwdMma = 0x302u,        // backward MMA warp
+  kErrBwdElem = 0x303u,       // backward element-wise warps
+  kErrBwdDrain = 0x304u,      // backward load warp draining after an abort
   kErrSelftest = 0x901u,      // the deliberate self-test wait
 };
 

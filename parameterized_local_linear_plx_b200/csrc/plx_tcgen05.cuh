@@ -149,6 +149,23 @@ __device__ __forceinline__ void st_16x128b_x8(uint32_t taddr, const uint32_t (&r
       : "memory");
 }
 
+// 32 lanes x 32 bits, 16 repetitions: thread t holds lane (base + t), columns
+// c .. c+15 of the address in registers 0..15.
+__device__ __forceinline__ void ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : PLX_R8(0), PLX_R8(8)
+      : "r"(taddr));
+}
+
+// 32 lanes x 32 bits, 8 repetitions: thread t writes lane (base + t), columns c .. c+7.
+__device__ __forceinline__ void st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               PLX_W8(0)
+               : "memory");
+}
+
 #undef PLX_R8
 #undef PLX_W8
 

@@ -33,6 +33,12 @@ _lib.plx_status_string.restype = ctypes.c_char_p
 _lib.plx_status_string.argtypes = [_I]
 _lib.plx_fwd.restype = _I
 _lib.plx_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
+_lib.plx_fwd_train.restype = _I
+_lib.plx_fwd_train.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
+_lib.plx_bwd_workspace_size.restype = _SZ
+_lib.plx_bwd_workspace_size.argtypes = [_I, _I, _I, _I, _I]
+_lib.plx_bwd.restype = _I
+_lib.plx_bwd.argtypes = [_P] * 13 + [_I, _I, _I, _I, _I, _I, _F, _P, _SZ, _P]
 _lib.plx_decode_num_splits.restype = _I
 _lib.plx_decode_num_splits.argtypes = [_I, _I, _I, _I, _I]
 _lib.plx_decode_workspace_size.restype = _SZ
@@ -124,6 +130,73 @@ def plx_fwd(q, k, v, r=None, causal=True, scale=None, out=None, lse=None, return
     if st != PLX_OK:
         raise PlxError(st, "plx_fwd")
     return out, lse
+
+
+def plx_fwd_train(q, k, v, r=None, causal=True, scale=None, out=None, lse=None, obar=None, sbar=None,
+                  stream=None):
+    """plx_fwd that also returns the per-row values the backward needs.
+    Returns (out, lse, obar [B, Hq, N, d] bf16, sbar [B, Hq, N] fp32 or None when r is None)."""
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    if r is not None:
+        _check(r, "r", torch.bfloat16, 4)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape or (r is not None and r.shape != q.shape):
+        raise ValueError("shape mismatch between q, k, v, r")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    obar = torch.empty_like(q) if obar is None else obar
+    if r is not None and sbar is None:
+        sbar = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
+    st = _lib.plx_fwd_train(_ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(out), _ptr(lse), _ptr(obar),
+                            _ptr(sbar if r is not None else None), B, Hq, Hkv, N, d, 1 if causal else 0,
+                            float(scale), _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_fwd_train")
+    return out, lse, obar, (sbar if r is not None else None)
+
+
+def plx_bwd_workspace_size(B, Hq, Hkv, N, d) -> int:
+    return int(_lib.plx_bwd_workspace_size(B, Hq, Hkv, N, d))
+
+
+def plx_bwd(q, k, v, r, out, dout, lse, obar, sbar=None, causal=True, scale=None, dq=None, dk=None, dv=None,
+            dr=None, want_dr=True, workspace=None, stream=None):
+    """Gradients of sum(dout * out) for the forward of plx_fwd_train with the same
+    arguments.  Returns (dq, dk, dv, dr); dr is None when want_dr is False."""
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout"), (obar, "obar")):
+        _check(t, name, torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    if r is not None:
+        _check(r, "r", torch.bfloat16, 4)
+        _check(sbar, "sbar", torch.float32, 3)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if (k.shape != (B, Hkv, N, d) or v.shape != k.shape or out.shape != q.shape or dout.shape != q.shape
+            or obar.shape != q.shape or lse.shape != (B, Hq, N) or (r is not None and r.shape != q.shape)):
+        raise ValueError("shape mismatch between the backward's arguments")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if want_dr and dr is None:
+        dr = torch.empty_like(q)
+    need = plx_bwd_workspace_size(B, Hq, Hkv, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _lib.plx_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(out), _ptr(dout), _ptr(lse), _ptr(obar),
+                      _ptr(sbar if r is not None else None), _ptr(dq), _ptr(dk), _ptr(dv),
+                      _ptr(dr if want_dr else None), B, Hq, Hkv, N, d, 1 if causal else 0, float(scale),
+                      _ptr(workspace), ws_bytes, _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_bwd")
+    return dq, dk, dv, (dr if want_dr else None)
 
 
 def plx_decode_num_splits(B, Hq, Hkv, S_max, d) -> int:

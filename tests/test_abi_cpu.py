@@ -27,7 +27,8 @@ def declared_entry_points():
 
 def test_header_declares_the_boundary():
     names = declared_entry_points()
-    for n in ["plx_fwd", "plx_decode", "plx_decode_workspace_size", "plx_decode_num_splits",
+    for n in ["plx_fwd", "plx_fwd_train", "plx_bwd", "plx_bwd_workspace_size",
+              "plx_decode", "plx_decode_workspace_size", "plx_decode_num_splits",
               "plx_check_device_status", "plx_status_string", "plx_version", "plx_selftest_wait_timeout"]:
         assert n in names
 
@@ -117,3 +118,50 @@ def test_split_planning(plx):
     # bad shapes: count 1, size 0
     assert plx.plx_decode_num_splits(0, 16, 8, 4096, 128) == 1
     assert plx.plx_decode_workspace_size(1, 3, 2, 128, 128, 2) == 0
+
+
+def fwdt(plx, q=A, k=A, v=A, r=A, out=A, lse=A, obar=A, sbar=A, B=1, Hq=2, Hkv=1, N=8, d=64):
+    return plx.lib.plx_fwd_train(P(q), P(k), P(v), P(r), P(out), P(lse), P(obar), P(sbar), B, Hq, Hkv, N, d, 1,
+                                 0.125, None)
+
+
+def bwd(plx, ws=A, wsb=None, B=1, Hq=2, Hkv=1, N=8, d=64, **ptrs):
+    names = ["q", "k", "v", "r", "out", "dout", "lse", "obar", "sbar", "dq", "dk", "dv", "dr"]
+    vals = [P(ptrs.get(n, A)) for n in names]
+    if wsb is None:
+        wsb = plx.plx_bwd_workspace_size(B, Hq, Hkv, N, d)
+    return plx.lib.plx_bwd(*vals, B, Hq, Hkv, N, d, 1, 0.125, P(ws), wsb, None)
+
+
+def test_train_forward_argument_errors(plx):
+    assert fwdt(plx, lse=None) == plx.PLX_ERR_NULL
+    assert fwdt(plx, obar=None) == plx.PLX_ERR_NULL
+    assert fwdt(plx, sbar=None) == plx.PLX_ERR_NULL          # rho given: s_bar required
+    assert fwdt(plx, q=None) == plx.PLX_ERR_NULL
+    assert fwdt(plx, N=0) == plx.PLX_ERR_SHAPE
+    assert fwdt(plx, d=80) == plx.PLX_ERR_HEADDIM
+    assert fwdt(plx, obar=A + 8) == plx.PLX_ERR_ALIGN
+    assert fwdt(plx, sbar=A + 1) == plx.PLX_ERR_ALIGN
+
+
+def test_bwd_workspace_size(plx):
+    # two fp32 arrays of B * Hq * N, each padded to 256 bytes
+    assert plx.plx_bwd_workspace_size(2, 4, 2, 100, 128) == 2 * 3328
+    assert plx.plx_bwd_workspace_size(1, 1, 1, 64, 64) == 2 * 256
+    assert plx.plx_bwd_workspace_size(0, 4, 2, 100, 128) == 0
+    assert plx.plx_bwd_workspace_size(1, 3, 2, 100, 128) == 0
+    assert plx.plx_bwd_workspace_size(1, 4, 2, 100, 96) == 0
+
+
+def test_bwd_argument_errors(plx):
+    for n in ["q", "k", "v", "out", "dout", "lse", "obar", "dq", "dk", "dv"]:
+        assert bwd(plx, **{n: None}) == plx.PLX_ERR_NULL, n
+    assert bwd(plx, sbar=None) == plx.PLX_ERR_NULL           # rho given: s_bar required
+    assert bwd(plx, N=0) == plx.PLX_ERR_SHAPE
+    assert bwd(plx, d=32) == plx.PLX_ERR_HEADDIM
+    assert bwd(plx, Hq=3, Hkv=2) == plx.PLX_ERR_GQA
+    assert bwd(plx, dk=A + 8) == plx.PLX_ERR_ALIGN
+    assert bwd(plx, dr=A + 8) == plx.PLX_ERR_ALIGN
+    assert bwd(plx, lse=A + 2) == plx.PLX_ERR_ALIGN
+    assert bwd(plx, ws=None) == plx.PLX_ERR_WORKSPACE
+    assert bwd(plx, wsb=plx.plx_bwd_workspace_size(1, 2, 1, 8, 64) - 1) == plx.PLX_ERR_WORKSPACE

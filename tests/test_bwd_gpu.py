@@ -1,0 +1,144 @@
+"""Training forward and backward on the GPU against the fp64 gradient oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import assert_close
+from parameterized_local_linear_plx_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+# Gradient tolerance: a CPU emulation of the kernels' rounding (bf16 W_hat,
+# scale*dA and dS operands, bf16 out / o_bar and bf16 results) gives a
+# relative L2 error of ~2.5e-3 and a max error of <= 5.5e-3 max|ref| on these
+# workloads (3.5e-3 and 4.3e-3 for peaked scores with a large probe); the
+# bounds below leave about 4x headroom.
+GRAD_REL_L2 = 1e-2
+GRAD_MAX_REL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def plx():
+    from parameterized_local_linear_plx_b200 import build
+    build.build()
+    from parameterized_local_linear_plx_b200 import plx as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def grad_close(got, ref, what):
+    got = got.float().cpu().numpy().astype(np.float64) if hasattr(got, "float") else np.asarray(got)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite"
+    err = np.abs(got - ref)
+    scale = max(1.0, float(np.abs(ref).max()))
+    assert err.max() <= GRAD_MAX_REL * scale, f"{what}: max err {err.max():.3e} > {GRAD_MAX_REL * scale:.3e}"
+    # the relative bound needs a reference that is not ~0 (one causal key, for
+    # instance, makes dq exactly 0: only the max bound applies there)
+    norm = float(np.linalg.norm(ref))
+    if norm > 1e-3 * np.sqrt(ref.size):
+        rel = float(np.linalg.norm(got - ref)) / norm
+        assert rel <= GRAD_REL_L2, f"{what}: rel L2 {rel:.3e} > {GRAD_REL_L2:.1e}"
+
+
+def make(B, Hq, Hkv, N, d, seed, r_scale=0.1, use_r=True, device="cpu"):
+    q, k, v, r = inputs.prefill_inputs(B, Hq, Hkv, N, d, seed=seed, r_scale=r_scale, device=device)
+    g = torch.Generator(device=device).manual_seed(seed + 7)
+    do = torch.randn(q.shape, generator=g, device=device).bfloat16()
+    return q, k, v, (r if use_r else None), do
+
+
+def run_bwd(plx, q, k, v, r, do, causal=True):
+    qc, kc, vc, doc = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    rc = None if r is None else r.cuda()
+    out, lse, obar, sbar = plx.plx_fwd_train(qc, kc, vc, rc, causal=causal)
+    grads = plx.plx_bwd(qc, kc, vc, rc, out, doc, lse, obar, sbar, causal=causal)
+    torch.cuda.synchronize()
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    return grads
+
+
+def check_grads(plx, B, Hq, Hkv, N, d, seed, causal=True, use_r=True, r_scale=0.1, what=""):
+    q, k, v, r, do = make(B, Hq, Hkv, N, d, seed, r_scale, use_r)
+    dq, dk, dv, dr = run_bwd(plx, q, k, v, r, do, causal)
+    ref = oracle.prefill_backward_closed(q, k, v, r, do, causal)
+    for got, want, name in zip((dq, dk, dv, dr), ref, ("dq", "dk", "dv", "dr")):
+        grad_close(got, want, f"{what} {name}")
+
+
+def test_train_forward_matches_forward_and_aux(plx):
+    """plx_fwd_train writes the same out and lse as plx_fwd, plus o_bar (the
+    softmax output) and s_bar against the oracle."""
+    B, Hq, Hkv, N, d = 2, 4, 2, 333, 128
+    q, k, v, r, _ = make(B, Hq, Hkv, N, d, seed=3, device="cuda")
+    out0, lse0 = plx.plx_fwd(q, k, v, r)
+    out, lse, obar, sbar = plx.plx_fwd_train(q, k, v, r)
+    torch.cuda.synchronize()
+    assert torch.equal(out0, out) and torch.equal(lse0, lse)
+    ob, sb = oracle.prefill_aux(q.cpu(), k.cpu(), v.cpu(), r.cpu(), True)
+    assert np.abs(obar.float().cpu().numpy() - ob).max() <= 2e-2
+    assert np.abs(sbar.cpu().numpy() - sb).max() <= 1e-2
+
+
+def test_tiny_config_against_autograd(plx):
+    """B=1, H=1, N=256 (tiny config) with d=64: the GPU gradients against
+    autograd of the explicit-Sigma definition."""
+    q, k, v, r, do = make(1, 1, 1, 256, 64, seed=0)
+    dq, dk, dv, dr = run_bwd(plx, q, k, v, r, do)
+    ref = oracle.prefill_backward_autograd(q, k, v, r, do, True)
+    for got, want, name in zip((dq, dk, dv, dr), ref, ("dq", "dk", "dv", "dr")):
+        grad_close(got, want, f"tiny {name}")
+
+
+@pytest.mark.parametrize("N", [1, 2, 17, 64, 127, 128, 129, 200, 300])
+@pytest.mark.parametrize("causal", [True, False])
+def test_ragged_lengths(plx, N, causal):
+    check_grads(plx, 1, 2, 1, N, 64, seed=N, causal=causal, what=f"N={N} causal={causal}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(1, 1), (2, 1), (4, 2), (3, 1), (16, 8)])
+def test_heads_and_head_dims(plx, d, Hq, Hkv):
+    check_grads(plx, 2, Hq, Hkv, 333, d, seed=Hq * 10 + Hkv + d, what=f"d={d} Hq={Hq} Hkv={Hkv}")
+
+
+def test_rho_none_is_softmax_attention_backward(plx):
+    """r = NULL: dq, dk, dv are softmax attention's gradients (dr is the
+    gradient at rho = 0)."""
+    check_grads(plx, 2, 4, 2, 300, 128, seed=31, use_r=False, what="rho=0")
+
+
+def test_stress_inputs(plx):
+    """Peaked scores (q x 4) and a large probe (rho ~ N(0,1))."""
+    q, k, v, r, do = make(1, 2, 1, 512, 128, seed=33, r_scale=1.0)
+    q = (q.float() * 4).bfloat16()
+    dq, dk, dv, dr = run_bwd(plx, q, k, v, r, do)
+    ref = oracle.prefill_backward_closed(q, k, v, r, do, True)
+    for got, want, name in zip((dq, dk, dv, dr), ref, ("dq", "dk", "dv", "dr")):
+        grad_close(got, want, f"stress {name}")
+
+
+def test_pretraining_shape_full_size(plx):
+    """B=8, N=4096, Hq=16, Hkv=8, d=128, causal: the launch the benchmark
+    times.  Two whole KV groups (both query heads each) by the closed form:
+    dq, dr of those heads and dk, dv of those KV heads."""
+    B, Hq, Hkv, N, d = 8, 16, 8, 4096, 128
+    q, k, v, r, do = make(B, Hq, Hkv, N, d, seed=0, device="cuda")
+    out, lse, obar, sbar = plx.plx_fwd_train(q, k, v, r)
+    dq, dk, dv, dr = plx.plx_bwd(q, k, v, r, out, do, lse, obar, sbar)
+    torch.cuda.synchronize()
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    for t in (dq, dk, dv, dr):
+        assert torch.isfinite(t.float()).all()
+    for b, g in [(0, 0), (5, 6)]:
+        sl = slice(b, b + 1)
+        heads = [(0, 2 * g), (0, 2 * g + 1)]
+        ref = oracle.prefill_backward_closed(q[sl].cpu(), k[sl].cpu(), v[sl].cpu(), r[sl].cpu(), do[sl].cpu(), True,
+                                             heads=heads)
+        for h in (2 * g, 2 * g + 1):
+            grad_close(dq[b, h], ref[0][0, h], f"dq ({b},{h})")
+            grad_close(dr[b, h], ref[3][0, h], f"dr ({b},{h})")
+        grad_close(dk[b, g], ref[1][0, g], f"dk ({b},{g})")
+        grad_close(dv[b, g], ref[2][0, g], f"dv ({b},{g})")
