@@ -65,6 +65,14 @@ def prefill_flops(B, Hq, N, d, causal=True):
     return 8 * d * pairs * B * Hq
 
 
+def backward_flops(B, Hq, N, d, causal=True):
+    """16d per unmasked (query, key) pair: the products the gradient needs once
+    each -- QK^T and RK^T (recomputed scores), dO V^T, W_hat^T dO, dA^T Q and
+    dS^T R (dK), dA K (dQ) and dS K (dR), 2d each."""
+    pairs = N * (N + 1) // 2 if causal else N * N
+    return 16 * d * pairs * B * Hq
+
+
 def prefill_bytes(B, Hq, Hkv, N, d):
     return (3 * B * Hq + 2 * B * Hkv) * N * d * 2 + 4 * B * Hq * N
 
@@ -82,6 +90,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "prefill": ("plx_fwd.cuh", "plx_tcgen05.cuh", "plx_ptx.cuh"),
     "decode": ("plx_decode.cuh", "plx_ptx.cuh"),
+    "backward": ("plx_bwd.cuh", "plx_tcgen05.cuh", "plx_ptx.cuh"),
 }
 
 
@@ -402,6 +411,9 @@ def run_gpu(args, world, rank, local):
     # ---- end to end through the public API: pinned host buffers, copies timed
     e2e = run_e2e(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes)
 
+    # ---- training backward of the prefill shape (timed on its own; not part of the step)
+    bwd = run_backward(plx, args, dev, stream, world, local, pq, pk, pv, pr, peaks, peak_src)
+
     # ---- CPU baseline: the oracle on this host, rank 0, N=1 only
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -427,12 +439,73 @@ def run_gpu(args, world, rank, local):
             "roofline": roof_pre,
             "roofline_decode": roof_dec,
             "e2e": e2e,
+            "backward": bwd,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
     return 0
+
+
+def run_backward(plx, args, dev, stream, world, local, pq, pk, pv, pr, peaks, peak_src):
+    """plx_fwd_train then plx_bwd at the prefill shape (B=8, N=4096, causal),
+    dO ~ N(0, 1) bf16; CUDA events around each call, max over ranks."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(7 + local)
+    dout = torch.randn(pq.shape, generator=g, device=dev).bfloat16()
+    out = torch.empty_like(pq)
+    obar = torch.empty_like(pq)
+    lse = torch.empty(PRE["B"], PRE["Hq"], PRE["N"], dtype=torch.float32, device=dev)
+    sbar = torch.empty_like(lse)
+    dq, dr, dk, dv = torch.empty_like(pq), torch.empty_like(pq), torch.empty_like(pk), torch.empty_like(pv)
+    ws = torch.empty(plx.plx_bwd_workspace_size(PRE["B"], PRE["Hq"], PRE["Hkv"], PRE["N"], PRE["d"]),
+                     dtype=torch.uint8, device=dev)
+
+    def one(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        plx.plx_fwd_train(pq, pk, pv, pr, causal=True, out=out, lse=lse, obar=obar, sbar=sbar, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        plx.plx_bwd(pq, pk, pv, pr, out, dout, lse, obar, sbar, causal=True, dq=dq, dk=dk, dv=dv, dr=dr,
+                    workspace=ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        one()
+    torch.cuda.synchronize(dev)
+    steps = max(1, min(args.steps, 20))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(steps):
+            one(evs[i])
+        torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    st = plx.plx_check_device_status(stream)
+    if st != plx.PLX_OK:
+        raise RuntimeError(f"device status after the backward: {plx.plx_status_string(st)}")
+    fwd_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs) / steps, world, dev)
+    bwd_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in evs) / steps, world, dev)
+    b_flops = backward_flops(PRE["B"], PRE["Hq"], PRE["N"], PRE["d"], True)
+    f_flops = prefill_flops(PRE["B"], PRE["Hq"], PRE["N"], PRE["d"], True)
+    tf_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = b_flops / (bwd_ms * 1e-3) / 1e12
+    return {
+        "workload": f"training backward of the prefill shape B={PRE['B']} N={PRE['N']} Hq={PRE['Hq']} "
+                    f"Hkv={PRE['Hkv']} d={PRE['d']} causal; dO ~ N(0,1) bf16",
+        "tflops": world * achieved, "ms_per_step": bwd_ms, "flops_per_step": b_flops,
+        "fwd_train_ms": fwd_ms, "fwd_train_tflops": world * f_flops / (fwd_ms * 1e-3) / 1e12,
+        "steps": steps, "launches_per_step": 4,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
+                     "frac": achieved / tf_peak, "traffic": load_traffic("backward"),
+                     "kernel": "plx_bwd (pre + q-side + kv-side), per call",
+                     "peak_source": f"{peak_src} bf16_tflops"},
+        "clocks": clk.summary(),
+    }
 
 
 def run_e2e(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes):

@@ -33,9 +33,13 @@
 //     dV += W_hat^T dO and dK += [scale dA^T | dS^T] [Q;R] (the stacked tile is
 //     the K-major B of the first product and the MN-major B of the last).
 //     Each CTA owns its output rows: no atomics anywhere.
-//   * In both: warps 0-3 element-wise (warp w reads TMEM lanes 32w..32w+31),
-//     warp 4 issues the TMA loads, warp 5 allocates tensor memory and one of
-//     its threads issues every MMA.  Every wait is bounded (device error word).
+//   * In both: warps 0-15 element-wise.  Warp w reads TMEM lanes
+//     32(w%4)..32(w%4)+31 and one quarter (w/4) of the columns; every
+//     (key, query) element is independent, so the warps share nothing, and
+//     each writes its bf16 results over fp32 columns it has itself already
+//     read.  Warp 16 issues the TMA loads, warp 17 allocates tensor memory and
+//     one of its threads issues every MMA.  Every wait is bounded (device
+//     error word).
 #pragma once
 
 #include <cuda.h>
@@ -50,9 +54,10 @@ namespace plx {
 
 constexpr int kBwdBM = 64;        // queries per tile (128 stacked rows with their probes)
 constexpr int kBwdBN = 128;       // keys per tile
-constexpr int kBwdThreads = 192;  // 4 element-wise warps, TMA warp, MMA warp
-constexpr int kBwdTmaWarp = 4;
-constexpr int kBwdMmaWarp = 5;
+constexpr int kBwdElemWarps = 16;
+constexpr int kBwdThreads = 32 * (kBwdElemWarps + 2);  // element-wise warps, TMA warp, MMA warp
+constexpr int kBwdTmaWarp = kBwdElemWarps;
+constexpr int kBwdMmaWarp = kBwdElemWarps + 1;
 constexpr int kBwdStages = 2;
 
 struct BwdParams {
@@ -137,7 +142,7 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
   uint64_t* kv_full = bars + 1;         // [NS]
   uint64_t* kv_empty = kv_full + NS;    // [NS]
   uint64_t* s_full = kv_empty + NS;     // [1] S and G of the current key tile are in TMEM
-  uint64_t* p_ready = s_full + 1;       // [1] [dA ; dS] written (128 arrivals)
+  uint64_t* p_ready = s_full + 1;       // [1] [dA ; dS] written (every element-wise thread)
   uint64_t* o_done = p_ready + 1;       // [1] every MMA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
 
@@ -159,7 +164,7 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       mbar_init(smem_u32(&kv_empty[s]), 1);
     }
     mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(p_ready), 128);
+    mbar_init(smem_u32(p_ready), 32 * kBwdElemWarps);
     mbar_init(smem_u32(o_done), 1);
     fence_barrier_init();
   }
@@ -252,10 +257,11 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         tc::commit(smem_u32(s_full));
         if (!mbar_wait(smem_u32(p_ready), j & 1, kErrBwdMma)) { ok = false; break; }
         tc::fence_after_sync();
-        // [dQ ; dR] += [scale dA ; dS] K: A = the bf16 pairs over S (128 keys = 64 columns)
+        // [dQ ; dR] += [scale dA ; dS] K.  A: the bf16 pairs of keys 32c..32c+31
+        // sit in columns 32c..32c+15, so keys 16kk.. start at 32(kk/2) + 8(kk%2).
 #pragma unroll
         for (int kk = 0; kk < kBwdBN / 16; ++kk)
-          tc::mma_ts(tmem + Cfg::kColAcc, tmem + Cfg::kColS + 8 * kk,
+          tc::mma_ts(tmem + Cfg::kColAcc, tmem + Cfg::kColS + 32 * (kk >> 1) + 8 * (kk & 1),
                      d_kmn + s * kStageStep + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
                      (j > 0 || kk > 0) ? 1u : 0u);
         tc::commit(smem_u32(&kv_empty[s]));
@@ -265,13 +271,14 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     }
   } else {
     // ================================================================ element-wise + epilogue
-    const int wq = warp;
+    // warp (wq, part): rows of TMEM quadrant wq, keys 32part..32part+31 of each tile
+    const int wq = warp & 3, part = warp >> 2;
     const int c4 = lane & 3;
     const int r_lo = lane >> 2;
     const uint32_t lane_a = static_cast<uint32_t>(32 * wq) << 16;
     const uint32_t lane_s = static_cast<uint32_t>(32 * wq + 16) << 16;
-    const uint32_t ta = tmem + lane_a + Cfg::kColS, ts = tmem + lane_s + Cfg::kColS;
-    const uint32_t tg = tmem + lane_a + Cfg::kColG;
+    const uint32_t ta = tmem + lane_a + Cfg::kColS + 32 * part, ts = tmem + lane_s + Cfg::kColS + 32 * part;
+    const uint32_t tg = tmem + lane_a + Cfg::kColG + 32 * part;
     const int q_lo = q0 + 16 * wq + r_lo, q_hi = q_lo + 8;
     const size_t rb = static_cast<size_t>(bh) * p.N;
     // per-row statistics (rows past N: lse = +inf gives w = 0)
@@ -293,42 +300,38 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       const bool landed = mbar_wait(smem_u32(s_full), j & 1, kErrBwdElem);
       if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
       tc::fence_after_sync();
+      uint32_t ra[16], rs[16], rg[16];
+      tc::ld_16x256b_x4(ta, ra);
+      tc::ld_16x256b_x4(ts, rs);
+      tc::ld_16x256b_x4(tg, rg);
+      tc::wait_ld();
+      // register i: rep gg = i/4, e = i%4; key = 128j + 32part + 8gg + 2c4 + (e&1);
+      // row lo for e < 2, row hi for e >= 2
+      uint32_t pa[8], pd[8];
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t ra[32], rs[32], rg[32];
-        tc::ld_16x256b_x8(ta + 64 * hf, ra);
-        tc::ld_16x256b_x8(ts + 64 * hf, rs);
-        tc::ld_16x256b_x8(tg + 64 * hf, rg);
-        tc::wait_ld();
-        // register i: rep gg = i/4, e = i%4; key = 128j + 64hf + 8gg + 2c4 + (e&1);
-        // row lo for e < 2, row hi for e >= 2
-        uint32_t pa[16], pd[16];
+      for (int gg = 0; gg < 4; ++gg) {
+        float da[4], ds[4];
 #pragma unroll
-        for (int gg = 0; gg < 8; ++gg) {
-          float da[4], ds[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = 4 * gg + e;
-            const int key = j * kBwdBN + 64 * hf + 8 * gg + 2 * c4 + (e & 1);
-            const bool hi = (e & 2) != 0;
-            const int q = hi ? q_hi : q_lo;
-            const bool valid = key < p.N && (!p.causal || key <= q);
-            const float a = __uint_as_float(ra[i]), s = __uint_as_float(rs[i]), g = __uint_as_float(rg[i]);
-            const float w = valid ? ex2(fmaf(a, p.scale_log2, -(hi ? l2_hi : l2_lo))) : 0.f;
-            const float sb = hi ? sb_hi : sb_lo, gb = hi ? gb_hi : gb_lo, d2 = hi ? dd_hi : dd_lo;
-            ds[e] = w * (gb - g);
-            da[e] = p.scale * w * (fmaf(g, 1.f - s + sb, s * gb) - d2);
-          }
-          pa[2 * gg] = pack_bf16(da[0], da[1]);
-          pa[2 * gg + 1] = pack_bf16(da[2], da[3]);
-          pd[2 * gg] = pack_bf16(ds[0], ds[1]);
-          pd[2 * gg + 1] = pack_bf16(ds[2], ds[3]);
+        for (int e = 0; e < 4; ++e) {
+          const int i = 4 * gg + e;
+          const int key = j * kBwdBN + 32 * part + 8 * gg + 2 * c4 + (e & 1);
+          const bool hi = (e & 2) != 0;
+          const int q = hi ? q_hi : q_lo;
+          const bool valid = key < p.N && (!p.causal || key <= q);
+          const float a = __uint_as_float(ra[i]), s = __uint_as_float(rs[i]), g = __uint_as_float(rg[i]);
+          const float w = valid ? ex2(fmaf(a, p.scale_log2, -(hi ? l2_hi : l2_lo))) : 0.f;
+          const float sb = hi ? sb_hi : sb_lo, gb = hi ? gb_hi : gb_lo, d2 = hi ? dd_hi : dd_lo;
+          ds[e] = w * (gb - g);
+          da[e] = p.scale * w * (fmaf(g, 1.f - s + sb, s * gb) - d2);
         }
-        // bf16 pairs over the fp32 columns this thread has already read
-        // (half hf writes columns 32hf..32hf+31, inside the half-0 range)
-        tc::st_16x128b_x8(ta + 32 * hf, pa);
-        tc::st_16x128b_x8(ts + 32 * hf, pd);
+        pa[2 * gg] = pack_bf16(da[0], da[1]);
+        pa[2 * gg + 1] = pack_bf16(da[2], da[3]);
+        pd[2 * gg] = pack_bf16(ds[0], ds[1]);
+        pd[2 * gg + 1] = pack_bf16(ds[2], ds[3]);
       }
+      // bf16 pairs over the first 16 of this warp's own 32 fp32 columns
+      tc::st_16x128b_x4(ta, pa);
+      tc::st_16x128b_x4(ts, pd);
       tc::wait_st();
       tc::fence_before_sync();
       mbar_arrive(smem_u32(p_ready));
@@ -337,32 +340,30 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       const bool done = mbar_wait(smem_u32(o_done), 0, kErrBwdElem);
       if (__all_sync(0xffffffffu, done)) {
         tc::fence_after_sync();
+        // this warp's quarter of the columns: [part * D/4, (part + 1) * D/4)
         const uint32_t t1 = tmem + lane_a + Cfg::kColAcc, t2 = tmem + lane_s + Cfg::kColAcc;
-        __nv_bfloat16* dq_row_lo = p.dq + (rb + q_lo) * D;
-        __nv_bfloat16* dq_row_hi = p.dq + (rb + q_hi) * D;
-        __nv_bfloat16* dr_row_lo = p.dr ? p.dr + (rb + q_lo) * D : nullptr;
-        __nv_bfloat16* dr_row_hi = p.dr ? p.dr + (rb + q_hi) * D : nullptr;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t o1[16], o2[16];
-          tc::ld_16x256b_x4(t1 + 32 * ch, o1);
-          tc::ld_16x256b_x4(t2 + 32 * ch, o2);
+        for (int ch = 0; ch < D / 64; ++ch) {
+          const int cbase = part * (D / 4) + 16 * ch;
+          uint32_t o1[8], o2[8];
+          tc::ld_16x256b_x2(t1 + cbase, o1);
+          tc::ld_16x256b_x2(t2 + cbase, o2);
           tc::wait_ld();
 #pragma unroll
-          for (int gg = 0; gg < 4; ++gg) {
-            const int col = 32 * ch + 8 * gg + 2 * c4;
+          for (int gg = 0; gg < 2; ++gg) {
+            const int col = cbase + 8 * gg + 2 * c4;
             if (q_lo < p.N) {
-              *reinterpret_cast<uint32_t*>(dq_row_lo + col) =
+              *reinterpret_cast<uint32_t*>(p.dq + (rb + q_lo) * D + col) =
                   pack_bf16(__uint_as_float(o1[4 * gg]), __uint_as_float(o1[4 * gg + 1]));
-              if (dr_row_lo)
-                *reinterpret_cast<uint32_t*>(dr_row_lo + col) =
+              if (p.dr)
+                *reinterpret_cast<uint32_t*>(p.dr + (rb + q_lo) * D + col) =
                     pack_bf16(__uint_as_float(o2[4 * gg]), __uint_as_float(o2[4 * gg + 1]));
             }
             if (q_hi < p.N) {
-              *reinterpret_cast<uint32_t*>(dq_row_hi + col) =
+              *reinterpret_cast<uint32_t*>(p.dq + (rb + q_hi) * D + col) =
                   pack_bf16(__uint_as_float(o1[4 * gg + 2]), __uint_as_float(o1[4 * gg + 3]));
-              if (dr_row_hi)
-                *reinterpret_cast<uint32_t*>(dr_row_hi + col) =
+              if (p.dr)
+                *reinterpret_cast<uint32_t*>(p.dr + (rb + q_hi) * D + col) =
                     pack_bf16(__uint_as_float(o2[4 * gg + 2]), __uint_as_float(o2[4 * gg + 3]));
             }
           }
@@ -390,11 +391,12 @@ struct BwdKVCfg {
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQR = 2 * kTileBytes;
   static constexpr int kOffDO = kOffQR + kBwdStages * kTileBytes;
-  static constexpr int kOffStat = kOffDO + kBwdStages * kDOBytes;  // per warp: float4 per query of the tile
-  static constexpr int kOffBar = kOffStat + 4 * kBwdBM * 16;
+  static constexpr int kOffStat = kOffDO + kBwdStages * kDOBytes;  // per warp: float4 per query of its 16
+  static constexpr int kOffBar = kOffStat + kBwdElemWarps * 16 * 16;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
-  // tensor memory: [A^T | S^T] [0,128), G^T [128,192), W_hat^T [192,224), dK [256,256+D), dV [384 or 320, +D)
-  static constexpr uint32_t kColS = 0, kColG = 128, kColW = 192, kColDK = 256, kColDV = 256 + D;
+  // tensor memory: [A^T | S^T] [0,128), G^T [128,192), dK [256,256+D), dV [256+D, 256+2D).
+  // bf16 results: scale dA^T and dS^T over the score columns, W_hat^T over G^T.
+  static constexpr uint32_t kColS = 0, kColG = 128, kColDK = 256, kColDV = 256 + D;
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -412,7 +414,7 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* q_full = bars + 1;          // [NS] [Q;R] and dO of a query tile landed
   uint64_t* q_empty = q_full + NS;      // [NS]
   uint64_t* s_full = q_empty + NS;      // [1] [A^T|S^T] and G^T in TMEM
-  uint64_t* p_ready = s_full + 1;       // [1] W_hat^T, dA^T, dS^T written (128 arrivals)
+  uint64_t* p_ready = s_full + 1;       // [1] W_hat^T, dA^T, dS^T written (every element-wise thread)
   uint64_t* o_done = p_ready + 1;       // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
 
@@ -434,7 +436,7 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       mbar_init(smem_u32(&q_empty[s]), 1);
     }
     mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(p_ready), 128);
+    mbar_init(smem_u32(p_ready), 32 * kBwdElemWarps);
     mbar_init(smem_u32(o_done), 1);
     fence_barrier_init();
   }
@@ -530,15 +532,16 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         tc::commit(smem_u32(s_full));
         if (!mbar_wait(smem_u32(p_ready), it & 1, kErrBwdMma)) { ok = false; break; }
         tc::fence_after_sync();
-        // dV += W_hat^T dO (K = 64 queries)
+        // dV += W_hat^T dO (K = 64 queries; the pairs of queries 16kk.. sit at G^T column 16kk)
 #pragma unroll
         for (int kk = 0; kk < kBwdBM / 16; ++kk)
-          tc::mma_ts(tmem + Cfg::kColDV, tmem + Cfg::kColW + 8 * kk,
+          tc::mma_ts(tmem + Cfg::kColDV, tmem + Cfg::kColG + 16 * kk,
                      d_do_mn + do_off + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
-        // dK += [scale dA^T | dS^T] [Q ; R] (K = 128 stacked rows)
+        // dK += [scale dA^T | dS^T] [Q ; R] (K = 128 stacked rows; the pairs of
+        // stacked rows 32c..32c+15 sit at column 32c, of rows 32c+16.. at 32c+8)
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          tc::mma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColS + 8 * kk,
+          tc::mma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColS + 32 * (kk >> 1) + 8 * (kk & 1),
                      d_qr_mn + qr_off + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
         tc::commit(smem_u32(&q_empty[s]));
       }
@@ -547,22 +550,20 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     }
   } else {
     // ================================================================ element-wise + epilogue
-    // thread = key: TMEM lane 32 * warp + lane; columns are queries
-    const int wq = warp;
+    // warp (wq, wp): keys 32wq..32wq+31 of the tile (thread = key: TMEM lane
+    // 32wq + lane), queries 16wp..16wp+15 of each query tile
+    const int wq = warp & 3, wp = warp >> 2;
     const int key = k0 + 32 * wq + lane;
     const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
     const bool key_ok = key < p.N;
-    float4* stat = reinterpret_cast<float4*>(smem + Cfg::kOffStat) + wq * kBwdBM;  // this warp's copy
+    float4* stat = reinterpret_cast<float4*>(smem + Cfg::kOffStat) + warp * 16;  // this warp's 16 queries
     for (int it = 0; it < n_items; ++it) {
       const int hq = g * p.G + it / n_qt;
-      const int q0 = (qt0 + it % n_qt) * kBwdBM;
+      const int q0 = (qt0 + it % n_qt) * kBwdBM + 16 * wp;  // first of this warp's queries
       const size_t rb = (static_cast<size_t>(b) * p.Hq + hq) * p.N;
-      // per-query statistics of this tile, one copy per warp (warp-level sync only)
       __syncwarp();
-#pragma unroll
-      for (int u = 0; u < kBwdBM / 32; ++u) {
-        const int qi = lane + 32 * u;
-        const int q = q0 + qi;
+      if (lane < 16) {
+        const int q = q0 + lane;
         float4 st4 = make_float4(INFINITY, 0.f, 0.f, 0.f);  // rows past N: w = 0
         if (q < p.N) {
           st4.x = p.lse[rb + q] * kLog2e;
@@ -570,48 +571,44 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           st4.z = p.gbar[rb + q];
           st4.w = p.dd[rb + q];
         }
-        stat[qi] = st4;
+        stat[lane] = st4;
       }
       __syncwarp();
       const bool landed = mbar_wait(smem_u32(s_full), it & 1, kErrBwdElem);
       if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
       tc::fence_after_sync();
-      // 16 queries at a time: stacked columns 32w'..32w'+15 (q.k) and
-      // 32w'+16..32w'+31 (rho.k), G^T columns 16w'..16w'+15.  Outputs go to
-      // bf16 pair columns 16w'..16w'+15 of the score region (already read)
-      // and to W_hat^T pair columns 8w'..8w'+7.
-#pragma unroll 1
-      for (int wp = 0; wp < 4; ++wp) {
-        uint32_t ra[16], rs[16], rg[16];
-        tc::ld_32x32b_x16(tmem + lane_base + Cfg::kColS + 32 * wp, ra);
-        tc::ld_32x32b_x16(tmem + lane_base + Cfg::kColS + 32 * wp + 16, rs);
-        tc::ld_32x32b_x16(tmem + lane_base + Cfg::kColG + 16 * wp, rg);
-        tc::wait_ld();
-        uint32_t pw[8], pa[8], pd[8];
+      // stacked columns 32wp..32wp+15 (q.k) and 32wp+16..32wp+31 (rho.k), G^T columns 16wp..16wp+15
+      const uint32_t tsa = tmem + lane_base + Cfg::kColS + 32 * wp;
+      const uint32_t tgw = tmem + lane_base + Cfg::kColG + 16 * wp;
+      uint32_t ra[16], rs[16], rg[16];
+      tc::ld_32x32b_x16(tsa, ra);
+      tc::ld_32x32b_x16(tsa + 16, rs);
+      tc::ld_32x32b_x16(tgw, rg);
+      tc::wait_ld();
+      uint32_t pw[8], pa[8], pd[8];
 #pragma unroll
-        for (int x = 0; x < 16; x += 2) {
-          float wh[2], da[2], ds[2];
+      for (int x = 0; x < 16; x += 2) {
+        float wh[2], da[2], ds[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int qi = 16 * wp + x + e;
-            const int q = q0 + qi;
-            const float4 st4 = stat[qi];
-            const bool valid = key_ok && (!p.causal || key <= q);
-            const float a = __uint_as_float(ra[x + e]), s = __uint_as_float(rs[x + e]), gv = __uint_as_float(rg[x + e]);
-            const float w = valid ? ex2(fmaf(a, p.scale_log2, -st4.x)) : 0.f;
-            const float f = 1.f - s + st4.y;
-            wh[e] = w * f;
-            ds[e] = w * (st4.z - gv);
-            da[e] = p.scale * w * (fmaf(gv, f, s * st4.z) - st4.w);
-          }
-          pw[x >> 1] = pack_bf16(wh[0], wh[1]);
-          pa[x >> 1] = pack_bf16(da[0], da[1]);
-          pd[x >> 1] = pack_bf16(ds[0], ds[1]);
+        for (int e = 0; e < 2; ++e) {
+          const int q = q0 + x + e;
+          const float4 st4 = stat[x + e];
+          const bool valid = key_ok && (!p.causal || key <= q);
+          const float a = __uint_as_float(ra[x + e]), s = __uint_as_float(rs[x + e]), gv = __uint_as_float(rg[x + e]);
+          const float w = valid ? ex2(fmaf(a, p.scale_log2, -st4.x)) : 0.f;
+          const float fct = 1.f - s + st4.y;
+          wh[e] = w * fct;
+          ds[e] = w * (st4.z - gv);
+          da[e] = p.scale * w * (fmaf(gv, fct, s * st4.z) - st4.w);
         }
-        tc::st_32x32b_x8(tmem + lane_base + Cfg::kColW + 8 * wp, pw);
-        tc::st_32x32b_x8(tmem + lane_base + Cfg::kColS + 16 * wp, pa);
-        tc::st_32x32b_x8(tmem + lane_base + Cfg::kColS + 16 * wp + 8, pd);
+        pw[x >> 1] = pack_bf16(wh[0], wh[1]);
+        pa[x >> 1] = pack_bf16(da[0], da[1]);
+        pd[x >> 1] = pack_bf16(ds[0], ds[1]);
       }
+      // bf16 pairs over this warp's own fp32 columns (already read)
+      tc::st_32x32b_x8(tgw, pw);
+      tc::st_32x32b_x8(tsa, pa);
+      tc::st_32x32b_x8(tsa + 8, pd);
       tc::wait_st();
       tc::fence_before_sync();
       mbar_arrive(smem_u32(p_ready));
@@ -621,14 +618,16 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       if (__all_sync(0xffffffffu, done)) {
         tc::fence_after_sync();
         const size_t row = static_cast<size_t>(bg) * p.N + key;
+        // this warp's quarter of the columns: [wp * D/4, (wp + 1) * D/4)
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
           const uint32_t col = which == 0 ? Cfg::kColDK : Cfg::kColDV;
           __nv_bfloat16* dst = (which == 0 ? p.dk : p.dv) + row * D;
 #pragma unroll
-          for (int ch = 0; ch < D / 16; ++ch) {
+          for (int ch = 0; ch < D / 64; ++ch) {
+            const int cbase = wp * (D / 4) + 16 * ch;
             uint32_t v[16];
-            tc::ld_32x32b_x16(tmem + lane_base + col + 16 * ch, v);
+            tc::ld_32x32b_x16(tmem + lane_base + col + cbase, v);
             tc::wait_ld();
             if (key_ok) {
               uint4 lo, hi;
@@ -640,8 +639,8 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
               hi.y = pack_bf16(__uint_as_float(v[10]), __uint_as_float(v[11]));
               hi.z = pack_bf16(__uint_as_float(v[12]), __uint_as_float(v[13]));
               hi.w = pack_bf16(__uint_as_float(v[14]), __uint_as_float(v[15]));
-              *reinterpret_cast<uint4*>(dst + 16 * ch) = lo;
-              *reinterpret_cast<uint4*>(dst + 16 * ch + 8) = hi;
+              *reinterpret_cast<uint4*>(dst + cbase) = lo;
+              *reinterpret_cast<uint4*>(dst + cbase + 8) = hi;
             }
           }
         }

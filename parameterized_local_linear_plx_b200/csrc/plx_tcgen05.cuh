@@ -149,6 +149,13 @@ __device__ __forceinline__ void st_16x128b_x8(uint32_t taddr, const uint32_t (&r
       : "memory");
 }
 
+// 16 lanes x 128 bits, 4 repetitions (16 columns): 8 registers, layout as x8.
+__device__ __forceinline__ void st_16x128b_x4(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               PLX_W8(0)
+               : "memory");
+}
+
 // 32 lanes x 32 bits, 16 repetitions: thread t holds lane (base + t), columns
 // c .. c+15 of the address in registers 0..15.
 __device__ __forceinline__ void ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
