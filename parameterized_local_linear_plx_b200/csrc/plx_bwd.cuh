@@ -21,7 +21,7 @@
 //   * plx_bwd_pre_kernel: one warp per query row: g_bar and Dd.
 //   * plx_bwd_q_kernel (dQ, dR): one CTA per 64-query tile, with the stacked
 //     [Q;R] operand of the forward (rows 32w..32w+15: queries 16w..16w+15; rows
-//     32w+16..32w+31: their probes).  Per 128-key tile: S = [Q;R] K^T and
+//     32w+16..32w+31: their probes).  Per 64-key tile: S = [Q;R] K^T and
 //     G = [dO;0] V^T (dO in the query slots of a second stacked operand and
 //     zeros in the probe slots, so g lands in the query lanes beside a), then
 //     the element-wise warps write [scale dA ; dS] in bf16 over S and one MMA
@@ -113,19 +113,27 @@ __global__ void __launch_bounds__(256) plx_bwd_pre_kernel(const __nv_bfloat16* _
 }
 
 // ---------------------------------------------------------------- dQ, dR
+// Keys come in tiles of 64 with the score and G accumulators double-buffered
+// in tensor memory, so the MMAs of tile j+1 (and the [dQ ; dR] product of
+// tile j-1) run while the element-wise warps work on tile j.
+constexpr int kBwdQBN = 64;      // keys per tile of the query-side kernel
+constexpr int kBwdQStages = 3;   // K/V ring
+
 template <int D>
 struct BwdQCfg {
   static constexpr int kCB = D / 64;              // 128-byte column blocks per row
   static constexpr int kBlock = 128 * 128;        // one [128 rows x 128 B] block
-  static constexpr int kTileBytes = kCB * kBlock;  // a 128-row tile
+  static constexpr int kKVBlock = kBwdQBN * 128;   // one [64 rows x 128 B] block
+  static constexpr int kTileBytes = kCB * kBlock;  // a 128-row stacked tile
+  static constexpr int kKVBytes = kCB * kKVBlock;  // a 64-key K or V tile
   static constexpr int kOffQR = 0;
   static constexpr int kOffDO = kTileBytes;        // [dO ; 0] stacked like [Q ; R]
   static constexpr int kOffK = 2 * kTileBytes;
-  static constexpr int kOffV = kOffK + kBwdStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kBwdStages * kTileBytes;
+  static constexpr int kOffV = kOffK + kBwdQStages * kKVBytes;
+  static constexpr int kOffBar = kOffV + kBwdQStages * kKVBytes;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
-  // tensor memory: S [0,128), G [128,256), [dQ ; dR] [256, 256 + D)
-  static constexpr uint32_t kColS = 0, kColG = 128, kColAcc = 256, kTmemCols = 512;
+  // tensor memory: buffer b in {0,1}: S at 128b, G at 128b + 64; [dQ ; dR] at 256
+  static constexpr uint32_t kColAcc = 256, kTmemCols = 512;
 };
 
 template <int D, bool HAS_R>
@@ -134,16 +142,19 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
                  const __grid_constant__ CUtensorMap omap, const __grid_constant__ CUtensorMap kmap,
                  const __grid_constant__ CUtensorMap vmap, const BwdParams p) {
   using Cfg = BwdQCfg<D>;
-  constexpr int NS = kBwdStages;
+  constexpr int NS = kBwdQStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
   uint64_t* q_full = bars;              // [1] [Q;R] and [dO;0] landed
   uint64_t* kv_full = bars + 1;         // [NS]
   uint64_t* kv_empty = kv_full + NS;    // [NS]
-  uint64_t* s_full = kv_empty + NS;     // [1] S and G of the current key tile are in TMEM
-  uint64_t* p_ready = s_full + 1;       // [1] [dA ; dS] written (every element-wise thread)
-  uint64_t* o_done = p_ready + 1;       // [1] every MMA complete
+  uint64_t* s_full = kv_empty + NS;     // [2] S and G of a key tile are in TMEM buffer b
+  // [2] [dA ; dS] of a key tile written to buffer b (every element-wise thread).  One
+  // barrier per buffer: a phase can then complete only after the MMA thread has
+  // waited for the previous one (the tile two ahead needs a buffer it frees).
+  uint64_t* p_ready = s_full + 2;
+  uint64_t* o_done = p_ready + 2;       // [1] every MMA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -155,7 +166,8 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
   const int q0 = qt * kBwdBM;
   const int plane_kv = b * p.Hkv + h / p.G;
   const int qmax = min(p.N - 1, q0 + kBwdBM - 1);
-  const int nkv = p.causal ? qmax / kBwdBN + 1 : p.n_ktiles;
+  const int n_all = (p.N + kBwdQBN - 1) / kBwdQBN;
+  const int nkv = p.causal ? qmax / kBwdQBN + 1 : n_all;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
@@ -163,8 +175,10 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       mbar_init(smem_u32(&kv_full[s]), 1);
       mbar_init(smem_u32(&kv_empty[s]), 1);
     }
-    mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(p_ready), 32 * kBwdElemWarps);
+    mbar_init(smem_u32(&s_full[0]), 1);
+    mbar_init(smem_u32(&s_full[1]), 1);
+    mbar_init(smem_u32(&p_ready[0]), 32 * kBwdElemWarps);
+    mbar_init(smem_u32(&p_ready[1]), 32 * kBwdElemWarps);
     mbar_init(smem_u32(o_done), 1);
     fence_barrier_init();
   }
@@ -213,13 +227,13 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         const int s = j % NS;
         if (j >= NS && !mbar_wait(smem_u32(&kv_empty[s]), ((j / NS) - 1) & 1, kErrBwdLoad)) { ok = false; break; }
         const uint32_t fb = smem_u32(&kv_full[s]);
-        mbar_arrive_expect_tx(fb, 2 * Cfg::kTileBytes);
+        mbar_arrive_expect_tx(fb, 2 * Cfg::kKVBytes);
 #pragma unroll
         for (int cb = 0; cb < Cfg::kCB; ++cb) {
-          tma_load_3d(&kmap, smem_u32(smem + Cfg::kOffK + s * Cfg::kTileBytes + cb * Cfg::kBlock), fb, cb * 64,
-                      j * kBwdBN, plane_kv);
-          tma_load_3d(&vmap, smem_u32(smem + Cfg::kOffV + s * Cfg::kTileBytes + cb * Cfg::kBlock), fb, cb * 64,
-                      j * kBwdBN, plane_kv);
+          tma_load_3d(&kmap, smem_u32(smem + Cfg::kOffK + s * Cfg::kKVBytes + cb * Cfg::kKVBlock), fb, cb * 64,
+                      j * kBwdQBN, plane_kv);
+          tma_load_3d(&vmap, smem_u32(smem + Cfg::kOffV + s * Cfg::kKVBytes + cb * Cfg::kKVBlock), fb, cb * 64,
+                      j * kBwdQBN, plane_kv);
         }
         issued = j + 1;
       }
@@ -231,54 +245,68 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
   } else if (warp == kBwdMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kBwdBN, 0, 0);  // [X;Y] x Z^T, both K-major
-      constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, 0, 1);       // [dA;dS] x K, K MN-major
-      constexpr uint64_t kStageStep = Cfg::kTileBytes >> 4;
+      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kBwdQBN, 0, 0);  // [X;Y] x Z^T, both K-major
+      constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, 0, 1);        // [dA;dS] x K, K MN-major
+      constexpr uint64_t kStageStep = Cfg::kKVBytes >> 4;
       const uint64_t d_qr = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffQR), 16, 1024);
       const uint64_t d_do = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffDO), 16, 1024);
       const uint64_t d_k = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffK), 16, 1024);
       const uint64_t d_v = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffV), 16, 1024);
-      const uint64_t d_kmn = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffK), Cfg::kBlock, 1024);
-      ok = mbar_wait(smem_u32(q_full), 0, kErrBwdMma);
-      for (int j = 0; j < nkv && ok; ++j) {
+      const uint64_t d_kmn = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffK), Cfg::kKVBlock, 1024);
+      // S and G of key tile j into buffer j&1
+      auto issue_sg = [&](int j) -> bool {
         const int s = j % NS;
-        if (!mbar_wait(smem_u32(&kv_full[s]), (j / NS) & 1, kErrBwdMma)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&kv_full[s]), (j / NS) & 1, kErrBwdMma)) return false;
         tc::fence_after_sync();
+        const uint32_t cs = tmem + 128 * (j & 1);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
-          tc::mma_ss(tmem + Cfg::kColS, d_qr + koff, d_k + s * kStageStep + koff, idesc_s, ks > 0 ? 1u : 0u);
+          const uint64_t koff_a = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
+          const uint64_t koff_b = static_cast<uint64_t>(((ks >> 2) * Cfg::kKVBlock + (ks & 3) * 32) >> 4);
+          tc::mma_ss(cs, d_qr + koff_a, d_k + s * kStageStep + koff_b, idesc_s, ks > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
-          tc::mma_ss(tmem + Cfg::kColG, d_do + koff, d_v + s * kStageStep + koff, idesc_s, ks > 0 ? 1u : 0u);
+          const uint64_t koff_a = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
+          const uint64_t koff_b = static_cast<uint64_t>(((ks >> 2) * Cfg::kKVBlock + (ks & 3) * 32) >> 4);
+          tc::mma_ss(cs + kBwdQBN, d_do + koff_a, d_v + s * kStageStep + koff_b, idesc_s, ks > 0 ? 1u : 0u);
         }
-        tc::commit(smem_u32(s_full));
-        if (!mbar_wait(smem_u32(p_ready), j & 1, kErrBwdMma)) { ok = false; break; }
+        tc::commit(smem_u32(&s_full[j & 1]));
+        return true;
+      };
+      // [dQ ; dR] += [scale dA ; dS] K of key tile j: A = the bf16 pairs that
+      // warp part c wrote at columns 16c..16c+7 of buffer j&1 (keys 16c..16c+15)
+      auto issue_dqr = [&](int j) -> bool {
+        if (!mbar_wait(smem_u32(&p_ready[j & 1]), (j >> 1) & 1, kErrBwdMma)) return false;
         tc::fence_after_sync();
-        // [dQ ; dR] += [scale dA ; dS] K.  A: the bf16 pairs of keys 32c..32c+31
-        // sit in columns 32c..32c+15, so keys 16kk.. start at 32(kk/2) + 8(kk%2).
+        const int s = j % NS;
+        const uint32_t cs = tmem + 128 * (j & 1);
 #pragma unroll
-        for (int kk = 0; kk < kBwdBN / 16; ++kk)
-          tc::mma_ts(tmem + Cfg::kColAcc, tmem + Cfg::kColS + 32 * (kk >> 1) + 8 * (kk & 1),
+        for (int kk = 0; kk < kBwdQBN / 16; ++kk)
+          tc::mma_ts(tmem + Cfg::kColAcc, cs + 16 * kk,
                      d_kmn + s * kStageStep + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
                      (j > 0 || kk > 0) ? 1u : 0u);
         tc::commit(smem_u32(&kv_empty[s]));
+        return true;
+      };
+      ok = mbar_wait(smem_u32(q_full), 0, kErrBwdMma) && (nkv == 0 || issue_sg(0));
+      for (int j = 0; j < nkv && ok; ++j) {
+        // S and G of tile j+1 go to the buffer of tile j-1: its element-wise
+        // pass is over (p_ready waited) and its [dQ ; dR] MMAs precede these
+        if (j + 1 < nkv && !issue_sg(j + 1)) { ok = false; break; }
+        if (!issue_dqr(j)) { ok = false; break; }
       }
       tc::commit(smem_u32(o_done));  // also on abort: every issued MMA completes before dealloc
       mbar_wait(smem_u32(o_done), 0, kErrBwdMma);
     }
   } else {
     // ================================================================ element-wise + epilogue
-    // warp (wq, part): rows of TMEM quadrant wq, keys 32part..32part+31 of each tile
+    // warp (wq, part): rows of TMEM quadrant wq, keys 16part..16part+15 of each tile
     const int wq = warp & 3, part = warp >> 2;
     const int c4 = lane & 3;
     const int r_lo = lane >> 2;
     const uint32_t lane_a = static_cast<uint32_t>(32 * wq) << 16;
     const uint32_t lane_s = static_cast<uint32_t>(32 * wq + 16) << 16;
-    const uint32_t ta = tmem + lane_a + Cfg::kColS + 32 * part, ts = tmem + lane_s + Cfg::kColS + 32 * part;
-    const uint32_t tg = tmem + lane_a + Cfg::kColG + 32 * part;
     const int q_lo = q0 + 16 * wq + r_lo, q_hi = q_lo + 8;
     const size_t rb = static_cast<size_t>(bh) * p.N;
     // per-row statistics (rows past N: lse = +inf gives w = 0)
@@ -297,24 +325,26 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       if (HAS_R) sb_hi = p.sbar[rb + q_hi];
     }
     for (int j = 0; j < nkv; ++j) {
-      const bool landed = mbar_wait(smem_u32(s_full), j & 1, kErrBwdElem);
+      const bool landed = mbar_wait(smem_u32(&s_full[j & 1]), (j >> 1) & 1, kErrBwdElem);
       if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
       tc::fence_after_sync();
-      uint32_t ra[16], rs[16], rg[16];
-      tc::ld_16x256b_x4(ta, ra);
-      tc::ld_16x256b_x4(ts, rs);
-      tc::ld_16x256b_x4(tg, rg);
+      const uint32_t cs = 128 * (j & 1) + 16 * part;
+      const uint32_t ta = tmem + lane_a + cs, ts = tmem + lane_s + cs, tg = tmem + lane_a + cs + kBwdQBN;
+      uint32_t ra[8], rs[8], rg[8];
+      tc::ld_16x256b_x2(ta, ra);
+      tc::ld_16x256b_x2(ts, rs);
+      tc::ld_16x256b_x2(tg, rg);
       tc::wait_ld();
-      // register i: rep gg = i/4, e = i%4; key = 128j + 32part + 8gg + 2c4 + (e&1);
+      // register i: rep gg = i/4, e = i%4; key = 64j + 16part + 8gg + 2c4 + (e&1);
       // row lo for e < 2, row hi for e >= 2
-      uint32_t pa[8], pd[8];
+      uint32_t pa[4], pd[4];
 #pragma unroll
-      for (int gg = 0; gg < 4; ++gg) {
+      for (int gg = 0; gg < 2; ++gg) {
         float da[4], ds[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = 4 * gg + e;
-          const int key = j * kBwdBN + 32 * part + 8 * gg + 2 * c4 + (e & 1);
+          const int key = j * kBwdQBN + 16 * part + 8 * gg + 2 * c4 + (e & 1);
           const bool hi = (e & 2) != 0;
           const int q = hi ? q_hi : q_lo;
           const bool valid = key < p.N && (!p.causal || key <= q);
@@ -329,12 +359,12 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         pd[2 * gg] = pack_bf16(ds[0], ds[1]);
         pd[2 * gg + 1] = pack_bf16(ds[2], ds[3]);
       }
-      // bf16 pairs over the first 16 of this warp's own 32 fp32 columns
-      tc::st_16x128b_x4(ta, pa);
-      tc::st_16x128b_x4(ts, pd);
+      // bf16 pairs over the first 8 of this warp's own 16 fp32 columns
+      tc::st_16x128b_x2(ta, pa);
+      tc::st_16x128b_x2(ts, pd);
       tc::wait_st();
       tc::fence_before_sync();
-      mbar_arrive(smem_u32(p_ready));
+      mbar_arrive(smem_u32(&p_ready[j & 1]));
     }
     if (ok) {
       const bool done = mbar_wait(smem_u32(o_done), 0, kErrBwdElem);

@@ -149,6 +149,13 @@ __device__ __forceinline__ void st_16x128b_x8(uint32_t taddr, const uint32_t (&r
       : "memory");
 }
 
+// 16 lanes x 128 bits, 2 repetitions (8 columns): 4 registers, layout as x8.
+__device__ __forceinline__ void st_16x128b_x2(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.16x128b.x2.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+
 // 16 lanes x 128 bits, 4 repetitions (16 columns): 8 registers, layout as x8.
 __device__ __forceinline__ void st_16x128b_x4(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile("tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
