@@ -150,7 +150,7 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
   uint64_t* kv_full = bars + 1;         // [NS]
   uint64_t* kv_empty = kv_full + NS;    // [NS]
   uint64_t* s_full = kv_empty + NS;     // [2] S and G of a key tile are in TMEM buffer b
-  // [2] [dA ; dS] of a key tile written to buffer b (every element-wise thread).  One
+  // [2] [dA ; dS] of a key tile written to buffer b (one arrival per element-wise warp).  One
   // barrier per buffer: a phase can then complete only after the MMA thread has
   // waited for the previous one (the tile two ahead needs a buffer it frees).
   uint64_t* p_ready = s_full + 2;
@@ -177,8 +177,8 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     }
     mbar_init(smem_u32(&s_full[0]), 1);
     mbar_init(smem_u32(&s_full[1]), 1);
-    mbar_init(smem_u32(&p_ready[0]), 32 * kBwdElemWarps);
-    mbar_init(smem_u32(&p_ready[1]), 32 * kBwdElemWarps);
+    mbar_init(smem_u32(&p_ready[0]), kBwdElemWarps);  // one arrival per element-wise warp
+    mbar_init(smem_u32(&p_ready[1]), kBwdElemWarps);
     mbar_init(smem_u32(o_done), 1);
     fence_barrier_init();
   }
@@ -364,7 +364,8 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       tc::st_16x128b_x2(ts, pd);
       tc::wait_st();
       tc::fence_before_sync();
-      mbar_arrive(smem_u32(&p_ready[j & 1]));
+      __syncwarp();  // every lane's stores are complete: one lane arrives for the warp
+      if (lane == 0) mbar_arrive(smem_u32(&p_ready[j & 1]));
     }
     if (ok) {
       const bool done = mbar_wait(smem_u32(o_done), 0, kErrBwdElem);
@@ -444,7 +445,7 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* q_full = bars + 1;          // [NS] [Q;R] and dO of a query tile landed
   uint64_t* q_empty = q_full + NS;      // [NS]
   uint64_t* s_full = q_empty + NS;      // [1] [A^T|S^T] and G^T in TMEM
-  uint64_t* p_ready = s_full + 1;       // [1] W_hat^T, dA^T, dS^T written (every element-wise thread)
+  uint64_t* p_ready = s_full + 1;       // [1] W_hat^T, dA^T, dS^T written (one arrival per element-wise warp)
   uint64_t* o_done = p_ready + 1;       // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
 
@@ -466,7 +467,7 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       mbar_init(smem_u32(&q_empty[s]), 1);
     }
     mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(p_ready), 32 * kBwdElemWarps);
+    mbar_init(smem_u32(p_ready), kBwdElemWarps);  // one arrival per element-wise warp
     mbar_init(smem_u32(o_done), 1);
     fence_barrier_init();
   }
@@ -641,7 +642,8 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       tc::st_32x32b_x8(tsa + 8, pd);
       tc::wait_st();
       tc::fence_before_sync();
-      mbar_arrive(smem_u32(p_ready));
+      __syncwarp();  // every lane's stores are complete: one lane arrives for the warp
+      if (lane == 0) mbar_arrive(smem_u32(p_ready));
     }
     if (ok) {
       const bool done = mbar_wait(smem_u32(o_done), 0, kErrBwdElem);

@@ -111,7 +111,7 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   uint64_t* s_full = v_empty + NS;      // [2]
   uint64_t* p_ready = s_full + 2;       // [2 tiles][2 halves]
   uint64_t* o_done = p_ready + 4;       // [2]
-  uint64_t* o_free = o_done + 2;        // [2] epilogue has read O (128 arrivals)
+  uint64_t* o_free = o_done + 2;        // [2] epilogue has read O (one arrival per softmax warp)
   uint64_t* fin = o_free + 2;           // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
 
@@ -141,12 +141,13 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   auto row0_of = [&](const Unit& w, int t) { return p.pair_heads ? w.qb * kFwdBM : (2 * w.qb + t) * kFwdBM; };
 
   if (threadIdx.x == 0) {
-    // arrivals per phase: p_ready and o_free get all 128 threads of a
-    // softmax warpgroup; every other barrier one arrival (+ TMA bytes / a commit)
+    // arrivals per phase: p_ready and o_free get one arrival from each of the
+    // 4 warps of a softmax warpgroup; every other barrier one arrival (+ TMA
+    // bytes / a commit)
     for (int i = 0; i < 3 + 4 * NS + 11; ++i) {
       uint64_t* bp = &bars[i];
       const bool wg = (bp >= &p_ready[0] && bp <= &p_ready[3]) || bp == &o_free[0] || bp == &o_free[1];
-      mbar_init(smem_u32(bp), wg ? 128u : 1u);
+      mbar_init(smem_u32(bp), wg ? 4u : 1u);
     }
     fence_barrier_init();
   }
@@ -466,7 +467,8 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           if (HAS_R) tc::st_16x128b_x8(ts + 32 * hf, pq);
           tc::wait_st();
           tc::fence_before_sync();
-          mbar_arrive(smem_u32(&p_ready[2 * t + hf]));
+          __syncwarp();  // every lane's stores are complete: one lane arrives for the warp
+          if (lane == 0) mbar_arrive(smem_u32(&p_ready[2 * t + hf]));
         }
         l_lo += f2_lo(ls_lo) + f2_hi(ls_lo);
         l_hi += f2_lo(ls_hi) + f2_hi(ls_hi);
@@ -526,7 +528,8 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       if (!SAVE_AUX) {
         // O has been read: the next unit's first value MMA may overwrite it
         tc::fence_before_sync();
-        mbar_arrive(smem_u32(&o_free[t]));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&o_free[t]));
       }
       if (p.lse && c4 == 0) {
         if (q_lo < p.N) p.lse[plane * p.N + q_lo] = l_lo > 0.f ? (m_lo + __log2f(l_lo)) * kLn2 : -INFINITY;
@@ -569,7 +572,8 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           }
         }
         tc::fence_before_sync();
-        mbar_arrive(smem_u32(&o_free[t]));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&o_free[t]));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && row0 < p.N) {
