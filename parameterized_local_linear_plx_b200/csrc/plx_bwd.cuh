@@ -225,7 +225,7 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       int issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int s = j % NS;
-        if (j >= NS && !mbar_wait(smem_u32(&kv_empty[s]), ((j / NS) - 1) & 1, kErrBwdLoad)) { ok = false; break; }
+        if (j >= NS && !mbar_wait_sleep(smem_u32(&kv_empty[s]), ((j / NS) - 1) & 1, kErrBwdLoad)) { ok = false; break; }
         const uint32_t fb = smem_u32(&kv_full[s]);
         mbar_arrive_expect_tx(fb, 2 * Cfg::kKVBytes);
 #pragma unroll
@@ -324,8 +324,15 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       dd_hi = p.dd[rb + q_hi];
       if (HAS_R) sb_hi = p.sbar[rb + q_hi];
     }
+    // the per-row constants as packed pairs (both elements of a pair share the row):
+    // -lse log2(e), 1 + s_bar, g_bar, -Dd
+    const uint64_t nl_lo = f2(-l2_lo, -l2_lo), nl_hi = f2(-l2_hi, -l2_hi);
+    const uint64_t f_lo = f2(1.f + sb_lo, 1.f + sb_lo), f_hi = f2(1.f + sb_hi, 1.f + sb_hi);
+    const uint64_t gb2_lo = f2(gb_lo, gb_lo), gb2_hi = f2(gb_hi, gb_hi);
+    const uint64_t nd_lo = f2(-dd_lo, -dd_lo), nd_hi = f2(-dd_hi, -dd_hi);
+    const uint64_t c_sl2 = f2(p.scale_log2, p.scale_log2), c_m1 = f2(-1.f, -1.f), c_sc = f2(p.scale, p.scale);
     for (int j = 0; j < nkv; ++j) {
-      const bool landed = mbar_wait(smem_u32(&s_full[j & 1]), (j >> 1) & 1, kErrBwdElem);
+      const bool landed = mbar_wait_sleep(smem_u32(&s_full[j & 1]), (j >> 1) & 1, kErrBwdElem);
       if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
       tc::fence_after_sync();
       const uint32_t cs = 128 * (j & 1) + 16 * part;
@@ -335,29 +342,37 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       tc::ld_16x256b_x2(ts, rs);
       tc::ld_16x256b_x2(tg, rg);
       tc::wait_ld();
+      // masks only where some (query, key) of this warp is out of the set:
+      // keys past N, or (causal) a key of the warp after its first row
+      const int kw = j * kBwdQBN + 16 * part;  // this warp's first key
+      const bool need_mask = (kw + 15 >= p.N) || (p.causal && kw + 15 > q0 + 16 * wq);
       // register i: rep gg = i/4, e = i%4; key = 64j + 16part + 8gg + 2c4 + (e&1);
-      // row lo for e < 2, row hi for e >= 2
+      // row lo for e < 2, row hi for e >= 2.  Registers (4gg, 4gg+1) and
+      // (4gg+2, 4gg+3) are key pairs of one row: packed f32x2 arithmetic.
       uint32_t pa[4], pd[4];
 #pragma unroll
-      for (int gg = 0; gg < 2; ++gg) {
-        float da[4], ds[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 4 * gg + e;
-          const int key = j * kBwdQBN + 16 * part + 8 * gg + 2 * c4 + (e & 1);
-          const bool hi = (e & 2) != 0;
+      for (int h2 = 0; h2 < 4; ++h2) {
+        const int i = 2 * h2;
+        const bool hi = (h2 & 1) != 0;
+        const uint64_t A = f2(__uint_as_float(ra[i]), __uint_as_float(ra[i + 1]));
+        const uint64_t S = f2(__uint_as_float(rs[i]), __uint_as_float(rs[i + 1]));
+        const uint64_t G = f2(__uint_as_float(rg[i]), __uint_as_float(rg[i + 1]));
+        const uint64_t X = f2_fma(A, c_sl2, hi ? nl_hi : nl_lo);
+        float w0 = ex2(f2_lo(X)), w1 = ex2(f2_hi(X));
+        if (need_mask) {
+          const int key = kw + 8 * (h2 >> 1) + 2 * c4;
           const int q = hi ? q_hi : q_lo;
-          const bool valid = key < p.N && (!p.causal || key <= q);
-          const float a = __uint_as_float(ra[i]), s = __uint_as_float(rs[i]), g = __uint_as_float(rg[i]);
-          const float w = valid ? ex2(fmaf(a, p.scale_log2, -(hi ? l2_hi : l2_lo))) : 0.f;
-          const float sb = hi ? sb_hi : sb_lo, gb = hi ? gb_hi : gb_lo, d2 = hi ? dd_hi : dd_lo;
-          ds[e] = w * (gb - g);
-          da[e] = p.scale * w * (fmaf(g, 1.f - s + sb, s * gb) - d2);
+          if (key >= p.N || (p.causal && key > q)) w0 = 0.f;
+          if (key + 1 >= p.N || (p.causal && key + 1 > q)) w1 = 0.f;
         }
-        pa[2 * gg] = pack_bf16(da[0], da[1]);
-        pa[2 * gg + 1] = pack_bf16(da[2], da[3]);
-        pd[2 * gg] = pack_bf16(ds[0], ds[1]);
-        pd[2 * gg + 1] = pack_bf16(ds[2], ds[3]);
+        const uint64_t W = f2(w0, w1);
+        const uint64_t Gb = hi ? gb2_hi : gb2_lo;
+        const uint64_t F = f2_fma(S, c_m1, hi ? f_hi : f_lo);                  // 1 + s_bar - s
+        const uint64_t DS = f2_mul(W, f2_fma(G, c_m1, Gb));                     // w (g_bar - g)
+        const uint64_t U = f2_fma(G, F, f2_fma(S, Gb, hi ? nd_hi : nd_lo));    // g f + s g_bar - Dd
+        const uint64_t DA = f2_mul(f2_mul(W, c_sc), U);
+        pa[h2] = pack_bf16(f2_lo(DA), f2_hi(DA));
+        pd[h2] = pack_bf16(f2_lo(DS), f2_hi(DS));
       }
       // bf16 pairs over the first 8 of this warp's own 16 fp32 columns
       tc::st_16x128b_x2(ta, pa);
@@ -368,7 +383,7 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       if (lane == 0) mbar_arrive(smem_u32(&p_ready[j & 1]));
     }
     if (ok) {
-      const bool done = mbar_wait(smem_u32(o_done), 0, kErrBwdElem);
+      const bool done = mbar_wait_sleep(smem_u32(o_done), 0, kErrBwdElem);
       if (__all_sync(0xffffffffu, done)) {
         tc::fence_after_sync();
         // this warp's quarter of the columns: [part * D/4, (part + 1) * D/4)
@@ -506,7 +521,7 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       int issued = 0;
       for (int it = 0; it < n_items; ++it) {
         const int s = it % NS;
-        if (it >= NS && !mbar_wait(smem_u32(&q_empty[s]), ((it / NS) - 1) & 1, kErrBwdLoad)) { ok = false; break; }
+        if (it >= NS && !mbar_wait_sleep(smem_u32(&q_empty[s]), ((it / NS) - 1) & 1, kErrBwdLoad)) { ok = false; break; }
         const int hq = g * p.G + it / n_qt;
         const int q0 = (qt0 + it % n_qt) * kBwdBM;
         const int plane = b * p.Hq + hq;
@@ -594,20 +609,24 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       const size_t rb = (static_cast<size_t>(b) * p.Hq + hq) * p.N;
       __syncwarp();
       if (lane < 16) {
+        // per query: -lse log2(e), 1 + s_bar, g_bar, -Dd (rows past N: w = 0)
         const int q = q0 + lane;
-        float4 st4 = make_float4(INFINITY, 0.f, 0.f, 0.f);  // rows past N: w = 0
+        float4 st4 = make_float4(-INFINITY, 1.f, 0.f, 0.f);
         if (q < p.N) {
-          st4.x = p.lse[rb + q] * kLog2e;
-          st4.y = HAS_R ? p.sbar[rb + q] : 0.f;
+          st4.x = -p.lse[rb + q] * kLog2e;
+          st4.y = 1.f + (HAS_R ? p.sbar[rb + q] : 0.f);
           st4.z = p.gbar[rb + q];
-          st4.w = p.dd[rb + q];
+          st4.w = -p.dd[rb + q];
         }
         stat[lane] = st4;
       }
       __syncwarp();
-      const bool landed = mbar_wait(smem_u32(s_full), it & 1, kErrBwdElem);
+      const bool landed = mbar_wait_sleep(smem_u32(s_full), it & 1, kErrBwdElem);
       if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
       tc::fence_after_sync();
+      // masks only where some (key, query) of this warp is out of the set:
+      // keys past N, or (causal) a key of the warp after its first query
+      const bool need_mask = (k0 + 32 * wq + 31 >= p.N) || (p.causal && k0 + 32 * wq + 31 > q0);
       // stacked columns 32wp..32wp+15 (q.k) and 32wp+16..32wp+31 (rho.k), G^T columns 16wp..16wp+15
       const uint32_t tsa = tmem + lane_base + Cfg::kColS + 32 * wp;
       const uint32_t tgw = tmem + lane_base + Cfg::kColG + 16 * wp;
@@ -616,25 +635,34 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       tc::ld_32x32b_x16(tsa + 16, rs);
       tc::ld_32x32b_x16(tgw, rg);
       tc::wait_ld();
+      // two queries at a time in packed f32x2 arithmetic:
+      //   w = 2^(a scale log2e - lse log2e), f = 1 + s_bar - s,
+      //   w_hat = w f,  dS = w (g_bar - g),  scale dA = (scale w)(g f + s g_bar - Dd)
+      const uint64_t c_sl2 = f2(p.scale_log2, p.scale_log2), c_m1 = f2(-1.f, -1.f), c_sc = f2(p.scale, p.scale);
       uint32_t pw[8], pa[8], pd[8];
 #pragma unroll
       for (int x = 0; x < 16; x += 2) {
-        float wh[2], da[2], ds[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int q = q0 + x + e;
-          const float4 st4 = stat[x + e];
-          const bool valid = key_ok && (!p.causal || key <= q);
-          const float a = __uint_as_float(ra[x + e]), s = __uint_as_float(rs[x + e]), gv = __uint_as_float(rg[x + e]);
-          const float w = valid ? ex2(fmaf(a, p.scale_log2, -st4.x)) : 0.f;
-          const float fct = 1.f - s + st4.y;
-          wh[e] = w * fct;
-          ds[e] = w * (st4.z - gv);
-          da[e] = p.scale * w * (fmaf(gv, fct, s * st4.z) - st4.w);
+        const float4 s0 = stat[x], s1 = stat[x + 1];
+        const uint64_t A = f2(__uint_as_float(ra[x]), __uint_as_float(ra[x + 1]));
+        const uint64_t S = f2(__uint_as_float(rs[x]), __uint_as_float(rs[x + 1]));
+        const uint64_t Gv = f2(__uint_as_float(rg[x]), __uint_as_float(rg[x + 1]));
+        const uint64_t X = f2_fma(A, c_sl2, f2(s0.x, s1.x));
+        float w0 = ex2(f2_lo(X)), w1 = ex2(f2_hi(X));
+        if (need_mask) {
+          const int q = q0 + x;
+          if (!key_ok || (p.causal && key > q)) w0 = 0.f;
+          if (!key_ok || (p.causal && key > q + 1)) w1 = 0.f;
         }
-        pw[x >> 1] = pack_bf16(wh[0], wh[1]);
-        pa[x >> 1] = pack_bf16(da[0], da[1]);
-        pd[x >> 1] = pack_bf16(ds[0], ds[1]);
+        const uint64_t W = f2(w0, w1);
+        const uint64_t Gb = f2(s0.z, s1.z);
+        const uint64_t F = f2_fma(S, c_m1, f2(s0.y, s1.y));                    // 1 + s_bar - s
+        const uint64_t WH = f2_mul(W, F);
+        const uint64_t DS = f2_mul(W, f2_fma(Gv, c_m1, Gb));                    // w (g_bar - g)
+        const uint64_t U = f2_fma(Gv, F, f2_fma(S, Gb, f2(s0.w, s1.w)));       // g f + s g_bar - Dd
+        const uint64_t DA = f2_mul(f2_mul(W, c_sc), U);
+        pw[x >> 1] = pack_bf16(f2_lo(WH), f2_hi(WH));
+        pa[x >> 1] = pack_bf16(f2_lo(DA), f2_hi(DA));
+        pd[x >> 1] = pack_bf16(f2_lo(DS), f2_hi(DS));
       }
       // bf16 pairs over this warp's own fp32 columns (already read)
       tc::st_32x32b_x8(tgw, pw);
@@ -646,7 +674,7 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       if (lane == 0) mbar_arrive(smem_u32(p_ready));
     }
     if (ok) {
-      const bool done = mbar_wait(smem_u32(o_done), 0, kErrBwdElem);
+      const bool done = mbar_wait_sleep(smem_u32(o_done), 0, kErrBwdElem);
       if (__all_sync(0xffffffffu, done)) {
         tc::fence_after_sync();
         const size_t row = static_cast<size_t>(bg) * p.N + key;

@@ -94,6 +94,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete.  Returns false (and
 // records `code` unless another error is already recorded) if it has not
 // completed within `limit` cycles or another CTA has given up.
+// try_wait with a suspend-time hint: the thread may sleep until the phase
+// completes (or about `ns` nanoseconds pass) instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0u;
+}
+// Bounded wait for warps that have nothing else to do: they sleep in the
+// barrier instead of spinning, so they leave the issue slots of their
+// sub-partition to the warps that work (the MMA-issuing thread above all).
+// Each sleep is at most 0.1 ms, so the time limit and the device error word
+// are checked as often as by mbar_wait.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, unsigned code,
+                                                long long limit = kWaitLimitCycles) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+    if (clock64() - t0 > limit) {
+      set_error(code);
+      return false;
+    }
+    if ((it & 15u) == 0u && error_is_set()) return false;
+  }
+}
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned code,
                                           long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
