@@ -411,6 +411,9 @@ def run_gpu(args, world, rank, local):
     # ---- end to end through the public API: pinned host buffers, copies timed
     e2e = run_e2e(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes)
 
+    # ---- the same decode step on a paged cache (block tables), timed on its own
+    paged = run_paged(plx, args, dev, stream, world, local, d_bytes, hbm, peak_src)
+
     # ---- training backward of the prefill shape (timed on its own; not part of the step)
     bwd = run_backward(plx, args, dev, stream, world, local, pq, pk, pv, pr, peaks, peak_src)
 
@@ -439,6 +442,7 @@ def run_gpu(args, world, rank, local):
             "roofline": roof_pre,
             "roofline_decode": roof_dec,
             "e2e": e2e,
+            "decode_paged": paged,
             "backward": bwd,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
@@ -446,6 +450,50 @@ def run_gpu(args, world, rank, local):
         }
         print(json.dumps(line), flush=True)
     return 0
+
+
+def run_paged(plx, args, dev, stream, world, local, d_bytes, hbm, peak_src):
+    """plx_decode_paged on the decode workload (B=64, context 4096, equal
+    seqlens) with pages of 16 and of 64 keys, slots assigned to pool pages by
+    a random permutation; CUDA events per call, max over ranks."""
+    import torch
+    res = {}
+    for ps in (64, 16):
+        q, kp, vp, r, table, sl = inputs_mod().paged_decode_inputs(
+            DEC["B"], DEC["Hq"], DEC["Hkv"], DEC["S"] // ps, ps, DEC["d"], seed=200 + local, seqlens="equal",
+            device=dev)
+        out = torch.empty_like(q)
+        lse = torch.empty(DEC["B"], DEC["Hq"], dtype=torch.float32, device=dev)
+        need = plx.plx_decode_workspace_size(DEC["B"], DEC["Hq"], DEC["Hkv"], DEC["S"], DEC["d"], 0)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        for _ in range(max(3, args.warmup)):
+            plx.plx_decode_paged(q, kp, vp, table, sl, r, out=out, lse=lse, workspace=ws, stream=stream)
+        steps = max(1, min(args.steps, 50))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(steps):
+            plx.plx_decode_paged(q, kp, vp, table, sl, r, out=out, lse=lse, workspace=ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        st = plx.plx_check_device_status(stream)
+        if st != plx.PLX_OK:
+            raise RuntimeError(f"device status after the paged decode: {plx.plx_status_string(st)}")
+        us = max_over_ranks(e0.elapsed_time(e1) / steps * 1e3, world, dev)
+        gbs = d_bytes / (us * 1e-6) / 1e9
+        res[f"page_{ps}"] = {"gbs": world * gbs, "us_per_step": us, "frac_of_hbm": gbs / hbm}
+        del q, kp, vp, r, table, sl, out, lse, ws
+    res["workload"] = (f"decode B={DEC['B']} ctx={DEC['S']} Hq={DEC['Hq']} Hkv={DEC['Hkv']} d={DEC['d']} on page "
+                       f"pools [pages, Hkv, page_size, d], random page assignment")
+    res["peak_source"] = f"{peak_src} hbm_gbs"
+    return res
+
+
+def inputs_mod():
+    from parameterized_local_linear_plx_b200 import inputs
+    return inputs
 
 
 def run_backward(plx, args, dev, stream, world, local, pq, pk, pv, pr, peaks, peak_src):

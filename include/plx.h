@@ -196,6 +196,36 @@ int plx_decode(const void* q, const void* r, const void* kcache, const void* vca
                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * plx_decode_paged -- plx_decode against a paged KV cache (block tables).
+ *
+ *   kpool, vpool [num_pages, Hkv, page_size, d] bf16   page pools: page p holds
+ *                page_size consecutive keys (values) of every KV head
+ *   block_table  [B, max_pages] int32, DEVICE   pool page of each page slot:
+ *                keys n*page_size .. (n+1)*page_size-1 of sequence b are in
+ *                page block_table[b * max_pages + n]
+ *   seqlens      [B] int32, DEVICE   live keys per sequence (clamped to
+ *                [0, max_pages * page_size])
+ *   page_size    a power of two, 16 .. 4096
+ *   q, r, out, lse, scale, num_splits, workspace: as plx_decode, with
+ *   S_max = max_pages * page_size (plx_decode_workspace_size and
+ *   plx_decode_num_splits take that S_max).
+ *
+ * Reads only the table entries of pages that hold live keys.  An entry
+ * outside [0, num_pages) is treated as a page of zeros (its keys then score
+ * 0 and carry zero values); nothing outside the pools is read.  Keys past
+ * seqlens[b] inside a live page are read and weighted 0: they must hold
+ * finite values, as must the unused rows of a contiguous cache.
+ * Results equal plx_decode on the gathered contiguous cache with the same
+ * S_max and split count.  This is the serving form of the decode step
+ * (paged caches); the pages themselves describe only a contiguous cache.
+ */
+int plx_decode_paged(const void* q, const void* r, const void* kpool, const void* vpool,
+                     const int32_t* block_table, const int32_t* seqlens, void* out, float* lse,
+                     int B, int Hq, int Hkv, int num_pages, int page_size, int max_pages,
+                     int d, float scale, int num_splits,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * PLX_NOALLOC_SCRATCH_BYTES -- size of the library's fixed device scratch
  * array used by plx_decode_noalloc (16 MiB, held on every GPU that loads the
  * library until the process exits).

@@ -120,14 +120,14 @@ size_t workspace_bytes_for(int B, int Hq, int d, int splits) {
   return static_cast<size_t>(B) * Hq * splits * (2 * d + 4) * sizeof(float);
 }
 
-template <int D, bool HAS_R>
+template <int D, bool HAS_R, bool PAGED>
 int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const plx::DecodeParams& p, int n_hg,
                   cudaStream_t st) {
   using Cfg = plx::DecodeCfg<D>;
   static bool done[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  auto kern = plx::plx_decode_split_kernel<D, HAS_R>;
+  auto kern = plx::plx_decode_split_kernel<D, HAS_R, PAGED>;
   if (ensure_smem(kern, Cfg::kSmemBytes, &done[dev]) != PLX_OK) return PLX_ERR_CUDA;
   dim3 grid(p.splits, p.Hkv * n_hg, p.B);
   kern<<<grid, plx::kDecThreads, Cfg::kSmemBytes, st>>>(km, vm, p);
@@ -289,6 +289,68 @@ int plx_fwd_train(const void* q, const void* k, const void* v, const void* r, vo
   return fwd_common(q, k, v, r, out, lse, obar, sbar, B, Hq, Hkv, N, d, causal, scale, stream);
 }
 
+int plx_decode_paged(const void* q, const void* r, const void* kpool, const void* vpool,
+                     const int32_t* block_table, const int32_t* seqlens, void* out, float* lse, int B, int Hq,
+                     int Hkv, int num_pages, int page_size, int max_pages, int d, float scale, int num_splits,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !kpool || !vpool || !block_table || !seqlens || !out) return PLX_ERR_NULL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || num_pages < 1 || max_pages < 1 || num_splits < 0) return PLX_ERR_SHAPE;
+  if (page_size < 16 || page_size > 4096 || (page_size & (page_size - 1))) return PLX_ERR_SHAPE;
+  if (B > 65535 || static_cast<long long>(max_pages) * page_size > 0x7fffffffLL ||
+      static_cast<long long>(num_pages) * Hkv > 0x7fffffffLL)
+    return PLX_ERR_SHAPE;
+  if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
+  if (Hq % Hkv) return PLX_ERR_GQA;
+  if (!aligned16(q) || (r && !aligned16(r)) || !aligned16(kpool) || !aligned16(vpool) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return PLX_ERR_ALIGN;
+  const int S_max = max_pages * page_size;
+  const SplitPlan plan = plan_splits(B, Hq, Hkv, S_max, num_splits);
+  const size_t need = workspace_bytes_for(B, Hq, d, plan.splits);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return PLX_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return PLX_ERR_ALIGN;
+  }
+  const int G = Hq / Hkv;
+  const int n_hg = (G + 7) / 8;
+  if (static_cast<long long>(Hkv) * n_hg > 65535) return PLX_ERR_SHAPE;
+  int dev = 0;
+  int rc = check_arch(&dev);
+  if (rc != PLX_OK) return rc;
+  if ((rc = get_encoder()) != PLX_OK) return rc;
+
+  // the pools as [num_pages * Hkv planes, page_size rows, d]; one box = one page part
+  const int box_rows = page_size < plx::kDecTileKeys ? page_size : plx::kDecTileKeys;
+  CUtensorMap km, vm;
+  const long long planes = static_cast<long long>(num_pages) * Hkv;
+  if (make_map_3d(&km, kpool, d, page_size, planes, box_rows) != PLX_OK ||
+      make_map_3d(&vm, vpool, d, page_size, planes, box_rows) != PLX_OK)
+    return PLX_ERR_CUDA;
+
+  plx::DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.r = static_cast<const __nv_bfloat16*>(r);
+  p.seqlens = seqlens;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.ws = static_cast<float*>(workspace);
+  p.block_table = block_table;
+  p.num_pages = num_pages;
+  p.max_pages = max_pages;
+  p.page_size = page_size;
+  int shift = 0;
+  while ((1 << shift) < page_size) ++shift;
+  p.page_shift = shift;
+  p.box_rows = box_rows;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.S_max = S_max; p.G = G; p.n_hgroups = n_hg;
+  p.splits = plan.splits; p.chunk = plan.chunk;
+  p.scale_log2 = scale * plx::kLog2e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 128) return r ? launch_decode<128, true, true>(km, vm, p, n_hg, st) : launch_decode<128, false, true>(km, vm, p, n_hg, st);
+  return r ? launch_decode<64, true, true>(km, vm, p, n_hg, st) : launch_decode<64, false, true>(km, vm, p, n_hg, st);
+}
+
 size_t plx_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv || (d != 64 && d != 128)) return 0;
   return bwd_workspace_bytes(B, Hq, N);
@@ -393,7 +455,7 @@ int plx_decode(const void* q, const void* r, const void* kcache, const void* vca
       make_map_3d(&vm, vcache, d, S_max, planes, plx::kDecTileKeys) != PLX_OK)
     return PLX_ERR_CUDA;
 
-  plx::DecodeParams p;
+  plx::DecodeParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.r = static_cast<const __nv_bfloat16*>(r);
   p.seqlens = seqlens;
@@ -404,8 +466,8 @@ int plx_decode(const void* q, const void* r, const void* kcache, const void* vca
   p.splits = plan.splits; p.chunk = plan.chunk;
   p.scale_log2 = scale * plx::kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 128) return r ? launch_decode<128, true>(km, vm, p, n_hg, st) : launch_decode<128, false>(km, vm, p, n_hg, st);
-  return r ? launch_decode<64, true>(km, vm, p, n_hg, st) : launch_decode<64, false>(km, vm, p, n_hg, st);
+  if (d == 128) return r ? launch_decode<128, true, false>(km, vm, p, n_hg, st) : launch_decode<128, false, false>(km, vm, p, n_hg, st);
+  return r ? launch_decode<64, true, false>(km, vm, p, n_hg, st) : launch_decode<64, false, false>(km, vm, p, n_hg, st);
 }
 
 int plx_check_device_status(void* stream) {

@@ -21,6 +21,14 @@
 // Each CTA writes its partial state (m, l, c, O1, O2) to the workspace, or,
 // with a single split, the final out = O1/l - (O2/l - (c/l)(O1/l)) and lse.
 // plx_decode_combine merges the partials of all splits.
+//
+// Paged caches (PAGED = true): K and V live in page pools
+// [num_pages, Hkv, page_size, D] and a block table maps the page slots of
+// each sequence to pool pages.  The producer looks up the page of every
+// min(page_size, 64)-key part of a tile and loads it from there; a part past
+// the sequence, or with a page id outside the pool, is loaded at a row past
+// the page, which TMA fills with zeros, so no page outside the pool is read.
+// The consumers are the same as for contiguous caches.
 #pragma once
 
 #include "plx_ptx.cuh"
@@ -46,6 +54,8 @@ struct DecodeParams {
   const __nv_bfloat16* r;   // [B, Hq, D] or nullptr
   const int32_t* seqlens;   // [B]
   __nv_bfloat16* out;       // [B, Hq, D]
+  const int32_t* block_table;  // [B, max_pages] pool page of each page slot (paged caches)
+  int num_pages, max_pages, page_size, page_shift, box_rows;  // paged caches: pool, table width, page
   float* lse;               // [B, Hq] or nullptr
   float* ws;                // [B, Hq, splits, 2D+4] or nullptr when splits == 1
                             //   per row: m (log2 units), l, c, pad, O1[D], O2[D]
@@ -59,7 +69,7 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int D, bool HAS_R>
+template <int D, bool HAS_R, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, 2)
 plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
@@ -132,10 +142,31 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
         const uint32_t kdst = smem_u32(smem + s * Cfg::kStageBytes);
         const uint32_t vdst = kdst + Cfg::kTileBytes;
         const int key0 = kbeg + t * kDecTileKeys;
+        if (!PAGED) {
 #pragma unroll
-        for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-          tma_load_3d(&kmap, kdst + hf * (kDecTileKeys * 128), fb, hf * 64, key0, kvrow);
-          tma_load_3d(&vmap, vdst + hf * (kDecTileKeys * 128), fb, hf * 64, key0, kvrow);
+          for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+            tma_load_3d(&kmap, kdst + hf * (kDecTileKeys * 128), fb, hf * 64, key0, kvrow);
+            tma_load_3d(&vmap, vdst + hf * (kDecTileKeys * 128), fb, hf * 64, key0, kvrow);
+          }
+        } else {
+          // one load per page part of the tile: plane = page * Hkv + g, row within the page
+          for (int part = 0; part * p.box_rows < kDecTileKeys; ++part) {
+            const int key = key0 + part * p.box_rows;
+            int plane = 0, row = p.page_size;  // default: past the page, zero fill
+            if (key < kend) {
+              const int pg = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + (key >> p.page_shift));
+              if (pg >= 0 && pg < p.num_pages) {
+                plane = pg * p.Hkv + g;
+                row = key & (p.page_size - 1);
+              }
+            }
+            const uint32_t off = static_cast<uint32_t>(part * p.box_rows * 128);
+#pragma unroll
+            for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+              tma_load_3d(&kmap, kdst + hf * (kDecTileKeys * 128) + off, fb, hf * 64, row, plane);
+              tma_load_3d(&vmap, vdst + hf * (kDecTileKeys * 128) + off, fb, hf * 64, row, plane);
+            }
+          }
         }
         issued = t + 1;
       }

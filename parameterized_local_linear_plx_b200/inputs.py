@@ -93,3 +93,42 @@ def decode_inputs(B, Hq, Hkv, S_max, d, seed=0, r_scale=0.1, seqlens="equal",
     else:
         sl = torch.tensor(list(seqlens), dtype=torch.int32, device=device)
     return q, kc, vc, r, sl
+
+
+def paged_decode_inputs(B, Hq, Hkv, max_pages, page_size, d, seed=0, r_scale=0.1, seqlens="ragged",
+                        spare_pages=3, dtype=torch.bfloat16, device="cpu"):
+    """Decode inputs on a paged cache: (q, kpool, vpool, r, block_table, seqlens).
+
+    The pools hold B * max_pages + spare_pages pages of [Hkv, page_size, d]
+    (drawn like the contiguous caches); page slots are assigned to pool pages
+    by a seeded random permutation, so neighbouring slots sit in unrelated
+    pages.  seqlens as in decode_inputs with S_max = max_pages * page_size.
+    """
+    S_max = max_pages * page_size
+    g = _gen(seed, device)
+    num_pages = B * max_pages + spare_pages
+    q = draw((B, Hq, d), g, device, 1.0, dtype)
+    kpool = draw((num_pages, Hkv, page_size, d), g, device, 1.0, dtype)
+    vpool = draw((num_pages, Hkv, page_size, d), g, device, 1.0, dtype)
+    r = draw((B, Hq, d), g, device, r_scale, dtype)
+    perm = torch.randperm(num_pages, generator=g, device=device)[: B * max_pages]
+    table = perm.to(torch.int32).reshape(B, max_pages).contiguous()
+    if isinstance(seqlens, str):
+        if seqlens == "equal":
+            sl = torch.full((B,), S_max, dtype=torch.int32, device=device)
+        elif seqlens == "ragged":
+            sl = torch.randint(S_max // 2, S_max + 1, (B,), generator=g, device=device, dtype=torch.int32)
+        else:
+            raise ValueError(f"unknown seqlens mode {seqlens!r}")
+    else:
+        sl = torch.tensor(list(seqlens), dtype=torch.int32, device=device)
+    return q, kpool, vpool, r, table, sl
+
+
+def gather_pages(pool, table):
+    """The contiguous cache [B, Hkv, max_pages * page_size, d] a block table
+    describes (page slot n of sequence b = pool page table[b, n])."""
+    B, max_pages = table.shape
+    _, Hkv, page_size, d = pool.shape
+    pages = pool[table.long().reshape(-1)].reshape(B, max_pages, Hkv, page_size, d)
+    return pages.permute(0, 2, 1, 3, 4).reshape(B, Hkv, max_pages * page_size, d).contiguous()

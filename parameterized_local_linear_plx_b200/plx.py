@@ -45,6 +45,8 @@ _lib.plx_decode_workspace_size.restype = _SZ
 _lib.plx_decode_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I]
 _lib.plx_decode.restype = _I
 _lib.plx_decode.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P]
+_lib.plx_decode_paged.restype = _I
+_lib.plx_decode_paged.argtypes = [_P] * 8 + [_I] * 7 + [_F, _I, _P, _SZ, _P]
 _lib.plx_decode_noalloc.restype = _I
 _lib.plx_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]
 _lib.plx_check_device_status.restype = _I
@@ -238,6 +240,42 @@ def plx_decode(q, kcache, vcache, seqlens, r=None, scale=None, num_splits=0, out
                          _stream(stream))
     if st != PLX_OK:
         raise PlxError(st, "plx_decode")
+    return out, lse
+
+
+def plx_decode_paged(q, kpool, vpool, block_table, seqlens, r=None, scale=None, num_splits=0, out=None, lse=None,
+                     workspace=None, return_lse=True, stream=None):
+    """One decode step against paged caches.  q/r [B, Hq, d] bf16; kpool/vpool
+    [num_pages, Hkv, page_size, d] bf16; block_table [B, max_pages] int32 and
+    seqlens [B] int32 on the device.  Returns (out, lse) as plx_decode."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(kpool, "kpool", torch.bfloat16, 4)
+    _check(vpool, "vpool", torch.bfloat16, 4)
+    _check(block_table, "block_table", torch.int32, 2)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    if r is not None:
+        _check(r, "r", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    num_pages, Hkv, page_size = kpool.shape[0], kpool.shape[1], kpool.shape[2]
+    max_pages = block_table.shape[1]
+    if (kpool.shape != (num_pages, Hkv, page_size, d) or vpool.shape != kpool.shape or block_table.shape[0] != B
+            or seqlens.shape != (B,) or (r is not None and r.shape != q.shape)):
+        raise ValueError("shape mismatch between q, pools, block_table, seqlens, r")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    need = plx_decode_workspace_size(B, Hq, Hkv, max_pages * page_size, d, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.plx_decode_paged(_ptr(q), _ptr(r), _ptr(kpool), _ptr(vpool), _ptr(block_table), _ptr(seqlens),
+                               _ptr(out), _ptr(lse), B, Hq, Hkv, num_pages, page_size, max_pages, d, float(scale),
+                               int(num_splits), _ptr(workspace), ws_bytes, _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_decode_paged")
     return out, lse
 
 

@@ -27,7 +27,7 @@ def declared_entry_points():
 
 def test_header_declares_the_boundary():
     names = declared_entry_points()
-    for n in ["plx_fwd", "plx_fwd_train", "plx_bwd", "plx_bwd_workspace_size",
+    for n in ["plx_fwd", "plx_fwd_train", "plx_bwd", "plx_bwd_workspace_size", "plx_decode_paged",
               "plx_decode", "plx_decode_workspace_size", "plx_decode_num_splits",
               "plx_check_device_status", "plx_status_string", "plx_version", "plx_selftest_wait_timeout"]:
         assert n in names
@@ -165,3 +165,25 @@ def test_bwd_argument_errors(plx):
     assert bwd(plx, lse=A + 2) == plx.PLX_ERR_ALIGN
     assert bwd(plx, ws=None) == plx.PLX_ERR_WORKSPACE
     assert bwd(plx, wsb=plx.plx_bwd_workspace_size(1, 2, 1, 8, 64) - 1) == plx.PLX_ERR_WORKSPACE
+
+
+def paged(plx, q=A, r=A, kp=A, vp=A, bt=A, sl=A, out=A, lse=A, B=1, Hq=2, Hkv=1, num_pages=4, ps=16, mp=2,
+          d=64, splits=1, ws=None, wsb=0):
+    return plx.lib.plx_decode_paged(P(q), P(r), P(kp), P(vp), P(bt), P(sl), P(out), P(lse), B, Hq, Hkv, num_pages,
+                                    ps, mp, d, 0.125, splits, P(ws), wsb, None)
+
+
+def test_paged_decode_argument_errors(plx):
+    for kw in [dict(q=None), dict(kp=None), dict(vp=None), dict(bt=None), dict(sl=None), dict(out=None)]:
+        assert paged(plx, **kw) == plx.PLX_ERR_NULL, kw
+    for ps in [0, 8, 24, 100, 8192]:
+        assert paged(plx, ps=ps) == plx.PLX_ERR_SHAPE, ps
+    for kw in [dict(B=0), dict(num_pages=0), dict(mp=0), dict(splits=-1)]:
+        assert paged(plx, **kw) == plx.PLX_ERR_SHAPE, kw
+    assert paged(plx, d=96) == plx.PLX_ERR_HEADDIM
+    assert paged(plx, Hq=3, Hkv=2) == plx.PLX_ERR_GQA
+    assert paged(plx, kp=A + 8) == plx.PLX_ERR_ALIGN
+    assert paged(plx, bt=A + 2) == plx.PLX_ERR_ALIGN
+    need = plx.plx_decode_workspace_size(1, 2, 1, 16 * 32, 64, 2)
+    assert paged(plx, mp=32, splits=2) == plx.PLX_ERR_WORKSPACE
+    assert paged(plx, mp=32, splits=2, ws=A, wsb=need - 1) == plx.PLX_ERR_WORKSPACE
