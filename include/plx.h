@@ -226,6 +226,35 @@ int plx_decode_paged(const void* q, const void* r, const void* kpool, const void
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * plx_kv_append -- writes the new token's key and value of every KV head into
+ * a contiguous cache at the slot after the live keys, before the decode step.
+ *
+ *   knew, vnew [B, Hkv, d] bf16          this step's keys and values
+ *   kcache, vcache [B, Hkv, S_max, d]     written at row seqlens[b] of (b, g)
+ *   seqlens [B] int32, DEVICE             read; when advance != 0, entry b
+ *                                         becomes seqlens[b] + 1 once written
+ *
+ * An entry with seqlens[b] < 0 or >= S_max is left unwritten (and not
+ * advanced).  One small kernel on `stream`; calls on one stream apply in
+ * order.  The pages describe a KV cache that grows by one token per step
+ * (zubnet.ai's Parallax page: a KV cache is still needed); this is that step.
+ */
+int plx_kv_append(const void* knew, const void* vnew, void* kcache, void* vcache,
+                  int32_t* seqlens, int B, int Hkv, int S_max, int d, int advance, void* stream);
+
+/*
+ * plx_kv_append_paged -- plx_kv_append for the page pools of plx_decode_paged
+ * ([num_pages, Hkv, page_size, d]; slot seqlens[b] of sequence b is row
+ * seqlens[b] % page_size of page block_table[b * max_pages + seqlens[b] / page_size]).
+ * An entry whose slot is past max_pages * page_size, or whose page id is
+ * outside [0, num_pages), is left unwritten and not advanced.
+ */
+int plx_kv_append_paged(const void* knew, const void* vnew, void* kpool, void* vpool,
+                        const int32_t* block_table, int32_t* seqlens, int B, int Hkv,
+                        int num_pages, int page_size, int max_pages, int d, int advance,
+                        void* stream);
+
+/*
  * PLX_NOALLOC_SCRATCH_BYTES -- size of the library's fixed device scratch
  * array used by plx_decode_noalloc (16 MiB, held on every GPU that loads the
  * library until the process exits).

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/plx.h"
+#include "plx_append.cuh"
 #include "plx_bwd.cuh"
 #include "plx_decode.cuh"
 #include "plx_fwd.cuh"
@@ -349,6 +350,64 @@ int plx_decode_paged(const void* q, const void* r, const void* kpool, const void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 128) return r ? launch_decode<128, true, true>(km, vm, p, n_hg, st) : launch_decode<128, false, true>(km, vm, p, n_hg, st);
   return r ? launch_decode<64, true, true>(km, vm, p, n_hg, st) : launch_decode<64, false, true>(km, vm, p, n_hg, st);
+}
+
+}  // extern "C"
+
+namespace {
+
+int append_common(const void* knew, const void* vnew, void* kc, void* vc, int32_t* seqlens,
+                  const int32_t* block_table, int B, int Hkv, int S_max, int num_pages, int page_size,
+                  int max_pages, int d, int advance, void* stream) {
+  if (!knew || !vnew || !kc || !vc || !seqlens) return PLX_ERR_NULL;
+  if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
+  if (!aligned16(knew) || !aligned16(vnew) || !aligned16(kc) || !aligned16(vc) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(block_table) & 3u))
+    return PLX_ERR_ALIGN;
+  int dev = 0;
+  int rc = check_arch(&dev);
+  if (rc != PLX_OK) return rc;
+  plx::AppendParams p{};
+  p.knew = static_cast<const __nv_bfloat16*>(knew);
+  p.vnew = static_cast<const __nv_bfloat16*>(vnew);
+  p.kcache = static_cast<__nv_bfloat16*>(kc);
+  p.vcache = static_cast<__nv_bfloat16*>(vc);
+  p.seqlens = seqlens;
+  p.block_table = block_table;
+  p.B = B; p.Hkv = Hkv; p.S_max = S_max;
+  p.num_pages = num_pages; p.page_size = page_size; p.max_pages = max_pages;
+  int shift = 0;
+  while (page_size > 0 && (1 << shift) < page_size) ++shift;
+  p.page_shift = shift;
+  p.advance = advance ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>((B + 7) / 8);
+  if (d == 128)
+    plx::plx_kv_append_kernel<128><<<grid, 256, 0, st>>>(p);
+  else
+    plx::plx_kv_append_kernel<64><<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int plx_kv_append(const void* knew, const void* vnew, void* kcache, void* vcache, int32_t* seqlens, int B,
+                  int Hkv, int S_max, int d, int advance, void* stream) {
+  if (B < 1 || Hkv < 1 || S_max < 1) return PLX_ERR_SHAPE;
+  return append_common(knew, vnew, kcache, vcache, seqlens, nullptr, B, Hkv, S_max, 0, 0, 0, d, advance, stream);
+}
+
+int plx_kv_append_paged(const void* knew, const void* vnew, void* kpool, void* vpool, const int32_t* block_table,
+                        int32_t* seqlens, int B, int Hkv, int num_pages, int page_size, int max_pages, int d,
+                        int advance, void* stream) {
+  if (!block_table) return PLX_ERR_NULL;
+  if (B < 1 || Hkv < 1 || num_pages < 1 || max_pages < 1) return PLX_ERR_SHAPE;
+  if (page_size < 16 || page_size > 4096 || (page_size & (page_size - 1))) return PLX_ERR_SHAPE;
+  if (static_cast<long long>(max_pages) * page_size > 0x7fffffffLL) return PLX_ERR_SHAPE;
+  return append_common(knew, vnew, kpool, vpool, seqlens, block_table, B, Hkv, 0, num_pages, page_size, max_pages,
+                       d, advance, stream);
 }
 
 size_t plx_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {

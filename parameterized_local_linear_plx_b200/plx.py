@@ -47,6 +47,10 @@ _lib.plx_decode.restype = _I
 _lib.plx_decode.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P]
 _lib.plx_decode_paged.restype = _I
 _lib.plx_decode_paged.argtypes = [_P] * 8 + [_I] * 7 + [_F, _I, _P, _SZ, _P]
+_lib.plx_kv_append.restype = _I
+_lib.plx_kv_append.argtypes = [_P] * 5 + [_I] * 5 + [_P]
+_lib.plx_kv_append_paged.restype = _I
+_lib.plx_kv_append_paged.argtypes = [_P] * 6 + [_I] * 7 + [_P]
 _lib.plx_decode_noalloc.restype = _I
 _lib.plx_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]
 _lib.plx_check_device_status.restype = _I
@@ -277,6 +281,46 @@ def plx_decode_paged(q, kpool, vpool, block_table, seqlens, r=None, scale=None, 
     if st != PLX_OK:
         raise PlxError(st, "plx_decode_paged")
     return out, lse
+
+
+def plx_kv_append(knew, vnew, kcache, vcache, seqlens, advance=True, stream=None):
+    """Write knew/vnew [B, Hkv, d] at row seqlens[b] of the caches [B, Hkv, S_max, d];
+    advance seqlens (in place) when asked."""
+    for t, n in ((knew, "knew"), (vnew, "vnew")):
+        _check(t, n, torch.bfloat16, 3)
+    for t, n in ((kcache, "kcache"), (vcache, "vcache")):
+        _check(t, n, torch.bfloat16, 4)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    B, Hkv, d = knew.shape
+    S_max = kcache.shape[2]
+    if vnew.shape != knew.shape or kcache.shape != (B, Hkv, S_max, d) or vcache.shape != kcache.shape \
+            or seqlens.shape != (B,):
+        raise ValueError("shape mismatch between knew, vnew, caches, seqlens")
+    st = _lib.plx_kv_append(_ptr(knew), _ptr(vnew), _ptr(kcache), _ptr(vcache), _ptr(seqlens), B, Hkv, S_max, d,
+                            1 if advance else 0, _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_kv_append")
+
+
+def plx_kv_append_paged(knew, vnew, kpool, vpool, block_table, seqlens, advance=True, stream=None):
+    """plx_kv_append for page pools [num_pages, Hkv, page_size, d] and a block table [B, max_pages]."""
+    for t, n in ((knew, "knew"), (vnew, "vnew")):
+        _check(t, n, torch.bfloat16, 3)
+    for t, n in ((kpool, "kpool"), (vpool, "vpool")):
+        _check(t, n, torch.bfloat16, 4)
+    _check(block_table, "block_table", torch.int32, 2)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    B, Hkv, d = knew.shape
+    num_pages, page_size = kpool.shape[0], kpool.shape[2]
+    max_pages = block_table.shape[1]
+    if vnew.shape != knew.shape or kpool.shape != (num_pages, Hkv, page_size, d) or vpool.shape != kpool.shape \
+            or block_table.shape[0] != B or seqlens.shape != (B,):
+        raise ValueError("shape mismatch between knew, vnew, pools, block_table, seqlens")
+    st = _lib.plx_kv_append_paged(_ptr(knew), _ptr(vnew), _ptr(kpool), _ptr(vpool), _ptr(block_table),
+                                  _ptr(seqlens), B, Hkv, num_pages, page_size, max_pages, d, 1 if advance else 0,
+                                  _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_kv_append_paged")
 
 
 PLX_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024

@@ -27,7 +27,7 @@ def declared_entry_points():
 
 def test_header_declares_the_boundary():
     names = declared_entry_points()
-    for n in ["plx_fwd", "plx_fwd_train", "plx_bwd", "plx_bwd_workspace_size", "plx_decode_paged",
+    for n in ["plx_fwd", "plx_fwd_train", "plx_bwd", "plx_bwd_workspace_size", "plx_decode_paged", "plx_kv_append", "plx_kv_append_paged",
               "plx_decode", "plx_decode_workspace_size", "plx_decode_num_splits",
               "plx_check_device_status", "plx_status_string", "plx_version", "plx_selftest_wait_timeout"]:
         assert n in names
@@ -187,3 +187,18 @@ def test_paged_decode_argument_errors(plx):
     need = plx.plx_decode_workspace_size(1, 2, 1, 16 * 32, 64, 2)
     assert paged(plx, mp=32, splits=2) == plx.PLX_ERR_WORKSPACE
     assert paged(plx, mp=32, splits=2, ws=A, wsb=need - 1) == plx.PLX_ERR_WORKSPACE
+
+
+def test_kv_append_argument_errors(plx):
+    ap = plx.lib.plx_kv_append
+    assert ap(P(None), P(A), P(A), P(A), P(A), 1, 1, 8, 64, 1, None) == plx.PLX_ERR_NULL
+    assert ap(P(A), P(A), P(A), P(A), P(None), 1, 1, 8, 64, 1, None) == plx.PLX_ERR_NULL
+    assert ap(P(A), P(A), P(A), P(A), P(A), 0, 1, 8, 64, 1, None) == plx.PLX_ERR_SHAPE
+    assert ap(P(A), P(A), P(A), P(A), P(A), 1, 1, 0, 64, 1, None) == plx.PLX_ERR_SHAPE
+    assert ap(P(A), P(A), P(A), P(A), P(A), 1, 1, 8, 80, 1, None) == plx.PLX_ERR_HEADDIM
+    assert ap(P(A + 8), P(A), P(A), P(A), P(A), 1, 1, 8, 64, 1, None) == plx.PLX_ERR_ALIGN
+    apg = plx.lib.plx_kv_append_paged
+    assert apg(P(A), P(A), P(A), P(A), P(None), P(A), 1, 1, 4, 16, 2, 64, 1, None) == plx.PLX_ERR_NULL
+    assert apg(P(A), P(A), P(A), P(A), P(A), P(A), 1, 1, 4, 24, 2, 64, 1, None) == plx.PLX_ERR_SHAPE
+    assert apg(P(A), P(A), P(A), P(A), P(A), P(A), 1, 1, 0, 16, 2, 64, 1, None) == plx.PLX_ERR_SHAPE
+    assert apg(P(A), P(A), P(A), P(A), P(A + 2), P(A), 1, 1, 4, 16, 2, 64, 1, None) == plx.PLX_ERR_ALIGN
