@@ -93,6 +93,29 @@ int plx_fwd(const void* q, const void* k, const void* v, const void* r,
             void* stream);
 
 /*
+ * plx_fwd_varlen -- plx_fwd over a batch of packed sequences of different
+ * lengths (variable-length prefill).
+ *
+ *   q, r, out [total, Hq, d] bf16; k, v [total, Hkv, d] bf16   token-major:
+ *              sequence b is tokens cu_seqlens[b] .. cu_seqlens[b+1]-1
+ *   cu_seqlens [B + 1] int32, DEVICE   non-decreasing, cu_seqlens[0] = 0,
+ *              cu_seqlens[B] = total
+ *   lse [Hq, total] fp32 (NULL: skipped)
+ *   max_seqlen >= every sequence's length (rows past it are not computed)
+ *
+ * Each sequence attends only its own tokens (causal: positions within the
+ * sequence).  Values in cu_seqlens outside [0, total] are clamped on the
+ * device, so nothing outside the tensors is addressed.  Same requirements
+ * and errors as plx_fwd, plus PLX_ERR_NULL for cu_seqlens and PLX_ERR_SHAPE
+ * for total < 1.  The pages train on fixed-length windows; packing is the
+ * serving / mixed-length form of the same computation.
+ */
+int plx_fwd_varlen(const void* q, const void* k, const void* v, const void* r,
+                   void* out, float* lse, const int32_t* cu_seqlens,
+                   int B, int Hq, int Hkv, int total, int max_seqlen, int d, int causal,
+                   float scale, void* stream);
+
+/*
  * plx_fwd_train -- plx_fwd for training: the same outputs, plus two per-row
  * values that plx_bwd needs.
  *

@@ -81,6 +81,22 @@ int make_map_3d(CUtensorMap* map, const void* base, int D, long long rows, long 
   return rc == CUDA_SUCCESS ? PLX_OK : PLX_ERR_CUDA;
 }
 
+// A token-major bf16 tensor [rows, planes, D] (packed sequences: a row is a
+// token, a plane a head) as the same 3-D view {D, rows, planes}: the row
+// stride is planes * D elements and the plane stride D elements.  Loads past
+// the last row are zero-filled.
+int make_map_3d_tokens(CUtensorMap* map, const void* base, int D, long long rows, long long planes, int box_rows) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(planes) * static_cast<cuuint64_t>(D) * 2u,
+                           static_cast<cuuint64_t>(D) * 2u};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult rc = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS ? PLX_OK : PLX_ERR_CUDA;
+}
+
 // Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
 template <typename K>
 int ensure_smem(K kernel, int bytes, bool* done) {
@@ -210,17 +226,21 @@ const char* plx_status_string(int status) {
 namespace {
 
 // plx_fwd and plx_fwd_train: obar / sbar non-NULL selects the training kernel.
+// cu_seqlens non-NULL: packed sequences (token-major [total, H, d]), N = the
+// longest sequence.
 int fwd_common(const void* q, const void* k, const void* v, const void* r, void* out, float* lse,
                void* obar, float* sbar, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
-               void* stream) {
+               void* stream, const int* cu_seqlens = nullptr, int total = 0) {
   if (!q || !k || !v || !out) return PLX_ERR_NULL;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return PLX_ERR_SHAPE;
   if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
   if (Hq % Hkv) return PLX_ERR_GQA;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (r && !aligned16(r)) || !aligned16(out) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (obar && !aligned16(obar)) ||
-      (sbar && (reinterpret_cast<uintptr_t>(sbar) & 3u)))
+      (sbar && (reinterpret_cast<uintptr_t>(sbar) & 3u)) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
     return PLX_ERR_ALIGN;
+  const bool packed = cu_seqlens != nullptr;
+  if (packed && total < 1) return PLX_ERR_SHAPE;
   const bool train = obar != nullptr;
   const int G = Hq / Hkv;
   const int pair_heads = (G % 2 == 0) ? 1 : 0;
@@ -235,16 +255,22 @@ int fwd_common(const void* q, const void* k, const void* v, const void* r, void*
 
   CUtensorMap qm, rm, km, vm, om, am;
   const long long pq = static_cast<long long>(B) * Hq, pkv = static_cast<long long>(B) * Hkv;
-  if (make_map_3d(&qm, q, d, N, pq, 16) != PLX_OK || make_map_3d(&km, k, d, N, pkv, plx::kFwdBN) != PLX_OK ||
-      make_map_3d(&vm, v, d, N, pkv, plx::kFwdBN) != PLX_OK || make_map_3d(&om, out, d, N, pq, 16) != PLX_OK)
+  // fixed length: [planes = B * H, rows = N]; packed: [planes = H, rows = total] over token-major storage
+  auto map_q = [&](CUtensorMap* m, const void* base) {
+    return packed ? make_map_3d_tokens(m, base, d, total, Hq, 16) : make_map_3d(m, base, d, N, pq, 16);
+  };
+  auto map_kv = [&](CUtensorMap* m, const void* base) {
+    return packed ? make_map_3d_tokens(m, base, d, total, Hkv, plx::kFwdBN) : make_map_3d(m, base, d, N, pkv, plx::kFwdBN);
+  };
+  if (map_q(&qm, q) != PLX_OK || map_kv(&km, k) != PLX_OK || map_kv(&vm, v) != PLX_OK || map_q(&om, out) != PLX_OK)
     return PLX_ERR_CUDA;
   if (r) {
-    if (make_map_3d(&rm, r, d, N, pq, 16) != PLX_OK) return PLX_ERR_CUDA;
+    if (map_q(&rm, r) != PLX_OK) return PLX_ERR_CUDA;
   } else {
     rm = qm;  // unused
   }
   if (train) {
-    if (make_map_3d(&am, obar, d, N, pq, 16) != PLX_OK) return PLX_ERR_CUDA;
+    if (map_q(&am, obar) != PLX_OK) return PLX_ERR_CUDA;
   } else {
     am = om;  // unused
   }
@@ -252,6 +278,10 @@ int fwd_common(const void* q, const void* k, const void* v, const void* r, void*
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.sbar = sbar;
+  p.obar = static_cast<__nv_bfloat16*>(obar);
+  p.cu_seqlens = cu_seqlens;
+  p.total = total;
+  p.lse_stride = packed ? total : N;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.G = G;
   p.pair_heads = pair_heads; p.n_pairs = n_pairs; p.n_qblocks = n_qblocks;
   p.num_units = static_cast<int>(grid);
@@ -288,6 +318,14 @@ int plx_fwd_train(const void* q, const void* k, const void* v, const void* r, vo
                   void* stream) {
   if (!lse || !obar || (r && !sbar)) return PLX_ERR_NULL;
   return fwd_common(q, k, v, r, out, lse, obar, sbar, B, Hq, Hkv, N, d, causal, scale, stream);
+}
+
+int plx_fwd_varlen(const void* q, const void* k, const void* v, const void* r, void* out, float* lse,
+                   const int32_t* cu_seqlens, int B, int Hq, int Hkv, int total, int max_seqlen, int d, int causal,
+                   float scale, void* stream) {
+  if (!cu_seqlens) return PLX_ERR_NULL;
+  return fwd_common(q, k, v, r, out, lse, nullptr, nullptr, B, Hq, Hkv, max_seqlen, d, causal, scale, stream,
+                    cu_seqlens, total);
 }
 
 int plx_decode_paged(const void* q, const void* r, const void* kpool, const void* vpool,

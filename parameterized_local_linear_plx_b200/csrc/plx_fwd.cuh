@@ -89,6 +89,16 @@ struct FwdParams {
   int causal;
   float scale_log2;    // scale * log2(e)
   float* sbar;         // [B, Hq, N] s_bar = c / l (training forward only)
+  __nv_bfloat16* obar; // o_bar (training forward only; written by TMA, by this pointer only for
+                       // the last rows of a packed sequence)
+  // variable-length packed sequences (nullptr: fixed length N).  Then q, r,
+  // out are [total, Hq, D] and k, v [total, Hkv, D] (token-major; the tensor
+  // maps take a head as the plane and a token as the row), sequence b is rows
+  // cu_seqlens[b] .. cu_seqlens[b+1]-1, N is the longest length, and lse /
+  // sbar are [Hq, total].
+  const int* cu_seqlens;
+  int total;
+  long long lse_stride;  // N (fixed length) or total (packed)
 };
 
 template <int D, bool HAS_R, bool SAVE_AUX>
@@ -120,8 +130,11 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 
   // ---- work units: index u -> (b, head pair / head, query block), longest
   // causal rows first; CTA c takes u = c, c + gridDim.x, ...
+  // (packed sequences: a unit whose query block starts past its sequence is
+  // empty, nkv = 0, and every role skips it the same way)
   struct Unit {
     int b, hp, qb, nkv;
+    int N, base;  // the sequence's length and first row
   };
   auto unit_of = [&](int u) {
     Unit w;
@@ -130,15 +143,27 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const int rem = u % per;
     w.b = rem / p.n_pairs;
     w.hp = rem % p.n_pairs;
+    w.base = 0;
+    w.N = p.N;
+    if (p.cu_seqlens) {  // clamped so that no row outside [0, total) is ever addressed
+      w.base = min(max(__ldg(p.cu_seqlens + w.b), 0), p.total);
+      w.N = min(max(__ldg(p.cu_seqlens + w.b + 1) - w.base, 0), min(p.total - w.base, p.N));
+    }
+    const int first_row = p.pair_heads ? w.qb * kFwdBM : 2 * w.qb * kFwdBM;
     const int last_row = p.pair_heads ? w.qb * kFwdBM + kFwdBM - 1 : (2 * w.qb + 2) * kFwdBM - 1;
-    const int qmax = min(p.N - 1, last_row);
-    const int nkv_all = (p.N + kFwdBN - 1) / kFwdBN;
-    w.nkv = p.causal ? min(nkv_all, qmax / kFwdBN + 1) : nkv_all;
+    const int qmax = min(w.N - 1, last_row);
+    const int nkv_all = (w.N + kFwdBN - 1) / kFwdBN;
+    w.nkv = first_row >= w.N ? 0 : (p.causal ? min(nkv_all, qmax / kFwdBN + 1) : nkv_all);
     return w;
   };
   // tile t in {0, 1} of a unit: query head and first query row
   auto head_of = [&](const Unit& w, int t) { return p.pair_heads ? 2 * w.hp + t : w.hp; };
   auto row0_of = [&](const Unit& w, int t) { return p.pair_heads ? w.qb * kFwdBM : (2 * w.qb + t) * kFwdBM; };
+  // tensor-map plane of a query head and of its KV head (packed: the head alone)
+  auto qplane_of = [&](const Unit& w, int t) { return p.cu_seqlens ? head_of(w, t) : w.b * p.Hq + head_of(w, t); };
+  auto kvplane_of = [&](const Unit& w) {
+    return p.cu_seqlens ? head_of(w, 0) / p.G : w.b * p.Hkv + head_of(w, 0) / p.G;
+  };
 
   if (threadIdx.x == 0) {
     // arrivals per phase: p_ready and o_free get one arrival from each of the
@@ -188,16 +213,17 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       int kv = 0;        // K/V tiles issued so far: ring stage kv % NS, phase (kv / NS) & 1
       int n_unit = 0;    // units whose Q/R were issued
       int issued_k = 0, issued_v = 0;
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++n_unit) {
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
         const Unit w = unit_of(u);
+        if (w.nkv == 0) continue;
         // the previous unit's last score MMA must have read Q/R
         if (n_unit > 0 && !mbar_wait(smem_u32(qr_empty), (n_unit - 1) & 1, kErrFwdLoad)) { ok = false; break; }
         for (int t = 0; t < 2; ++t) {
           const uint32_t fb = smem_u32(&qr_full[t]);
           mbar_arrive_expect_tx(fb, HAS_R ? Cfg::kQRBytes : Cfg::kQRBytes / 2);
           const uint32_t base = smem_u32(smem + Cfg::kOffQR + t * Cfg::kQRBytes);
-          const int plane = w.b * p.Hq + head_of(w, t);
-          const int row0 = row0_of(w, t);
+          const int plane = qplane_of(w, t);
+          const int row0 = w.base + row0_of(w, t);
 #pragma unroll
           for (int wq = 0; wq < 4; ++wq)
 #pragma unroll
@@ -207,7 +233,7 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
               if (HAS_R) tma_load_3d(&rmap, dst + 16 * 128, fb, cb * 64, row0 + 16 * wq, plane);
             }
         }
-        const int plane_kv = w.b * p.Hkv + head_of(w, 0) / p.G;
+        const int plane_kv = kvplane_of(w);
         for (int j = 0; j < w.nkv; ++j, ++kv) {
           const int s = kv % NS;
           if (kv >= NS && !mbar_wait(smem_u32(&k_empty[s]), ((kv / NS) - 1) & 1, kErrFwdLoad)) { ok = false; break; }
@@ -217,7 +243,7 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             const uint32_t dst = smem_u32(smem + Cfg::kOffK + s * Cfg::kKVBytes);
 #pragma unroll
             for (int cb = 0; cb < Cfg::kCB; ++cb)
-              tma_load_3d(&kmap, dst + cb * Cfg::kBlock, fb, cb * 64, j * kFwdBN, plane_kv);
+              tma_load_3d(&kmap, dst + cb * Cfg::kBlock, fb, cb * 64, w.base + j * kFwdBN, plane_kv);
             issued_k = kv + 1;
           }
           if (kv >= NS && !mbar_wait(smem_u32(&v_empty[s]), ((kv / NS) - 1) & 1, kErrFwdLoad)) { ok = false; break; }
@@ -227,10 +253,11 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             const uint32_t dst = smem_u32(smem + Cfg::kOffV + s * Cfg::kKVBytes);
 #pragma unroll
             for (int cb = 0; cb < Cfg::kCB; ++cb)
-              tma_load_3d(&vmap, dst + cb * Cfg::kBlock, fb, cb * 64, j * kFwdBN, plane_kv);
+              tma_load_3d(&vmap, dst + cb * Cfg::kBlock, fb, cb * 64, w.base + j * kFwdBN, plane_kv);
             issued_v = kv + 1;
           }
         }
+        ++n_unit;
       }
       if (!ok) {  // let every issued load land before the CTA can exit
         if (n_unit > 0)
@@ -282,8 +309,9 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 
       int kv = 0;       // global K/V tile index of the current unit's first tile
       int n_unit = 0;
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++n_unit) {
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
         const Unit w = unit_of(u);
+        if (w.nkv == 0) continue;
         const uint32_t uph = n_unit & 1;
         ok = mbar_wait(smem_u32(&qr_full[0]), uph, kErrFwdMma) && mbar_wait(smem_u32(&qr_full[1]), uph, kErrFwdMma) &&
              mbar_wait(smem_u32(&k_full[kv % NS]), (kv / NS) & 1, kErrFwdMma);
@@ -322,6 +350,7 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           }
         }
         kv += w.nkv;
+        ++n_unit;
       }
       // Every MMA issued must be complete before tensor memory is released.
       tc::commit(smem_u32(&fin[0]));
@@ -347,8 +376,9 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const uint32_t to1 = tmem + lane_a + col_o(t);
     const uint32_t to2 = tmem + lane_s + col_o(t);
     int kv = 0, n_unit = 0;
-    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++n_unit) {
+    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
       const Unit w = unit_of(u);
+      if (w.nkv == 0) continue;
       const int q0 = row0_of(w, t);
       const int q_lo = q0 + 16 * wq + (lane >> 2);
       const int q_hi = q_lo + 8;
@@ -378,13 +408,13 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         // Masked scores become -inf in place; the max is taken on raw q.k and
         // scaled afterwards (scale_log2 > 0), and the scale folds into exp2's FMA.
         const int kbase = j * kFwdBN;
-        const bool need_mask = (p.causal && kbase + kFwdBN - 1 > q0) || (kbase + kFwdBN > p.N);
+        const bool need_mask = (p.causal && kbase + kFwdBN - 1 > q0) || (kbase + kFwdBN > w.N);
         if (need_mask) {
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
             const int key = kbase + 64 * (i >> 5) + 8 * ((i & 31) >> 2) + 2 * c4 + (i & 1);
             const int q = (i & 2) ? q_hi : q_lo;
-            const bool valid = key < p.N && (!p.causal || key <= q);
+            const bool valid = key < w.N && (!p.causal || key <= q);
             if (!valid) ra[i] = 0xFF800000u;  // -inf
           }
         }
@@ -492,7 +522,8 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const float inv_lo = l_lo > 0.f ? 1.f / l_lo : 0.f;
       const float inv_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
       const float sb_lo = c_lo * inv_lo, sb_hi = c_hi * inv_hi;  // s_bar = c / l
-      const size_t plane = static_cast<size_t>(w.b) * p.Hq + head_of(w, t);
+      const size_t plane = static_cast<size_t>(qplane_of(w, t));
+      const size_t lse_row0 = plane * p.lse_stride + w.base;  // lse / sbar index of the sequence's row 0
       // This warp's 16 output rows are staged in shared memory in the 128-byte
       // swizzled layout of the output tensor map and written by one TMA store.
       const uint32_t stage = smem_u32(smem + Cfg::kOffOut) + (t * 4 + wq) * Cfg::kOutWarpBytes;
@@ -532,15 +563,35 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         if (lane == 0) mbar_arrive(smem_u32(&o_free[t]));
       }
       if (p.lse && c4 == 0) {
-        if (q_lo < p.N) p.lse[plane * p.N + q_lo] = l_lo > 0.f ? (m_lo + __log2f(l_lo)) * kLn2 : -INFINITY;
-        if (q_hi < p.N) p.lse[plane * p.N + q_hi] = l_hi > 0.f ? (m_hi + __log2f(l_hi)) * kLn2 : -INFINITY;
+        if (q_lo < w.N) p.lse[lse_row0 + q_lo] = l_lo > 0.f ? (m_lo + __log2f(l_lo)) * kLn2 : -INFINITY;
+        if (q_hi < w.N) p.lse[lse_row0 + q_hi] = l_hi > 0.f ? (m_hi + __log2f(l_hi)) * kLn2 : -INFINITY;
       }
       fence_proxy_async_smem();
       __syncwarp();
       const int row0 = q0 + 16 * wq;
-      if (lane == 0 && row0 < p.N) {
+      // Packed sequences: a 16-row group that runs past its sequence would
+      // overwrite the next sequence's rows, so its live rows are copied out of
+      // the staging block with plain stores instead of the TMA store.
+      const bool partial = p.cu_seqlens != nullptr && row0 < w.N && row0 + 16 > w.N;
+      auto copy_rows = [&](__nv_bfloat16* dst) {
+        const int nrows = w.N - row0;
+        for (int i = lane; i < nrows * Cfg::kCB * 8; i += 32) {
+          const int rr = i / (Cfg::kCB * 8), cb = (i / 8) % Cfg::kCB, c = i % 8;
+          uint4 v;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(stage + cb * 2048 + rr * 128 + ((c ^ (rr & 7)) << 4)));
+          const size_t tok = static_cast<size_t>(w.base + row0 + rr);
+          *reinterpret_cast<uint4*>(dst + (tok * p.Hq + head_of(w, t)) * D + cb * 64 + c * 8) = v;
+        }
+        __syncwarp();
+      };
+      if (partial) {
+        copy_rows(p.out);
+      } else if (lane == 0 && row0 < w.N) {
 #pragma unroll
-        for (int cb = 0; cb < Cfg::kCB; ++cb) tma_store_3d(&omap, stage + cb * 2048, cb * 64, row0, static_cast<int>(plane));
+        for (int cb = 0; cb < Cfg::kCB; ++cb)
+          tma_store_3d(&omap, stage + cb * 2048, cb * 64, w.base + row0, static_cast<int>(plane));
         bulk_commit();
       }
       if (SAVE_AUX) {
@@ -548,8 +599,8 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         // output) for the backward.  o_bar goes through the same staging
         // block once the output store has read it.
         if (p.sbar && c4 == 0) {
-          if (q_lo < p.N) p.sbar[plane * p.N + q_lo] = sb_lo;
-          if (q_hi < p.N) p.sbar[plane * p.N + q_hi] = sb_hi;
+          if (q_lo < w.N) p.sbar[lse_row0 + q_lo] = sb_lo;
+          if (q_hi < w.N) p.sbar[lse_row0 + q_hi] = sb_hi;
         }
         if (lane == 0) bulk_wait_read();
         __syncwarp();
@@ -576,13 +627,17 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         if (lane == 0) mbar_arrive(smem_u32(&o_free[t]));
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && row0 < p.N) {
+        if (partial) {
+          copy_rows(p.obar);
+        } else if (lane == 0 && row0 < w.N) {
 #pragma unroll
-          for (int cb = 0; cb < Cfg::kCB; ++cb) tma_store_3d(&amap, stage + cb * 2048, cb * 64, row0, static_cast<int>(plane));
+          for (int cb = 0; cb < Cfg::kCB; ++cb)
+            tma_store_3d(&amap, stage + cb * 2048, cb * 64, w.base + row0, static_cast<int>(plane));
           bulk_commit();
         }
       }
       kv += w.nkv;
+      ++n_unit;
     }
     if (lane == 0) bulk_wait_all();  // output stores complete before exit
     tc::fence_before_sync();

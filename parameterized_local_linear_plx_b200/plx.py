@@ -33,6 +33,8 @@ _lib.plx_status_string.restype = ctypes.c_char_p
 _lib.plx_status_string.argtypes = [_I]
 _lib.plx_fwd.restype = _I
 _lib.plx_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
+_lib.plx_fwd_varlen.restype = _I
+_lib.plx_fwd_varlen.argtypes = [_P] * 7 + [_I] * 7 + [_F, _P]
 _lib.plx_fwd_train.restype = _I
 _lib.plx_fwd_train.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
 _lib.plx_bwd_workspace_size.restype = _SZ
@@ -135,6 +137,35 @@ def plx_fwd(q, k, v, r=None, causal=True, scale=None, out=None, lse=None, return
                       1 if causal else 0, float(scale), _stream(stream))
     if st != PLX_OK:
         raise PlxError(st, "plx_fwd")
+    return out, lse
+
+
+def plx_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, r=None, causal=True, scale=None, out=None, lse=None,
+                   return_lse=True, stream=None):
+    """Packed variable-length forward.  q, r [total, Hq, d], k, v [total, Hkv, d]
+    bf16; cu_seqlens [B+1] int32 on the device; max_seqlen (host int) >= every
+    length.  Returns (out [total, Hq, d] bf16, lse [Hq, total] fp32 or None)."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k, "k", torch.bfloat16, 3)
+    _check(v, "v", torch.bfloat16, 3)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    if r is not None:
+        _check(r, "r", torch.bfloat16, 3)
+    total, Hq, d = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.shape[0] - 1
+    if k.shape != (total, Hkv, d) or v.shape != k.shape or (r is not None and r.shape != q.shape) or B < 1:
+        raise ValueError("shape mismatch between q, k, v, r, cu_seqlens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, total), device=q.device, dtype=torch.float32)
+    st = _lib.plx_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(out), _ptr(lse), _ptr(cu_seqlens), B, Hq,
+                             Hkv, total, int(max_seqlen), d, 1 if causal else 0, float(scale), _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_fwd_varlen")
     return out, lse
 
 

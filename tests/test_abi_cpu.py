@@ -27,7 +27,7 @@ def declared_entry_points():
 
 def test_header_declares_the_boundary():
     names = declared_entry_points()
-    for n in ["plx_fwd", "plx_fwd_train", "plx_bwd", "plx_bwd_workspace_size", "plx_decode_paged", "plx_kv_append", "plx_kv_append_paged",
+    for n in ["plx_fwd", "plx_fwd_train", "plx_bwd", "plx_bwd_workspace_size", "plx_decode_paged", "plx_kv_append", "plx_kv_append_paged", "plx_fwd_varlen",
               "plx_decode", "plx_decode_workspace_size", "plx_decode_num_splits",
               "plx_check_device_status", "plx_status_string", "plx_version", "plx_selftest_wait_timeout"]:
         assert n in names
@@ -202,3 +202,15 @@ def test_kv_append_argument_errors(plx):
     assert apg(P(A), P(A), P(A), P(A), P(A), P(A), 1, 1, 4, 24, 2, 64, 1, None) == plx.PLX_ERR_SHAPE
     assert apg(P(A), P(A), P(A), P(A), P(A), P(A), 1, 1, 0, 16, 2, 64, 1, None) == plx.PLX_ERR_SHAPE
     assert apg(P(A), P(A), P(A), P(A), P(A + 2), P(A), 1, 1, 4, 16, 2, 64, 1, None) == plx.PLX_ERR_ALIGN
+
+
+def test_varlen_argument_errors(plx):
+    vf = plx.lib.plx_fwd_varlen
+    args = lambda **kw: [P(kw.get(n, A)) for n in ("q", "k", "v", "r", "out", "lse", "cu")]
+    assert vf(*args(cu=None), 2, 2, 1, 100, 64, 64, 1, 0.125, None) == plx.PLX_ERR_NULL
+    assert vf(*args(q=None), 2, 2, 1, 100, 64, 64, 1, 0.125, None) == plx.PLX_ERR_NULL
+    assert vf(*args(), 2, 2, 1, 0, 64, 64, 1, 0.125, None) == plx.PLX_ERR_SHAPE      # total < 1
+    assert vf(*args(), 2, 2, 1, 100, 0, 64, 1, 0.125, None) == plx.PLX_ERR_SHAPE     # max_seqlen < 1
+    assert vf(*args(), 2, 2, 1, 100, 64, 48, 1, 0.125, None) == plx.PLX_ERR_HEADDIM
+    assert vf(*args(), 2, 3, 2, 100, 64, 64, 1, 0.125, None) == plx.PLX_ERR_GQA
+    assert vf(*args(cu=A + 2), 2, 2, 1, 100, 64, 64, 1, 0.125, None) == plx.PLX_ERR_ALIGN
