@@ -414,6 +414,9 @@ def run_gpu(args, world, rank, local):
     # ---- the same decode step on a paged cache (block tables), timed on its own
     paged = run_paged(plx, args, dev, stream, world, local, d_bytes, hbm, peak_src)
 
+    # ---- packed variable-length prefill with the same token count (timed on its own)
+    varlen = run_varlen(plx, args, dev, stream, world, local, tf_peak, peak_src, tf_key)
+
     # ---- training backward of the prefill shape (timed on its own; not part of the step)
     bwd = run_backward(plx, args, dev, stream, world, local, pq, pk, pv, pr, peaks, peak_src)
 
@@ -443,6 +446,7 @@ def run_gpu(args, world, rank, local):
             "roofline_decode": roof_dec,
             "e2e": e2e,
             "decode_paged": paged,
+            "prefill_varlen": varlen,
             "backward": bwd,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
@@ -489,6 +493,47 @@ def run_paged(plx, args, dev, stream, world, local, d_bytes, hbm, peak_src):
                        f"pools [pages, Hkv, page_size, d], random page assignment")
     res["peak_source"] = f"{peak_src} hbm_gbs"
     return res
+
+
+VARLEN_LENS = [4096, 1, 2048, 777, 1024, 3000, 64, 65, 512, 1500, 4000, 129, 333, 2500, 100, 900,
+               4096, 2048, 1200, 3100]  # 31,493 tokens in 20 sequences of 1 .. 4096
+
+
+def run_varlen(plx, args, dev, stream, world, local, tf_peak, peak_src, tf_key):
+    """plx_fwd_varlen on 20 packed causal sequences of 1 .. 4096 tokens
+    (31,493 tokens, about the prefill step's 32,768), Hq=16, Hkv=8, d=128."""
+    import torch
+    lens = VARLEN_LENS if not args.small else VARLEN_LENS[:5]
+    total = sum(lens)
+    g = torch.Generator(device=dev).manual_seed(300 + local)
+    mk = lambda h: (torch.randn(total, h, PRE["d"], generator=g, device=dev)).bfloat16()
+    q, k, v = mk(PRE["Hq"]), mk(PRE["Hkv"]), mk(PRE["Hkv"])
+    r = (0.1 * torch.randn(total, PRE["Hq"], PRE["d"], generator=g, device=dev)).bfloat16()
+    cu = torch.tensor([0] + list(torch.cumsum(torch.tensor(lens), 0)), dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(PRE["Hq"], total, dtype=torch.float32, device=dev)
+    for _ in range(max(3, args.warmup)):
+        plx.plx_fwd_varlen(q, k, v, cu, max(lens), r, out=out, lse=lse, stream=stream)
+    steps = max(1, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(steps):
+        plx.plx_fwd_varlen(q, k, v, cu, max(lens), r, out=out, lse=lse, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    st = plx.plx_check_device_status(stream)
+    if st != plx.PLX_OK:
+        raise RuntimeError(f"device status after the packed prefill: {plx.plx_status_string(st)}")
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+    flops = sum(8 * PRE["d"] * (n * (n + 1) // 2) * PRE["Hq"] for n in lens)
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"{len(lens)} packed causal sequences of 1..{max(lens)} tokens ({total} tokens), "
+                        f"Hq={PRE['Hq']} Hkv={PRE['Hkv']} d={PRE['d']}, out+lse",
+            "tflops": world * achieved, "ms_per_step": ms, "flops_per_step": flops,
+            "frac_of_peak": achieved / tf_peak, "peak_source": f"{peak_src} {tf_key}"}
 
 
 def inputs_mod():
