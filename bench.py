@@ -274,6 +274,19 @@ def oracle_decode_sample(q, r, kc, vc, sl, budget_s=10.0, max_entries=None):
     return done, time.perf_counter() - t0, nbytes
 
 
+def oracle_explicit_tiny():
+    """Seconds the explicit-Sigma oracle takes on the tiny prefill (B=1, H=1,
+    N=256, d=64, causal, fp32 draws rounded to bf16)."""
+    import torch
+    import oracle
+    from parameterized_local_linear_plx_b200 import inputs
+    q, k, v, r = inputs.prefill_inputs(1, 1, 1, 256, 64, seed=0, dtype=torch.float32)
+    q, k, v, r = (t.bfloat16() for t in (q, k, v, r))
+    t0 = time.perf_counter()
+    oracle.prefill_explicit(q, k, v, r, causal=True)
+    return time.perf_counter() - t0
+
+
 def bench_config(world):
     """The `config` object of the JSON line, identical in both arms."""
     return {
@@ -427,7 +440,8 @@ def run_gpu(args, world, rank, local):
         n, secs, nb = oracle_decode_sample(qh, rh, kh, vh, slh, budget_s=10.0)
         cpu = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{n} (b) entries of the B={DEC['B']} decode step, cycling (each: all {DEC['Hq']} "
-                         f"heads x {DEC['S']} keys), effective-weight fp64 form, {secs:.1f} s"}
+                         f"heads x {DEC['S']} keys), effective-weight fp64 form, {secs:.1f} s",
+               "explicit_tiny_prefill_s": oracle_explicit_tiny()}
 
     clocks = clk.summary()
     if rank == 0:
@@ -436,9 +450,11 @@ def run_gpu(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": bench_config(world),
-            "decode": {"gbs": value, "us_per_step": dec_avg * 1e3, "bytes_per_step": d_bytes, "splits": n_splits,
+            "decode": {"gbs": value, "us_per_step": dec_avg * 1e3, "us_median": statistics.median(dec_ms) * 1e3,
+                       "bytes_per_step": d_bytes, "splits": n_splits,
                        "tflops": world * d_flops / (dec_avg * 1e-3) / 1e12},
-            "prefill": {"tflops": prefill_tflops, "ms_per_step": pre_avg, "flops_per_step": p_flops,
+            "prefill": {"tflops": prefill_tflops, "ms_per_step": pre_avg, "ms_median": statistics.median(pre_ms),
+                        "flops_per_step": p_flops,
                         "gbs_io": world * prefill_bytes(**PRE) / (pre_avg * 1e-3) / 1e9,
                         "roofline": roof_pre},
             # the dominant kernel of the step by time is the prefill kernel
