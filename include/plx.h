@@ -278,6 +278,52 @@ int plx_kv_append_paged(const void* knew, const void* vnew, void* kpool, void* v
                         void* stream);
 
 /*
+ * Context-parallel decode: the KV cache of each sequence is split along the
+ * sequence over `ranks` GPUs (rank r holds a contiguous slice of the keys).
+ * Each rank computes the partial state of its slice with
+ * plx_decode_partial, the ranks all-gather the partials (a collective the
+ * caller runs, e.g. NCCL all-gather into [ranks, ...]), and every rank merges
+ * them with plx_decode_merge.  The partial state of a set of keys is the
+ * streamed form's 5-tuple (news.chathome.org, "Parallax: ...", section
+ * "Hardware argument"): m (running max of the scaled scores, log2 units),
+ * l = sum p, c = sum p s, O1 = sum p v, O2 = sum p s v; the merge rescales
+ * each tuple to the common max and sums, as the split-KV combine does.
+ *
+ * plx_decode_partial_size -- bytes of the partial block of one rank:
+ *   B * Hq * splits * (2d + 4) fp32, where splits is the count the kernel
+ *   uses: plx_decode_num_splits for these shapes when num_splits == 0, else
+ *   num_splits rounded so that every split is a whole number of 64-key tiles
+ *   (the byte count gives it).  Every rank must use the same count.
+ */
+size_t plx_decode_partial_size(int B, int Hq, int Hkv, int S_max, int d, int num_splits);
+
+/*
+ * plx_decode_partial -- the partial states of this rank's slice of the keys.
+ *   q, r, kcache, vcache, scale, num_splits: as plx_decode, where the caches
+ *   hold this rank's slice [B, Hkv, S_max, d]: keys key_offset ..
+ *   key_offset + S_max - 1 of every sequence.
+ *   seqlens [B] int32, DEVICE: the sequences' full lengths; the slice's live
+ *   keys are min(max(seqlens[b] - key_offset, 0), S_max).
+ *   partial [B, Hq, splits, 2d + 4] fp32, DEVICE: per (b, h, split)
+ *   m (log2 units; -inf for an empty split), l, c, pad, O1[d], O2[d].
+ * Errors as plx_decode; PLX_ERR_WORKSPACE when partial_bytes is too small,
+ * PLX_ERR_SHAPE for a negative key_offset.
+ */
+int plx_decode_partial(const void* q, const void* r, const void* kcache, const void* vcache,
+                       const int32_t* seqlens, int key_offset, int B, int Hq, int Hkv, int S_max,
+                       int d, float scale, int num_splits, float* partial, size_t partial_bytes,
+                       void* stream);
+
+/*
+ * plx_decode_merge -- out and lse from the gathered partials of all ranks.
+ *   partials [ranks, B, Hq, num_splits, 2d + 4] fp32, DEVICE (rank-major)
+ *   out [B, Hq, d] bf16; lse [B, Hq] fp32 (NULL: skipped)
+ * A row with no live key in any rank gives out = 0, lse = -inf.
+ */
+int plx_decode_merge(const float* partials, int ranks, int B, int Hq, int d, int num_splits,
+                     void* out, float* lse, void* stream);
+
+/*
  * PLX_NOALLOC_SCRATCH_BYTES -- size of the library's fixed device scratch
  * array used by plx_decode_noalloc (16 MiB, held on every GPU that loads the
  * library until the process exits).

@@ -1,0 +1,52 @@
+"""Context-parallel decode over torch.distributed: one rank per GPU, each
+holding a contiguous slice of every sequence's KV cache.
+
+Every rank computes the partial states of its slice (plx_decode_partial),
+the ranks all-gather them in rank order (the one exchange step: B * Hq *
+splits * (2d + 4) fp32 per rank, over NCCL on NVLink), and every rank merges
+them (plx_decode_merge).  The slices follow one another: rank r holds keys
+r * slice_len .. (r + 1) * slice_len - 1 of every sequence.
+
+The arithmetic runs in the library's kernels; this module only plans the
+slices and moves the partial states.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+
+def slice_start(rank: int, slice_len: int) -> int:
+    """Global index of the first key of `rank`'s slice."""
+    return rank * slice_len
+
+
+def gather_partials(partial: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gather one partial block per rank into [world, *partial.shape], rank-major."""
+    world = dist.get_world_size(group)
+    part = partial.contiguous()
+    # the ranks' blocks concatenated along the first dimension (the layout every
+    # backend accepts), then viewed rank-major
+    out = torch.empty((world * part.shape[0],) + tuple(part.shape[1:]), dtype=part.dtype, device=part.device)
+    dist.all_gather_into_tensor(out, part, group=group)
+    return out.view((world,) + tuple(part.shape))
+
+
+def context_parallel_decode(q, kslice, vslice, seqlens, r=None, scale=None, num_splits=0, group=None,
+                            return_lse=True, stream=None):
+    """One decode step with the KV cache split along the sequence over the ranks of `group`.
+
+    q, r [B, Hq, d] bf16 (the same on every rank); kslice, vslice
+    [B, Hkv, slice_len, d] bf16: this rank's slice; seqlens [B] int32: the full
+    lengths (the same on every rank).  Every rank returns the full (out, lse).
+    num_splits must resolve to the same count on every rank (0: automatic,
+    which depends on the shapes only).
+    """
+    from . import plx
+
+    rank = dist.get_rank(group)
+    slice_len = kslice.shape[2]
+    partial = plx.plx_decode_partial(q, kslice, vslice, seqlens, r, key_offset=slice_start(rank, slice_len),
+                                     scale=scale, num_splits=num_splits, stream=stream)
+    gathered = gather_partials(partial, group)
+    return plx.plx_decode_merge(gathered, return_lse=return_lse, stream=stream)

@@ -149,8 +149,8 @@ int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const plx::Decod
   dim3 grid(p.splits, p.Hkv * n_hg, p.B);
   kern<<<grid, plx::kDecThreads, Cfg::kSmemBytes, st>>>(km, vm, p);
   if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
-  if (p.splits > 1) {
-    plx::plx_decode_combine_kernel<D><<<p.B * p.Hq, D, 0, st>>>(p.ws, p.out, p.lse, p.splits);
+  if (p.splits > 1 && !p.partial_out) {
+    plx::plx_decode_combine_kernel<D><<<p.B * p.Hq, D, 0, st>>>(p.ws, p.out, p.lse, p.splits, 1, 0);
     if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
   }
   return PLX_OK;
@@ -519,21 +519,28 @@ size_t plx_decode_workspace_size(int B, int Hq, int Hkv, int S_max, int d, int n
   return workspace_bytes_for(B, Hq, d, plan_splits(B, Hq, Hkv, S_max, num_splits).splits);
 }
 
-int plx_decode(const void* q, const void* r, const void* kcache, const void* vcache,
-               const int32_t* seqlens, void* out, float* lse, int B, int Hq, int Hkv, int S_max,
-               int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
-               void* stream) {
-  if (!q || !kcache || !vcache || !seqlens || !out) return PLX_ERR_NULL;
+}  // extern "C"
+
+namespace {
+
+// plx_decode, or (partial_out) plx_decode_partial: the same validation and
+// launch; partial_out writes every split's partial state to `workspace` and
+// never runs the combine.
+int decode_common(const void* q, const void* r, const void* kcache, const void* vcache, const int32_t* seqlens,
+                  void* out, float* lse, int B, int Hq, int Hkv, int S_max, int d, float scale, int num_splits,
+                  void* workspace, size_t workspace_bytes, void* stream, bool partial_out, int key_offset = 0) {
+  if (!q || !kcache || !vcache || !seqlens || (!out && !partial_out)) return PLX_ERR_NULL;
   if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || num_splits < 0) return PLX_ERR_SHAPE;
   if (B > 65535) return PLX_ERR_SHAPE;
   if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
   if (Hq % Hkv) return PLX_ERR_GQA;
   if (!aligned16(q) || (r && !aligned16(r)) || !aligned16(kcache) || !aligned16(vcache) ||
-      !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+      (out && !aligned16(out)) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return PLX_ERR_ALIGN;
   const SplitPlan plan = plan_splits(B, Hq, Hkv, S_max, num_splits);
-  const size_t need = workspace_bytes_for(B, Hq, d, plan.splits);
+  const size_t need = partial_out ? static_cast<size_t>(B) * Hq * plan.splits * (2 * d + 4) * sizeof(float)
+                                  : workspace_bytes_for(B, Hq, d, plan.splits);
   if (need > 0) {
     if (!workspace || workspace_bytes < need) return PLX_ERR_WORKSPACE;
     if (!aligned16(workspace)) return PLX_ERR_ALIGN;
@@ -557,14 +564,66 @@ int plx_decode(const void* q, const void* r, const void* kcache, const void* vca
   p.r = static_cast<const __nv_bfloat16*>(r);
   p.seqlens = seqlens;
   p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
+  p.lse = partial_out ? nullptr : lse;
   p.ws = static_cast<float*>(workspace);
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.S_max = S_max; p.G = G; p.n_hgroups = n_hg;
   p.splits = plan.splits; p.chunk = plan.chunk;
+  p.partial_out = partial_out ? 1 : 0;
+  p.key_offset = key_offset;
   p.scale_log2 = scale * plx::kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 128) return r ? launch_decode<128, true, false>(km, vm, p, n_hg, st) : launch_decode<128, false, false>(km, vm, p, n_hg, st);
   return r ? launch_decode<64, true, false>(km, vm, p, n_hg, st) : launch_decode<64, false, false>(km, vm, p, n_hg, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int plx_decode(const void* q, const void* r, const void* kcache, const void* vcache,
+               const int32_t* seqlens, void* out, float* lse, int B, int Hq, int Hkv, int S_max,
+               int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
+               void* stream) {
+  return decode_common(q, r, kcache, vcache, seqlens, out, lse, B, Hq, Hkv, S_max, d, scale, num_splits,
+                       workspace, workspace_bytes, stream, false);
+}
+
+size_t plx_decode_partial_size(int B, int Hq, int Hkv, int S_max, int d, int num_splits) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128) || num_splits < 0) return 0;
+  return static_cast<size_t>(B) * Hq * plan_splits(B, Hq, Hkv, S_max, num_splits).splits * (2 * d + 4) *
+         sizeof(float);
+}
+
+int plx_decode_partial(const void* q, const void* r, const void* kcache, const void* vcache,
+                       const int32_t* seqlens, int key_offset, int B, int Hq, int Hkv, int S_max, int d,
+                       float scale, int num_splits, float* partial, size_t partial_bytes, void* stream) {
+  if (!partial) return PLX_ERR_NULL;
+  if (key_offset < 0) return PLX_ERR_SHAPE;
+  return decode_common(q, r, kcache, vcache, seqlens, nullptr, nullptr, B, Hq, Hkv, S_max, d, scale, num_splits,
+                       partial, partial_bytes, stream, true, key_offset);
+}
+
+int plx_decode_merge(const float* partials, int ranks, int B, int Hq, int d, int num_splits, void* out, float* lse,
+                     void* stream) {
+  if (!partials || !out) return PLX_ERR_NULL;
+  if (ranks < 1 || B < 1 || Hq < 1 || num_splits < 1) return PLX_ERR_SHAPE;
+  if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
+  if (!aligned16(partials) || !aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return PLX_ERR_ALIGN;
+  const long long rows = static_cast<long long>(B) * Hq;
+  if (rows > 0x7fffffffLL) return PLX_ERR_SHAPE;
+  int dev = 0;
+  int rc = check_arch(&dev);
+  if (rc != PLX_OK) return rc;
+  const size_t rank_stride = static_cast<size_t>(rows) * num_splits * (2 * d + 4);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    plx::plx_decode_combine_kernel<128><<<static_cast<unsigned>(rows), 128, 0, st>>>(
+        partials, static_cast<__nv_bfloat16*>(out), lse, num_splits, ranks, rank_stride);
+  else
+    plx::plx_decode_combine_kernel<64><<<static_cast<unsigned>(rows), 64, 0, st>>>(
+        partials, static_cast<__nv_bfloat16*>(out), lse, num_splits, ranks, rank_stride);
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
 int plx_check_device_status(void* stream) {

@@ -60,6 +60,8 @@ struct DecodeParams {
   float* ws;                // [B, Hq, splits, 2D+4] or nullptr when splits == 1
                             //   per row: m (log2 units), l, c, pad, O1[D], O2[D]
   int B, Hq, Hkv, S_max, G, n_hgroups, splits, chunk;
+  int partial_out;          // 1: always write partial states to ws (context parallel), never out
+  int key_offset;           // global index of the cache's first key (context parallel; else 0)
   float scale_log2;         // scale * log2(e)
 };
 
@@ -89,7 +91,8 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  int seqlen = p.seqlens[b];
+  // live keys of this cache: the sequence's keys past key_offset, at most S_max
+  int seqlen = p.seqlens[b] - p.key_offset;
   seqlen = seqlen < 0 ? 0 : (seqlen > p.S_max ? p.S_max : seqlen);
   const int kbeg = split * p.chunk;
   const int kend = min(kbeg + p.chunk, seqlen);
@@ -101,7 +104,7 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     for (int idx = threadIdx.x; idx < nh * D; idx += kDecConsumerWarps * 32) {
       const int hh = idx / D, dd = idx % D;
       const size_t row = static_cast<size_t>(b) * p.Hq + h0 + hh;
-      if (p.splits == 1) {
+      if (p.splits == 1 && !p.partial_out) {
         p.out[row * D + dd] = __float2bfloat16(0.f);
         if (dd == 0 && p.lse) p.lse[row] = -INFINITY;
       } else {
@@ -330,7 +333,7 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
       O2 += beta * rw[4 + D + dd];
     }
     const size_t row = static_cast<size_t>(b) * p.Hq + h0 + hh;
-    if (p.splits == 1) {
+    if (p.splits == 1 && !p.partial_out) {
       float res = 0.f;
       if (L > 0.f) {
         const float inv = 1.f / L;
@@ -352,22 +355,29 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 template <int D>
 __global__ void __launch_bounds__(D)
 plx_decode_combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ out,
-                          float* __restrict__ lse, int splits) {
+                          float* __restrict__ lse, int splits, int ranks, size_t rank_stride) {
+  // partial states of row `row`: `ranks` blocks (rank_stride floats apart) of
+  // `splits` consecutive states each; one block = one shard of the keys
   constexpr int PF = DecodeCfg<D>::kPartialFloats;
   const size_t row = blockIdx.x;
-  const float* base = ws + row * splits * PF;
   const int dd = threadIdx.x;
   float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldg(base + s * PF));
+  for (int rk = 0; rk < ranks; ++rk) {
+    const float* base = ws + rk * rank_stride + row * splits * PF;
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldg(base + s * PF));
+  }
   const float Mu = M == -INFINITY ? 0.f : M;
   float L = 0.f, C = 0.f, O1 = 0.f, O2 = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float* ps = base + s * PF;
-    const float beta = ex2(__ldg(ps) - Mu);
-    L += beta * __ldg(ps + 1);
-    C += beta * __ldg(ps + 2);
-    O1 += beta * __ldg(ps + 4 + dd);
-    O2 += beta * __ldg(ps + 4 + D + dd);
+  for (int rk = 0; rk < ranks; ++rk) {
+    const float* base = ws + rk * rank_stride + row * splits * PF;
+    for (int s = 0; s < splits; ++s) {
+      const float* ps = base + s * PF;
+      const float beta = ex2(__ldg(ps) - Mu);
+      L += beta * __ldg(ps + 1);
+      C += beta * __ldg(ps + 2);
+      O1 += beta * __ldg(ps + 4 + dd);
+      O2 += beta * __ldg(ps + 4 + D + dd);
+    }
   }
   float res = 0.f;
   if (L > 0.f) {

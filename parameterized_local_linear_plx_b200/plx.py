@@ -53,6 +53,12 @@ _lib.plx_kv_append.restype = _I
 _lib.plx_kv_append.argtypes = [_P] * 5 + [_I] * 5 + [_P]
 _lib.plx_kv_append_paged.restype = _I
 _lib.plx_kv_append_paged.argtypes = [_P] * 6 + [_I] * 7 + [_P]
+_lib.plx_decode_partial_size.restype = _SZ
+_lib.plx_decode_partial_size.argtypes = [_I] * 6
+_lib.plx_decode_partial.restype = _I
+_lib.plx_decode_partial.argtypes = [_P] * 5 + [_I] * 6 + [_F, _I, _P, _SZ, _P]
+_lib.plx_decode_merge.restype = _I
+_lib.plx_decode_merge.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P]
 _lib.plx_decode_noalloc.restype = _I
 _lib.plx_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]
 _lib.plx_check_device_status.restype = _I
@@ -352,6 +358,55 @@ def plx_kv_append_paged(knew, vnew, kpool, vpool, block_table, seqlens, advance=
                                   _stream(stream))
     if st != PLX_OK:
         raise PlxError(st, "plx_kv_append_paged")
+
+
+def plx_decode_partial_size(B, Hq, Hkv, S_max, d, num_splits=0) -> int:
+    return int(_lib.plx_decode_partial_size(B, Hq, Hkv, S_max, d, num_splits))
+
+
+def plx_decode_partial(q, kcache, vcache, seqlens, r=None, key_offset=0, scale=None, num_splits=0, partial=None,
+                       stream=None):
+    """Partial states of a slice of the keys (keys key_offset .. key_offset + S_max - 1
+    of each sequence; seqlens are the full lengths): fp32 [B, Hq, splits, 2d + 4]
+    (m in log2 units, l, c, pad, O1[d], O2[d])."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(kcache, "kcache", torch.bfloat16, 4)
+    _check(vcache, "vcache", torch.bfloat16, 4)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    if r is not None:
+        _check(r, "r", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    Hkv, S_max = kcache.shape[1], kcache.shape[2]
+    if kcache.shape != (B, Hkv, S_max, d) or vcache.shape != kcache.shape or seqlens.shape != (B,):
+        raise ValueError("shape mismatch between q, caches, seqlens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    # the split count the kernel uses (a requested count is rounded to whole 64-key chunks)
+    splits = plx_decode_partial_size(B, Hq, Hkv, S_max, d, num_splits) // (B * Hq * (2 * d + 4) * 4)
+    if partial is None:
+        partial = torch.empty((B, Hq, splits, 2 * d + 4), device=q.device, dtype=torch.float32)
+    st = _lib.plx_decode_partial(_ptr(q), _ptr(r), _ptr(kcache), _ptr(vcache), _ptr(seqlens), int(key_offset), B, Hq,
+                                 Hkv, S_max, d,
+                                 float(scale), int(num_splits), _ptr(partial),
+                                 partial.numel() * partial.element_size(), _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_decode_partial")
+    return partial
+
+
+def plx_decode_merge(partials, out=None, lse=None, return_lse=True, stream=None):
+    """Merge gathered partials [ranks, B, Hq, splits, 2d + 4] into (out, lse)."""
+    _check(partials, "partials", torch.float32, 5)
+    ranks, B, Hq, splits, pf = partials.shape
+    d = (pf - 4) // 2
+    if out is None:
+        out = torch.empty((B, Hq, d), device=partials.device, dtype=torch.bfloat16)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), device=partials.device, dtype=torch.float32)
+    st = _lib.plx_decode_merge(_ptr(partials), ranks, B, Hq, d, splits, _ptr(out), _ptr(lse), _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_decode_merge")
+    return out, lse
 
 
 PLX_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024

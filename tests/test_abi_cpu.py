@@ -27,7 +27,7 @@ def declared_entry_points():
 
 def test_header_declares_the_boundary():
     names = declared_entry_points()
-    for n in ["plx_fwd", "plx_fwd_train", "plx_bwd", "plx_bwd_workspace_size", "plx_decode_paged", "plx_kv_append", "plx_kv_append_paged", "plx_fwd_varlen",
+    for n in ["plx_fwd", "plx_fwd_train", "plx_bwd", "plx_bwd_workspace_size", "plx_decode_paged", "plx_kv_append", "plx_kv_append_paged", "plx_fwd_varlen", "plx_decode_partial", "plx_decode_merge", "plx_decode_partial_size",
               "plx_decode", "plx_decode_workspace_size", "plx_decode_num_splits",
               "plx_check_device_status", "plx_status_string", "plx_version", "plx_selftest_wait_timeout"]:
         assert n in names
@@ -214,3 +214,21 @@ def test_varlen_argument_errors(plx):
     assert vf(*args(), 2, 2, 1, 100, 64, 48, 1, 0.125, None) == plx.PLX_ERR_HEADDIM
     assert vf(*args(), 2, 3, 2, 100, 64, 64, 1, 0.125, None) == plx.PLX_ERR_GQA
     assert vf(*args(cu=A + 2), 2, 2, 1, 100, 64, 64, 1, 0.125, None) == plx.PLX_ERR_ALIGN
+
+
+def test_partial_and_merge_argument_errors(plx):
+    dp = plx.lib.plx_decode_partial
+    ok = lambda **kw: [P(kw.get(n, A)) for n in ("q", "r", "kc", "vc", "sl")]
+    need = plx.plx_decode_partial_size(1, 2, 1, 64, 64, 1)
+    assert need == 1 * 2 * 1 * (2 * 64 + 4) * 4
+    assert dp(*ok(), 0, 1, 2, 1, 64, 64, 0.125, 1, P(None), need, None) == plx.PLX_ERR_NULL
+    assert dp(*ok(), -1, 1, 2, 1, 64, 64, 0.125, 1, P(A), need, None) == plx.PLX_ERR_SHAPE
+    assert dp(*ok(), 0, 1, 2, 1, 64, 64, 0.125, 1, P(A), need - 4, None) == plx.PLX_ERR_WORKSPACE
+    assert dp(*ok(kc=None), 0, 1, 2, 1, 64, 64, 0.125, 1, P(A), need, None) == plx.PLX_ERR_NULL
+    assert dp(*ok(), 0, 1, 2, 1, 64, 96, 0.125, 1, P(A), need, None) == plx.PLX_ERR_HEADDIM
+    mg = plx.lib.plx_decode_merge
+    assert mg(P(None), 2, 1, 2, 64, 1, P(A), P(A), None) == plx.PLX_ERR_NULL
+    assert mg(P(A), 0, 1, 2, 64, 1, P(A), P(A), None) == plx.PLX_ERR_SHAPE
+    assert mg(P(A), 2, 1, 2, 64, 0, P(A), P(A), None) == plx.PLX_ERR_SHAPE
+    assert mg(P(A), 2, 1, 2, 80, 1, P(A), P(A), None) == plx.PLX_ERR_HEADDIM
+    assert mg(P(A + 4), 2, 1, 2, 64, 1, P(A), P(A), None) == plx.PLX_ERR_ALIGN

@@ -1,0 +1,53 @@
+"""Host side of context-parallel decode, run as two gloo ranks on the CPU:
+slice planning and the exchange step (the all-gather of partial states in
+rank order).  The kernels themselves are covered by test_cp_decode_gpu.py."""
+import os
+import socket
+import sys
+
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        from parameterized_local_linear_plx_b200 import cp
+        B, Hq, splits, d = 3, 4, 2, 8
+        # a rank's partial block, filled with values that name the rank and the position
+        part = torch.arange(B * Hq * splits * (2 * d + 4), dtype=torch.float32).reshape(B, Hq, splits, 2 * d + 4)
+        part = part + 1000.0 * rank
+        g = cp.gather_partials(part)
+        q.put((rank, tuple(g.shape), [float(g[i, 0, 0, 0, 0]) for i in range(world)],
+               cp.slice_start(rank, 512)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_gather_rank_major():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = sorted(q.get(timeout=5) for _ in range(2))
+    assert res == [(0, (2, 3, 4, 2, 20), [0.0, 1000.0], 0), (1, (2, 3, 4, 2, 20), [0.0, 1000.0], 512)]
