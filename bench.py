@@ -427,6 +427,9 @@ def run_gpu(args, world, rank, local):
     # ---- the same decode step on a paged cache (block tables), timed on its own
     paged = run_paged(plx, args, dev, stream, world, local, d_bytes, hbm, peak_src)
 
+    # ---- context-parallel decode, ranks emulated as slices on this GPU (timed on its own)
+    cpd = run_cp(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes)
+
     # ---- packed variable-length prefill with the same token count (timed on its own)
     varlen = run_varlen(plx, args, dev, stream, world, local, tf_peak, peak_src, tf_key)
 
@@ -463,6 +466,7 @@ def run_gpu(args, world, rank, local):
             "e2e": e2e,
             "decode_paged": paged,
             "prefill_varlen": varlen,
+            "decode_cp_emulated": cpd,
             "backward": bwd,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
@@ -509,6 +513,48 @@ def run_paged(plx, args, dev, stream, world, local, d_bytes, hbm, peak_src):
                        f"pools [pages, Hkv, page_size, d], random page assignment")
     res["peak_source"] = f"{peak_src} hbm_gbs"
     return res
+
+
+def run_cp(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes, ranks=8):
+    """The per-rank costs of context-parallel decode for the decode workload
+    split over `ranks` ranks along the sequence, measured on this one GPU:
+    one rank's plx_decode_partial on its 4096/ranks-key slice, the merge of
+    all ranks' partials, and the bytes each rank sends in the all-gather."""
+    import torch
+    L = DEC["S"] // ranks
+    ks = kc[:, :, :L].contiguous()
+    vs = vc[:, :, :L].contiguous()
+    part = plx.plx_decode_partial(q, ks, vs, sl, r, key_offset=0, stream=stream)
+    gathered = torch.stack([part] * ranks)
+    out = torch.empty_like(q)
+    lse = torch.empty(DEC["B"], DEC["Hq"], dtype=torch.float32, device=dev)
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n * 1e3
+
+    n = max(1, min(args.steps, 50))
+    t_part = timed(lambda: plx.plx_decode_partial(q, ks, vs, sl, r, key_offset=0, partial=part, stream=stream), n)
+    t_merge = timed(lambda: plx.plx_decode_merge(gathered, out=out, lse=lse, stream=stream), n)
+    st = plx.plx_check_device_status(stream)
+    if st != plx.PLX_OK:
+        raise RuntimeError(f"device status after the context-parallel legs: {plx.plx_status_string(st)}")
+    slice_bytes = d_bytes // ranks
+    return {"workload": f"decode B={DEC['B']} ctx={DEC['S']} split over {ranks} ranks along the sequence "
+                        f"({L} keys per rank); ranks emulated on one GPU",
+            "ranks": ranks, "partial_us_per_rank": t_part, "merge_us": t_merge,
+            "slice_gbs": slice_bytes / (t_part * 1e-6) / 1e9,
+            "exchange_bytes_per_rank": part.numel() * 4,
+            "note": "per-rank step time = partial + all-gather of exchange_bytes_per_rank + merge; the "
+                    "all-gather is not measured (one GPU per run)"}
 
 
 VARLEN_LENS = [4096, 1, 2048, 777, 1024, 3000, 64, 65, 512, 1500, 4000, 129, 333, 2500, 100, 900,
