@@ -437,7 +437,7 @@ struct BwdKVCfg {
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQR = 2 * kTileBytes;
   static constexpr int kOffDO = kOffQR + kBwdStages * kTileBytes;
-  static constexpr int kOffStat = kOffDO + kBwdStages * kDOBytes;  // per warp: float4 per query of its 16
+  static constexpr int kOffStat = kOffDO + kBwdStages * kDOBytes;  // per warp: 64 floats (its 16 queries)
   static constexpr int kOffBar = kOffStat + kBwdElemWarps * 16 * 16;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
   // tensor memory: [A^T | S^T] [0,128), G^T [128,192), dK [256,256+D), dV [256+D, 256+2D).
@@ -602,23 +602,31 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     const int key = k0 + 32 * wq + lane;
     const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
     const bool key_ok = key < p.N;
-    float4* stat = reinterpret_cast<float4*>(smem + Cfg::kOffStat) + warp * 16;  // this warp's 16 queries
+    // this warp's 16 queries, pair-interleaved: for queries (2i, 2i+1) the
+    // float4s {L0, L1, F0, F1} and {G0, G1, D0, D1}, so that one load yields
+    // the packed pairs the f32x2 arithmetic takes
+    float* statf = reinterpret_cast<float*>(smem + Cfg::kOffStat) + warp * 64;
+    const float4* stat = reinterpret_cast<const float4*>(statf);
     for (int it = 0; it < n_items; ++it) {
       const int hq = g * p.G + it / n_qt;
       const int q0 = (qt0 + it % n_qt) * kBwdBM + 16 * wp;  // first of this warp's queries
       const size_t rb = (static_cast<size_t>(b) * p.Hq + hq) * p.N;
       __syncwarp();
       if (lane < 16) {
-        // per query: -lse log2(e), 1 + s_bar, g_bar, -Dd (rows past N: w = 0)
+        // per query: L = -lse log2(e), F = 1 + s_bar, G = g_bar, D = -Dd (rows past N: w = 0)
         const int q = q0 + lane;
-        float4 st4 = make_float4(-INFINITY, 1.f, 0.f, 0.f);
+        float L = -INFINITY, F = 1.f, G = 0.f, Dn = 0.f;
         if (q < p.N) {
-          st4.x = -p.lse[rb + q] * kLog2e;
-          st4.y = 1.f + (HAS_R ? p.sbar[rb + q] : 0.f);
-          st4.z = p.gbar[rb + q];
-          st4.w = -p.dd[rb + q];
+          L = -p.lse[rb + q] * kLog2e;
+          F = 1.f + (HAS_R ? p.sbar[rb + q] : 0.f);
+          G = p.gbar[rb + q];
+          Dn = -p.dd[rb + q];
         }
-        stat[lane] = st4;
+        float* sp = statf + (lane >> 1) * 8 + (lane & 1);
+        sp[0] = L;
+        sp[2] = F;
+        sp[4] = G;
+        sp[6] = Dn;
       }
       __syncwarp();
       const bool landed = mbar_wait_sleep(smem_u32(s_full), it & 1, kErrBwdElem);
@@ -642,11 +650,11 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       uint32_t pw[8], pa[8], pd[8];
 #pragma unroll
       for (int x = 0; x < 16; x += 2) {
-        const float4 s0 = stat[x], s1 = stat[x + 1];
+        const float4 sa = stat[x], sb = stat[x + 1];  // {L0, L1, F0, F1}, {G0, G1, D0, D1} of queries x, x+1
         const uint64_t A = f2(__uint_as_float(ra[x]), __uint_as_float(ra[x + 1]));
         const uint64_t S = f2(__uint_as_float(rs[x]), __uint_as_float(rs[x + 1]));
         const uint64_t Gv = f2(__uint_as_float(rg[x]), __uint_as_float(rg[x + 1]));
-        const uint64_t X = f2_fma(A, c_sl2, f2(s0.x, s1.x));
+        const uint64_t X = f2_fma(A, c_sl2, f2(sa.x, sa.y));
         float w0 = ex2(f2_lo(X)), w1 = ex2(f2_hi(X));
         if (need_mask) {
           const int q = q0 + x;
@@ -654,11 +662,11 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (!key_ok || (p.causal && key > q + 1)) w1 = 0.f;
         }
         const uint64_t W = f2(w0, w1);
-        const uint64_t Gb = f2(s0.z, s1.z);
-        const uint64_t F = f2_fma(S, c_m1, f2(s0.y, s1.y));                    // 1 + s_bar - s
+        const uint64_t Gb = f2(sb.x, sb.y);
+        const uint64_t F = f2_fma(S, c_m1, f2(sa.z, sa.w));                    // 1 + s_bar - s
         const uint64_t WH = f2_mul(W, F);
         const uint64_t DS = f2_mul(W, f2_fma(Gv, c_m1, Gb));                    // w (g_bar - g)
-        const uint64_t U = f2_fma(Gv, F, f2_fma(S, Gb, f2(s0.w, s1.w)));       // g f + s g_bar - Dd
+        const uint64_t U = f2_fma(Gv, F, f2_fma(S, Gb, f2(sb.z, sb.w)));       // g f + s g_bar - Dd
         const uint64_t DA = f2_mul(f2_mul(W, c_sc), U);
         pw[x >> 1] = pack_bf16(f2_lo(WH), f2_hi(WH));
         pa[x >> 1] = pack_bf16(f2_lo(DA), f2_hi(DA));
