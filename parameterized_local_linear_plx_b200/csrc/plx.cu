@@ -150,8 +150,22 @@ int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const plx::Decod
   kern<<<grid, plx::kDecThreads, Cfg::kSmemBytes, st>>>(km, vm, p);
   if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
   if (p.splits > 1 && !p.partial_out) {
-    plx::plx_decode_combine_kernel<D><<<p.B * p.Hq, D, 0, st>>>(p.ws, p.out, p.lse, p.splits, 1, 0);
-    if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+    // programmatic dependent launch: the combine is scheduled as the split
+    // CTAs finish, and griddepcontrol.wait inside it orders it after them
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.B * p.Hq));
+    cfg.blockDim = dim3(D);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float* ws = p.ws;
+    if (cudaLaunchKernelEx(&cfg, plx::plx_decode_combine_kernel<D>, ws, p.out, p.lse, p.splits, 1,
+                           static_cast<size_t>(0)) != cudaSuccess)
+      return PLX_ERR_CUDA;
   }
   return PLX_OK;
 }

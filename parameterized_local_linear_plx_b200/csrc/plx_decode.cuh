@@ -349,6 +349,9 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
       ws[4 + D + dd] = O2;
     }
   }
+  // this CTA's results are written: the combine (launched as a programmatic
+  // dependent) may be scheduled; it still waits for this grid to complete
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Merge the per-split partial states of one (b, h) row: one CTA of D threads.
@@ -361,6 +364,9 @@ plx_decode_combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restric
   constexpr int PF = DecodeCfg<D>::kPartialFloats;
   const size_t row = blockIdx.x;
   const int dd = threadIdx.x;
+  // launched as a programmatic dependent of the split kernel: wait until that
+  // grid has completed and its writes are visible (a no-op otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   float M = -INFINITY;
   for (int rk = 0; rk < ranks; ++rk) {
     const float* base = ws + rk * rank_stride + row * splits * PF;
