@@ -32,7 +32,10 @@
 //     element-wise warps write W_hat^T, scale dA^T and dS^T in bf16; then
 //     dV += W_hat^T dO and dK += [scale dA^T | dS^T] [Q;R] (the stacked tile is
 //     the K-major B of the first product and the MN-major B of the last).
-//     Each CTA owns its output rows: no atomics anywhere.
+//     G^T has two buffers in tensor memory, so the next tile's G^T and this
+//     tile's dV products run during the element-wise pass; only dK and the
+//     next scores stand between two passes.  Each CTA owns its output rows:
+//     no atomics anywhere.
 //   * In both: warps 0-15 element-wise.  Warp w reads TMEM lanes
 //     32(w%4)..32(w%4)+31 and one quarter (w/4) of the columns; every
 //     (key, query) element is independent, so the warps share nothing, and
@@ -58,7 +61,7 @@ constexpr int kBwdElemWarps = 16;
 constexpr int kBwdThreads = 32 * (kBwdElemWarps + 2);  // element-wise warps, TMA warp, MMA warp
 constexpr int kBwdTmaWarp = kBwdElemWarps;
 constexpr int kBwdMmaWarp = kBwdElemWarps + 1;
-constexpr int kBwdStages = 2;
+constexpr int kBwdStages = 3;
 
 struct BwdParams {
   __nv_bfloat16* dq;  // [B, Hq, N, D]
@@ -440,8 +443,9 @@ struct BwdKVCfg {
   static constexpr int kOffStat = kOffDO + kBwdStages * kDOBytes;  // per warp: 64 floats (its 16 queries)
   static constexpr int kOffBar = kOffStat + kBwdElemWarps * 16 * 16;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
-  // tensor memory: [A^T | S^T] [0,128), G^T [128,192), dK [256,256+D), dV [256+D, 256+2D).
-  // bf16 results: scale dA^T and dS^T over the score columns, W_hat^T over G^T.
+  // tensor memory: [A^T | S^T] [0,128), G^T of item i at 128 + 64 (i & 1) (two
+  // buffers), dK [256,256+D), dV [256+D, 256+2D).  bf16 results: scale dA^T and
+  // dS^T over the score columns, W_hat^T over its G^T.
   static constexpr uint32_t kColS = 0, kColG = 128, kColDK = 256, kColDV = 256 + D;
   static constexpr uint32_t kTmemCols = 512;
 };
@@ -557,38 +561,64 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       const uint64_t d_do = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffDO), 16, 1024);
       const uint64_t d_qr_mn = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffQR), Cfg::kBlock, 1024);
       const uint64_t d_do_mn = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffDO), Cfg::kDOBlock, 1024);
-      ok = mbar_wait(smem_u32(kv_full), 0, kErrBwdMma);
-      for (int it = 0; it < n_items && ok; ++it) {
-        const int s = it % NS;
-        if (!mbar_wait(smem_u32(&q_full[s]), (it / NS) & 1, kErrBwdMma)) { ok = false; break; }
-        tc::fence_after_sync();
-        const uint64_t qr_off = static_cast<uint64_t>(s) * (Cfg::kTileBytes >> 4);
-        const uint64_t do_off = static_cast<uint64_t>(s) * (Cfg::kDOBytes >> 4);
+      // Per item i, in issue order (the tensor pipe runs them in that order):
+      // G^T(i+1) into the other G^T buffer, then after the element-wise pass
+      // of i: dK(i) (the last reader of the score columns), [A^T|S^T](i+1),
+      // dV(i).  The element-wise pass of i+1 waits only for dK(i) and the
+      // scores of i+1; dV(i) and G^T(i+2) run during it.
+      auto issue_s = [&](int it) {
+        const uint64_t qr_off = static_cast<uint64_t>(it % NS) * (Cfg::kTileBytes >> 4);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t koff = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
           tc::mma_ss(tmem + Cfg::kColS, d_k + koff, d_qr + qr_off + koff, idesc_s, ks > 0 ? 1u : 0u);
         }
+      };
+      auto issue_g = [&](int it) {
+        const uint64_t do_off = static_cast<uint64_t>(it % NS) * (Cfg::kDOBytes >> 4);
+        const uint32_t gcol = Cfg::kColG + 64 * static_cast<uint32_t>(it & 1);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t koff_a = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
           const uint64_t koff_b = static_cast<uint64_t>(((ks >> 2) * Cfg::kDOBlock + (ks & 3) * 32) >> 4);
-          tc::mma_ss(tmem + Cfg::kColG, d_v + koff_a, d_do + do_off + koff_b, idesc_g, ks > 0 ? 1u : 0u);
+          tc::mma_ss(tmem + gcol, d_v + koff_a, d_do + do_off + koff_b, idesc_g, ks > 0 ? 1u : 0u);
         }
+      };
+      ok = mbar_wait(smem_u32(kv_full), 0, kErrBwdMma) && (n_items == 0 || mbar_wait(smem_u32(&q_full[0]), 0, kErrBwdMma));
+      if (ok && n_items > 0) {
+        tc::fence_after_sync();
+        issue_s(0);
+        issue_g(0);
         tc::commit(smem_u32(s_full));
+      }
+      for (int it = 0; it < n_items && ok; ++it) {
+        const int s = it % NS;
+        const bool more = it + 1 < n_items;
+        if (more) {
+          if (!mbar_wait(smem_u32(&q_full[(it + 1) % NS]), ((it + 1) / NS) & 1, kErrBwdMma)) { ok = false; break; }
+          tc::fence_after_sync();
+          issue_g(it + 1);
+        }
         if (!mbar_wait(smem_u32(p_ready), it & 1, kErrBwdMma)) { ok = false; break; }
         tc::fence_after_sync();
-        // dV += W_hat^T dO (K = 64 queries; the pairs of queries 16kk.. sit at G^T column 16kk)
-#pragma unroll
-        for (int kk = 0; kk < kBwdBM / 16; ++kk)
-          tc::mma_ts(tmem + Cfg::kColDV, tmem + Cfg::kColG + 16 * kk,
-                     d_do_mn + do_off + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
+        const uint64_t qr_off = static_cast<uint64_t>(s) * (Cfg::kTileBytes >> 4);
+        const uint64_t do_off = static_cast<uint64_t>(s) * (Cfg::kDOBytes >> 4);
         // dK += [scale dA^T | dS^T] [Q ; R] (K = 128 stacked rows; the pairs of
         // stacked rows 32c..32c+15 sit at column 32c, of rows 32c+16.. at 32c+8)
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
           tc::mma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColS + 32 * (kk >> 1) + 8 * (kk & 1),
                      d_qr_mn + qr_off + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
+        if (more) {
+          issue_s(it + 1);
+          tc::commit(smem_u32(s_full));  // scores of i+1, and G^T(i+1) issued before
+        }
+        // dV += W_hat^T dO (K = 64 queries; the pairs of queries 16kk.. sit at G^T column 16kk)
+        const uint32_t gcol = Cfg::kColG + 64 * static_cast<uint32_t>(it & 1);
+#pragma unroll
+        for (int kk = 0; kk < kBwdBM / 16; ++kk)
+          tc::mma_ts(tmem + Cfg::kColDV, tmem + gcol + 16 * kk,
+                     d_do_mn + do_off + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
         tc::commit(smem_u32(&q_empty[s]));
       }
       tc::commit(smem_u32(o_done));
@@ -637,7 +667,7 @@ plx_bwd_kv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       const bool need_mask = (k0 + 32 * wq + 31 >= p.N) || (p.causal && k0 + 32 * wq + 31 > q0);
       // stacked columns 32wp..32wp+15 (q.k) and 32wp+16..32wp+31 (rho.k), G^T columns 16wp..16wp+15
       const uint32_t tsa = tmem + lane_base + Cfg::kColS + 32 * wp;
-      const uint32_t tgw = tmem + lane_base + Cfg::kColG + 16 * wp;
+      const uint32_t tgw = tmem + lane_base + Cfg::kColG + 64 * static_cast<uint32_t>(it & 1) + 16 * wp;
       uint32_t ra[16], rs[16], rg[16];
       tc::ld_32x32b_x16(tsa, ra);
       tc::ld_32x32b_x16(tsa + 16, rs);
