@@ -186,7 +186,7 @@ int launch_fwd(const CUtensorMap& qm, const CUtensorMap& rm, const CUtensorMap& 
 
 template <int D, bool HAS_R>
 int launch_bwd(const CUtensorMap& qm, const CUtensorMap& rm, const CUtensorMap& om, const CUtensorMap& km,
-               const CUtensorMap& vm, const CUtensorMap& km64, const CUtensorMap& vm64, const plx::BwdParams& p, const void* dout, const void* out,
+               const CUtensorMap& vm, const CUtensorMap& kmq, const CUtensorMap& vmq, const plx::BwdParams& p, const void* dout, const void* out,
                const void* obar, float* gbar, float* dd, cudaStream_t st) {
   using QCfg = plx::BwdQCfg<D>;
   using KVCfg = plx::BwdKVCfg<D>;
@@ -200,7 +200,7 @@ int launch_bwd(const CUtensorMap& qm, const CUtensorMap& rm, const CUtensorMap& 
   if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
   auto kq = plx::plx_bwd_q_kernel<D, HAS_R>;
   if (ensure_smem(kq, QCfg::kSmemBytes, &done_q[dev]) != PLX_OK) return PLX_ERR_CUDA;
-  kq<<<static_cast<unsigned>(p.B * p.Hq * p.n_qtiles), plx::kBwdThreads, QCfg::kSmemBytes, st>>>(qm, rm, om, km64, vm64, p);
+  kq<<<static_cast<unsigned>(p.B * p.Hq * p.n_qtiles), plx::kBwdThreads, QCfg::kSmemBytes, st>>>(qm, rm, om, kmq, vmq, p);
   if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
   auto kkv = plx::plx_bwd_kv_kernel<D, HAS_R>;
   if (ensure_smem(kkv, KVCfg::kSmemBytes, &done_kv[dev]) != PLX_OK) return PLX_ERR_CUDA;
@@ -489,11 +489,11 @@ int plx_bwd(const void* q, const void* k, const void* v, const void* r, const vo
   int rc = check_arch(&dev);
   if (rc != PLX_OK) return rc;
   if ((rc = get_encoder()) != PLX_OK) return rc;
-  CUtensorMap qm, rm, om, km, vm, km64, vm64;
+  CUtensorMap qm, rm, om, km, vm, kmq, vmq;
   const long long pq = static_cast<long long>(B) * Hq, pkv = static_cast<long long>(B) * Hkv;
   if (make_map_3d(&qm, q, d, N, pq, 16) != PLX_OK || make_map_3d(&om, dout, d, N, pq, 16) != PLX_OK ||
       make_map_3d(&km, k, d, N, pkv, plx::kBwdBN) != PLX_OK || make_map_3d(&vm, v, d, N, pkv, plx::kBwdBN) != PLX_OK ||
-      make_map_3d(&km64, k, d, N, pkv, plx::kBwdQBN) != PLX_OK || make_map_3d(&vm64, v, d, N, pkv, plx::kBwdQBN) != PLX_OK)
+      make_map_3d(&kmq, k, d, N, pkv, plx::kBwdQBN) != PLX_OK || make_map_3d(&vmq, v, d, N, pkv, plx::kBwdQBN) != PLX_OK)
     return PLX_ERR_CUDA;
   if (r) {
     if (make_map_3d(&rm, r, d, N, pq, 16) != PLX_OK) return PLX_ERR_CUDA;
@@ -516,10 +516,10 @@ int plx_bwd(const void* q, const void* k, const void* v, const void* r, const vo
   p.scale_log2 = scale * plx::kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 128)
-    return r ? launch_bwd<128, true>(qm, rm, om, km, vm, km64, vm64, p, dout, out, obar, gbar, dd, st)
-             : launch_bwd<128, false>(qm, rm, om, km, vm, km64, vm64, p, dout, out, obar, gbar, dd, st);
-  return r ? launch_bwd<64, true>(qm, rm, om, km, vm, km64, vm64, p, dout, out, obar, gbar, dd, st)
-           : launch_bwd<64, false>(qm, rm, om, km, vm, km64, vm64, p, dout, out, obar, gbar, dd, st);
+    return r ? launch_bwd<128, true>(qm, rm, om, km, vm, kmq, vmq, p, dout, out, obar, gbar, dd, st)
+             : launch_bwd<128, false>(qm, rm, om, km, vm, kmq, vmq, p, dout, out, obar, gbar, dd, st);
+  return r ? launch_bwd<64, true>(qm, rm, om, km, vm, kmq, vmq, p, dout, out, obar, gbar, dd, st)
+           : launch_bwd<64, false>(qm, rm, om, km, vm, kmq, vmq, p, dout, out, obar, gbar, dd, st);
 }
 
 int plx_decode_num_splits(int B, int Hq, int Hkv, int S_max, int d) {

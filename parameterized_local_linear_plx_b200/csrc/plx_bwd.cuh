@@ -21,11 +21,12 @@
 //   * plx_bwd_pre_kernel: one warp per query row: g_bar and Dd.
 //   * plx_bwd_q_kernel (dQ, dR): one CTA per 64-query tile, with the stacked
 //     [Q;R] operand of the forward (rows 32w..32w+15: queries 16w..16w+15; rows
-//     32w+16..32w+31: their probes).  Per 64-key tile: S = [Q;R] K^T and
+//     32w+16..32w+31: their probes).  Per 128-key tile: S = [Q;R] K^T and
 //     G = [dO;0] V^T (dO in the query slots of a second stacked operand and
 //     zeros in the probe slots, so g lands in the query lanes beside a), then
 //     the element-wise warps write [scale dA ; dS] in bf16 over S and one MMA
-//     [scale dA ; dS] K accumulates [dQ ; dR] in tensor memory.
+//     [scale dA ; dS] K accumulates [dQ ; dR] in tensor memory.  G has two
+//     buffers, so the next tile's G runs during the element-wise pass.
 //   * plx_bwd_kv_kernel (dK, dV): one CTA per 128-key tile, keys as the MMA
 //     rows.  For each 64-query tile of each query head of the KV group:
 //     [A^T | S^T] = K [Q;R]^T and G^T = V dO^T; per (key, query) the
@@ -116,27 +117,31 @@ __global__ void __launch_bounds__(256) plx_bwd_pre_kernel(const __nv_bfloat16* _
 }
 
 // ---------------------------------------------------------------- dQ, dR
-// Keys come in tiles of 64 with the score and G accumulators double-buffered
-// in tensor memory, so the MMAs of tile j+1 (and the [dQ ; dR] product of
-// tile j-1) run while the element-wise warps work on tile j.
-constexpr int kBwdQBN = 64;      // keys per tile of the query-side kernel
-constexpr int kBwdQStages = 3;   // K/V ring
+// Keys come in tiles of 128 (N = 128 score MMAs: half the instructions per key
+// of 64-key tiles).  Tensor memory holds one score buffer, two G buffers and
+// [dQ ; dR]: G of tile j+1 runs during the element-wise pass of tile j, and
+// only [dQ ; dR] of tile j and the scores of tile j+1 stand between two
+// passes.  K and V have rings of their own: V is free once G has read it, K
+// only after the [dQ ; dR] product.
+constexpr int kBwdQBN = 128;     // keys per tile of the query-side kernel
+constexpr int kBwdQKStages = 3;  // K ring
+constexpr int kBwdQVStages = 2;  // V ring
 
 template <int D>
 struct BwdQCfg {
   static constexpr int kCB = D / 64;              // 128-byte column blocks per row
   static constexpr int kBlock = 128 * 128;        // one [128 rows x 128 B] block
-  static constexpr int kKVBlock = kBwdQBN * 128;   // one [64 rows x 128 B] block
+  static constexpr int kKVBlock = kBwdQBN * 128;  // one [128 keys x 128 B] block
   static constexpr int kTileBytes = kCB * kBlock;  // a 128-row stacked tile
-  static constexpr int kKVBytes = kCB * kKVBlock;  // a 64-key K or V tile
+  static constexpr int kKVBytes = kCB * kKVBlock;  // a 128-key K or V tile
   static constexpr int kOffQR = 0;
   static constexpr int kOffDO = kTileBytes;        // [dO ; 0] stacked like [Q ; R]
   static constexpr int kOffK = 2 * kTileBytes;
-  static constexpr int kOffV = kOffK + kBwdQStages * kKVBytes;
-  static constexpr int kOffBar = kOffV + kBwdQStages * kKVBytes;
-  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
-  // tensor memory: buffer b in {0,1}: S at 128b, G at 128b + 64; [dQ ; dR] at 256
-  static constexpr uint32_t kColAcc = 256, kTmemCols = 512;
+  static constexpr int kOffV = kOffK + kBwdQKStages * kKVBytes;
+  static constexpr int kOffBar = kOffV + kBwdQVStages * kKVBytes;
+  static constexpr int kSmemBytes = kOffBar + 128 + 1024;
+  // tensor memory: S [0,128), G of tile j at 128 + 128 (j & 1), [dQ ; dR] at 384
+  static constexpr uint32_t kColS = 0, kColG = 128, kColAcc = 384, kTmemCols = 512;
 };
 
 template <int D, bool HAS_R>
@@ -145,19 +150,18 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
                  const __grid_constant__ CUtensorMap omap, const __grid_constant__ CUtensorMap kmap,
                  const __grid_constant__ CUtensorMap vmap, const BwdParams p) {
   using Cfg = BwdQCfg<D>;
-  constexpr int NS = kBwdQStages;
+  constexpr int NK = kBwdQKStages, NV = kBwdQVStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
   uint64_t* q_full = bars;              // [1] [Q;R] and [dO;0] landed
-  uint64_t* kv_full = bars + 1;         // [NS]
-  uint64_t* kv_empty = kv_full + NS;    // [NS]
-  uint64_t* s_full = kv_empty + NS;     // [2] S and G of a key tile are in TMEM buffer b
-  // [2] [dA ; dS] of a key tile written to buffer b (one arrival per element-wise warp).  One
-  // barrier per buffer: a phase can then complete only after the MMA thread has
-  // waited for the previous one (the tile two ahead needs a buffer it frees).
-  uint64_t* p_ready = s_full + 2;
-  uint64_t* o_done = p_ready + 2;       // [1] every MMA complete
+  uint64_t* k_full = bars + 1;          // [NK]
+  uint64_t* k_empty = k_full + NK;      // [NK]
+  uint64_t* v_full = k_empty + NK;      // [NV]
+  uint64_t* v_empty = v_full + NV;      // [NV]
+  uint64_t* s_full = v_empty + NV;      // [1] S of a key tile (and its G, issued before) in TMEM
+  uint64_t* p_ready = s_full + 1;       // [1] [dA ; dS] written (one arrival per element-wise warp)
+  uint64_t* o_done = p_ready + 1;       // [1] every MMA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -174,14 +178,16 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(smem_u32(&kv_full[s]), 1);
-      mbar_init(smem_u32(&kv_empty[s]), 1);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(smem_u32(&k_full[s]), 1);
+      mbar_init(smem_u32(&k_empty[s]), 1);
     }
-    mbar_init(smem_u32(&s_full[0]), 1);
-    mbar_init(smem_u32(&s_full[1]), 1);
-    mbar_init(smem_u32(&p_ready[0]), kBwdElemWarps);  // one arrival per element-wise warp
-    mbar_init(smem_u32(&p_ready[1]), kBwdElemWarps);
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(smem_u32(&v_full[s]), 1);
+      mbar_init(smem_u32(&v_empty[s]), 1);
+    }
+    mbar_init(smem_u32(s_full), 1);
+    mbar_init(smem_u32(p_ready), kBwdElemWarps);  // one arrival per element-wise warp
     mbar_init(smem_u32(o_done), 1);
     fence_barrier_init();
   }
@@ -225,24 +231,34 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
             tma_load_3d(&omap, smem_u32(smem + Cfg::kOffDO + off), fb, cb * 64, q0 + 16 * wq, plane);
           }
       }
-      int issued = 0;
+      int issued_k = 0, issued_v = 0;
       for (int j = 0; j < nkv; ++j) {
-        const int s = j % NS;
-        if (j >= NS && !mbar_wait_sleep(smem_u32(&kv_empty[s]), ((j / NS) - 1) & 1, kErrBwdLoad)) { ok = false; break; }
-        const uint32_t fb = smem_u32(&kv_full[s]);
-        mbar_arrive_expect_tx(fb, 2 * Cfg::kKVBytes);
+        const int sk = j % NK, sv = j % NV;
+        if (j >= NK && !mbar_wait_sleep(smem_u32(&k_empty[sk]), ((j / NK) - 1) & 1, kErrBwdLoad)) { ok = false; break; }
+        {
+          const uint32_t fb = smem_u32(&k_full[sk]);
+          mbar_arrive_expect_tx(fb, Cfg::kKVBytes);
 #pragma unroll
-        for (int cb = 0; cb < Cfg::kCB; ++cb) {
-          tma_load_3d(&kmap, smem_u32(smem + Cfg::kOffK + s * Cfg::kKVBytes + cb * Cfg::kKVBlock), fb, cb * 64,
-                      j * kBwdQBN, plane_kv);
-          tma_load_3d(&vmap, smem_u32(smem + Cfg::kOffV + s * Cfg::kKVBytes + cb * Cfg::kKVBlock), fb, cb * 64,
-                      j * kBwdQBN, plane_kv);
+          for (int cb = 0; cb < Cfg::kCB; ++cb)
+            tma_load_3d(&kmap, smem_u32(smem + Cfg::kOffK + sk * Cfg::kKVBytes + cb * Cfg::kKVBlock), fb, cb * 64,
+                        j * kBwdQBN, plane_kv);
+          issued_k = j + 1;
         }
-        issued = j + 1;
+        if (j >= NV && !mbar_wait_sleep(smem_u32(&v_empty[sv]), ((j / NV) - 1) & 1, kErrBwdLoad)) { ok = false; break; }
+        {
+          const uint32_t fb = smem_u32(&v_full[sv]);
+          mbar_arrive_expect_tx(fb, Cfg::kKVBytes);
+#pragma unroll
+          for (int cb = 0; cb < Cfg::kCB; ++cb)
+            tma_load_3d(&vmap, smem_u32(smem + Cfg::kOffV + sv * Cfg::kKVBytes + cb * Cfg::kKVBlock), fb, cb * 64,
+                        j * kBwdQBN, plane_kv);
+          issued_v = j + 1;
+        }
       }
       if (!ok) {  // let every issued load land before the CTA can exit
         mbar_wait(smem_u32(q_full), 0, kErrBwdDrain);
-        for (int j = max(0, issued - NS); j < issued; ++j) mbar_wait(smem_u32(&kv_full[j % NS]), (j / NS) & 1, kErrBwdDrain);
+        for (int j = max(0, issued_k - NK); j < issued_k; ++j) mbar_wait(smem_u32(&k_full[j % NK]), (j / NK) & 1, kErrBwdDrain);
+        for (int j = max(0, issued_v - NV); j < issued_v; ++j) mbar_wait(smem_u32(&v_full[j % NV]), (j / NV) & 1, kErrBwdDrain);
       }
     }
   } else if (warp == kBwdMmaWarp) {
@@ -256,55 +272,67 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       const uint64_t d_k = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffK), 16, 1024);
       const uint64_t d_v = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffV), 16, 1024);
       const uint64_t d_kmn = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffK), Cfg::kKVBlock, 1024);
-      // S and G of key tile j into buffer j&1
-      auto issue_sg = [&](int j) -> bool {
-        const int s = j % NS;
-        if (!mbar_wait(smem_u32(&kv_full[s]), (j / NS) & 1, kErrBwdMma)) return false;
+      // Per key tile j, in issue order (the tensor pipe runs them in that
+      // order): G(j+1) into the other G buffer; after the element-wise pass of
+      // j, [dQ ; dR] += [scale dA ; dS] K (the last reader of the score
+      // columns); then the scores of j+1.
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % NK;
+        if (!mbar_wait(smem_u32(&k_full[s]), (j / NK) & 1, kErrBwdMma)) return false;
         tc::fence_after_sync();
-        const uint32_t cs = tmem + 128 * (j & 1);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t koff_a = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
           const uint64_t koff_b = static_cast<uint64_t>(((ks >> 2) * Cfg::kKVBlock + (ks & 3) * 32) >> 4);
-          tc::mma_ss(cs, d_qr + koff_a, d_k + s * kStageStep + koff_b, idesc_s, ks > 0 ? 1u : 0u);
+          tc::mma_ss(tmem + Cfg::kColS, d_qr + koff_a, d_k + s * kStageStep + koff_b, idesc_s, ks > 0 ? 1u : 0u);
         }
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t koff_a = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
-          const uint64_t koff_b = static_cast<uint64_t>(((ks >> 2) * Cfg::kKVBlock + (ks & 3) * 32) >> 4);
-          tc::mma_ss(cs + kBwdQBN, d_do + koff_a, d_v + s * kStageStep + koff_b, idesc_s, ks > 0 ? 1u : 0u);
-        }
-        tc::commit(smem_u32(&s_full[j & 1]));
         return true;
       };
-      // [dQ ; dR] += [scale dA ; dS] K of key tile j: A = the bf16 pairs that
-      // warp part c wrote at columns 16c..16c+7 of buffer j&1 (keys 16c..16c+15)
-      auto issue_dqr = [&](int j) -> bool {
-        if (!mbar_wait(smem_u32(&p_ready[j & 1]), (j >> 1) & 1, kErrBwdMma)) return false;
+      auto issue_g = [&](int j) -> bool {
+        const int s = j % NV;
+        if (!mbar_wait(smem_u32(&v_full[s]), (j / NV) & 1, kErrBwdMma)) return false;
         tc::fence_after_sync();
-        const int s = j % NS;
-        const uint32_t cs = tmem + 128 * (j & 1);
+        const uint32_t cg = tmem + Cfg::kColG + 128 * static_cast<uint32_t>(j & 1);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t koff_a = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
+          const uint64_t koff_b = static_cast<uint64_t>(((ks >> 2) * Cfg::kKVBlock + (ks & 3) * 32) >> 4);
+          tc::mma_ss(cg, d_do + koff_a, d_v + s * kStageStep + koff_b, idesc_s, ks > 0 ? 1u : 0u);
+        }
+        tc::commit(smem_u32(&v_empty[s]));  // G is V's only reader
+        return true;
+      };
+      ok = mbar_wait(smem_u32(q_full), 0, kErrBwdMma);
+      if (ok && nkv > 0) {
+        ok = issue_g(0) && issue_s(0);
+        if (ok) tc::commit(smem_u32(s_full));
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const bool more = j + 1 < nkv;
+        // G(j+1) goes to the buffer of tile j-1, whose element-wise pass is over (p_ready waited)
+        if (more && !issue_g(j + 1)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(p_ready), j & 1, kErrBwdMma)) { ok = false; break; }
+        tc::fence_after_sync();
+        // A = the bf16 pairs of keys 16kk..16kk+15: warp part c wrote keys
+        // 32c..32c+31 as pairs at columns 32c..32c+15
+        const int sk = j % NK;
 #pragma unroll
         for (int kk = 0; kk < kBwdQBN / 16; ++kk)
-          tc::mma_ts(tmem + Cfg::kColAcc, cs + 16 * kk,
-                     d_kmn + s * kStageStep + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
+          tc::mma_ts(tmem + Cfg::kColAcc, tmem + Cfg::kColS + 32 * (kk >> 1) + 8 * (kk & 1),
+                     d_kmn + sk * kStageStep + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
                      (j > 0 || kk > 0) ? 1u : 0u);
-        tc::commit(smem_u32(&kv_empty[s]));
-        return true;
-      };
-      ok = mbar_wait(smem_u32(q_full), 0, kErrBwdMma) && (nkv == 0 || issue_sg(0));
-      for (int j = 0; j < nkv && ok; ++j) {
-        // S and G of tile j+1 go to the buffer of tile j-1: its element-wise
-        // pass is over (p_ready waited) and its [dQ ; dR] MMAs precede these
-        if (j + 1 < nkv && !issue_sg(j + 1)) { ok = false; break; }
-        if (!issue_dqr(j)) { ok = false; break; }
+        tc::commit(smem_u32(&k_empty[sk]));
+        if (more) {
+          if (!issue_s(j + 1)) { ok = false; break; }
+          tc::commit(smem_u32(s_full));  // scores of j+1, and G(j+1) issued before
+        }
       }
       tc::commit(smem_u32(o_done));  // also on abort: every issued MMA completes before dealloc
       mbar_wait(smem_u32(o_done), 0, kErrBwdMma);
     }
   } else {
     // ================================================================ element-wise + epilogue
-    // warp (wq, part): rows of TMEM quadrant wq, keys 16part..16part+15 of each tile
+    // warp (wq, part): rows of TMEM quadrant wq, keys 32part..32part+31 of each tile
     const int wq = warp & 3, part = warp >> 2;
     const int c4 = lane & 3;
     const int r_lo = lane >> 2;
@@ -335,26 +363,27 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     const uint64_t nd_lo = f2(-dd_lo, -dd_lo), nd_hi = f2(-dd_hi, -dd_hi);
     const uint64_t c_sl2 = f2(p.scale_log2, p.scale_log2), c_m1 = f2(-1.f, -1.f), c_sc = f2(p.scale, p.scale);
     for (int j = 0; j < nkv; ++j) {
-      const bool landed = mbar_wait_sleep(smem_u32(&s_full[j & 1]), (j >> 1) & 1, kErrBwdElem);
+      const bool landed = mbar_wait_sleep(smem_u32(s_full), j & 1, kErrBwdElem);
       if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
       tc::fence_after_sync();
-      const uint32_t cs = 128 * (j & 1) + 16 * part;
-      const uint32_t ta = tmem + lane_a + cs, ts = tmem + lane_s + cs, tg = tmem + lane_a + cs + kBwdQBN;
-      uint32_t ra[8], rs[8], rg[8];
-      tc::ld_16x256b_x2(ta, ra);
-      tc::ld_16x256b_x2(ts, rs);
-      tc::ld_16x256b_x2(tg, rg);
+      const uint32_t cs = Cfg::kColS + 32 * part;
+      const uint32_t ta = tmem + lane_a + cs, ts = tmem + lane_s + cs;
+      const uint32_t tg = tmem + lane_a + Cfg::kColG + 128 * static_cast<uint32_t>(j & 1) + 32 * part;
+      uint32_t ra[16], rs[16], rg[16];
+      tc::ld_16x256b_x4(ta, ra);
+      tc::ld_16x256b_x4(ts, rs);
+      tc::ld_16x256b_x4(tg, rg);
       tc::wait_ld();
       // masks only where some (query, key) of this warp is out of the set:
       // keys past N, or (causal) a key of the warp after its first row
-      const int kw = j * kBwdQBN + 16 * part;  // this warp's first key
-      const bool need_mask = (kw + 15 >= p.N) || (p.causal && kw + 15 > q0 + 16 * wq);
-      // register i: rep gg = i/4, e = i%4; key = 64j + 16part + 8gg + 2c4 + (e&1);
+      const int kw = j * kBwdQBN + 32 * part;  // this warp's first key
+      const bool need_mask = (kw + 31 >= p.N) || (p.causal && kw + 31 > q0 + 16 * wq);
+      // register i: rep gg = i/4, e = i%4; key = 128j + 32part + 8gg + 2c4 + (e&1);
       // row lo for e < 2, row hi for e >= 2.  Registers (4gg, 4gg+1) and
       // (4gg+2, 4gg+3) are key pairs of one row: packed f32x2 arithmetic.
-      uint32_t pa[4], pd[4];
+      uint32_t pa[8], pd[8];
 #pragma unroll
-      for (int h2 = 0; h2 < 4; ++h2) {
+      for (int h2 = 0; h2 < 8; ++h2) {
         const int i = 2 * h2;
         const bool hi = (h2 & 1) != 0;
         const uint64_t A = f2(__uint_as_float(ra[i]), __uint_as_float(ra[i + 1]));
@@ -377,13 +406,13 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         pa[h2] = pack_bf16(f2_lo(DA), f2_hi(DA));
         pd[h2] = pack_bf16(f2_lo(DS), f2_hi(DS));
       }
-      // bf16 pairs over the first 8 of this warp's own 16 fp32 columns
-      tc::st_16x128b_x2(ta, pa);
-      tc::st_16x128b_x2(ts, pd);
+      // bf16 pairs over the first 16 of this warp's own 32 fp32 columns
+      tc::st_16x128b_x4(ta, pa);
+      tc::st_16x128b_x4(ts, pd);
       tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();  // every lane's stores are complete: one lane arrives for the warp
-      if (lane == 0) mbar_arrive(smem_u32(&p_ready[j & 1]));
+      if (lane == 0) mbar_arrive(smem_u32(p_ready));
     }
     if (ok) {
       const bool done = mbar_wait_sleep(smem_u32(o_done), 0, kErrBwdElem);
