@@ -116,6 +116,51 @@ int plx_fwd_varlen(const void* q, const void* k, const void* v, const void* r,
                    float scale, void* stream);
 
 /*
+ * Context-parallel prefill.  The sequence is cut into consecutive chunks, one
+ * per rank.  A rank's queries attend its own chunk causally and every earlier
+ * chunk in full; each (query chunk, key chunk) block yields one partial state
+ * per query row, and the merge combines them.  The partial state over a set
+ * of keys is the streamed form's 5-tuple (news.chathome.org, "Parallax: ...",
+ * section "Hardware argument"): m (running max of the scaled scores, log2
+ * units), l = sum p, c = sum p s, O1 = sum p v, O2 = sum p s v.  Rescaled to a
+ * common max, the tuples of disjoint key sets add, so the merged output is
+ * o = O1/l - (O2/l - (c/l)(O1/l)) over the union of the keys.
+ *
+ * plx_fwd_partial_size -- bytes of one block: B * Hq * N * (2d + 4) fp32
+ *   (0 for invalid shapes).
+ */
+size_t plx_fwd_partial_size(int B, int Hq, int N, int d);
+
+/*
+ * plx_fwd_partial -- the partial states of the queries q against the keys
+ * k, v (one block).
+ *   q, r [B, Hq, N, d] bf16; k, v [B, Hkv, N, d] bf16: as plx_fwd, where the
+ *     N keys are one chunk (the query chunk itself with causal != 0, an
+ *     earlier chunk with causal == 0).
+ *   partial [B, Hq, N, 2d + 4] fp32, DEVICE, written: per query row m (log2
+ *     units; -inf for a row that saw no key), l, c, pad, O1[d], O2[d], with
+ *     l, c, O1, O2 relative to 2^m.
+ * Requirements and errors as plx_fwd; PLX_ERR_NULL for partial,
+ * PLX_ERR_WORKSPACE when partial_bytes < plx_fwd_partial_size.  One kernel
+ * (the prefill kernel with a partial-state epilogue) on `stream`.
+ */
+int plx_fwd_partial(const void* q, const void* k, const void* v, const void* r,
+                    float* partial, size_t partial_bytes,
+                    int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                    void* stream);
+
+/*
+ * plx_fwd_merge -- out and lse from `ranks` blocks of partial states.
+ *   partials [ranks, B, Hq, N, 2d + 4] fp32, DEVICE (block-major)
+ *   out [B, Hq, N, d] bf16; lse [B, Hq, N] fp32 (NULL: skipped)
+ * A row with no live key in any block gives out = 0, lse = -inf.  Errors:
+ * PLX_ERR_NULL, PLX_ERR_SHAPE (ranks, B, Hq or N < 1), PLX_ERR_HEADDIM,
+ * PLX_ERR_ALIGN (partials and out 16-byte, lse 4-byte aligned).
+ */
+int plx_fwd_merge(const float* partials, int ranks, int B, int Hq, int N, int d,
+                  void* out, float* lse, void* stream);
+
+/*
  * plx_fwd_train -- plx_fwd for training: the same outputs, plus two per-row
  * values that plx_bwd needs.
  *

@@ -1,14 +1,23 @@
-"""Context-parallel decode over torch.distributed: one rank per GPU, each
-holding a contiguous slice of every sequence's KV cache.
+"""Context parallelism over torch.distributed: one rank per GPU, each holding
+a contiguous slice of every sequence.
 
-Every rank computes the partial states of its slice (plx_decode_partial),
-the ranks all-gather them in rank order (the one exchange step: B * Hq *
-splits * (2d + 4) fp32 per rank, over NCCL on NVLink), and every rank merges
-them (plx_decode_merge).  The slices follow one another: rank r holds keys
-r * slice_len .. (r + 1) * slice_len - 1 of every sequence.
+Decode: every rank computes the partial states of its slice of the KV cache
+(plx_decode_partial), the ranks all-gather them in rank order (the one
+exchange step: B * Hq * splits * (2d + 4) fp32 per rank, over NCCL on
+NVLink), and every rank merges them (plx_decode_merge).  The slices follow
+one another: rank r holds keys r * slice_len .. (r + 1) * slice_len - 1 of
+every sequence.
+
+Prefill: rank r holds positions r * C .. (r + 1) * C - 1 of the queries,
+probes, keys and values.  The ranks all-gather the key and value chunks (the
+exchange step: 2 * B * Hkv * C * d bf16 per rank); rank r then computes the
+partial states of its queries against its own chunk (causal) and against
+each earlier chunk (in full), plx_fwd_partial, and merges the r + 1 blocks
+(plx_fwd_merge).  Later ranks do more blocks: the causal work is not
+balanced across ranks.
 
 The arithmetic runs in the library's kernels; this module only plans the
-slices and moves the partial states.
+slices and moves the data.
 """
 from __future__ import annotations
 
@@ -22,7 +31,8 @@ def slice_start(rank: int, slice_len: int) -> int:
 
 
 def gather_partials(partial: torch.Tensor, group=None) -> torch.Tensor:
-    """All-gather one partial block per rank into [world, *partial.shape], rank-major."""
+    """All-gather one block per rank (partial states, or a key / value chunk)
+    into [world, *partial.shape], rank-major."""
     world = dist.get_world_size(group)
     part = partial.contiguous()
     # the ranks' blocks concatenated along the first dimension (the layout every
@@ -50,3 +60,22 @@ def context_parallel_decode(q, kslice, vslice, seqlens, r=None, scale=None, num_
                                      scale=scale, num_splits=num_splits, stream=stream)
     gathered = gather_partials(partial, group)
     return plx.plx_decode_merge(gathered, return_lse=return_lse, stream=stream)
+
+
+def context_parallel_prefill(q, k, v, r=None, scale=None, group=None, return_lse=True, stream=None):
+    """Causal prefill with every sequence cut into consecutive chunks over the ranks of `group`.
+
+    q, r [B, Hq, C, d]; k, v [B, Hkv, C, d] bf16: this rank's chunk, positions
+    rank * C .. rank * C + C - 1 (the same C on every rank).  Returns this
+    rank's (out [B, Hq, C, d], lse [B, Hq, C]).
+    """
+    from . import plx
+
+    rank = dist.get_rank(group)
+    ks = gather_partials(k, group)  # [world, B, Hkv, C, d]
+    vs = gather_partials(v, group)
+    B, Hq, C, d = q.shape
+    partials = torch.empty((rank + 1, B, Hq, C, 2 * d + 4), dtype=torch.float32, device=q.device)
+    for j in range(rank + 1):
+        plx.plx_fwd_partial(q, ks[j], vs[j], r, causal=(j == rank), scale=scale, partial=partials[j], stream=stream)
+    return plx.plx_fwd_merge(partials, return_lse=return_lse, stream=stream)

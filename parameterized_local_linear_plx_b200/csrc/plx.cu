@@ -170,7 +170,7 @@ int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const plx::Decod
   return PLX_OK;
 }
 
-template <int D, bool HAS_R, bool SAVE_AUX>
+template <int D, bool HAS_R, int MODE>
 int launch_fwd(const CUtensorMap& qm, const CUtensorMap& rm, const CUtensorMap& km, const CUtensorMap& vm,
                const CUtensorMap& om, const CUtensorMap& am, const plx::FwdParams& p, unsigned grid,
                cudaStream_t st) {
@@ -178,7 +178,7 @@ int launch_fwd(const CUtensorMap& qm, const CUtensorMap& rm, const CUtensorMap& 
   static bool done[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  auto kern = plx::plx_fwd_kernel<D, HAS_R, SAVE_AUX>;
+  auto kern = plx::plx_fwd_kernel<D, HAS_R, MODE>;
   if (ensure_smem(kern, Cfg::kSmemBytes, &done[dev]) != PLX_OK) return PLX_ERR_CUDA;
   kern<<<grid, plx::kFwdThreads, Cfg::kSmemBytes, st>>>(qm, rm, km, vm, om, am, p);
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
@@ -244,12 +244,13 @@ namespace {
 // longest sequence.
 int fwd_common(const void* q, const void* k, const void* v, const void* r, void* out, float* lse,
                void* obar, float* sbar, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
-               void* stream, const int* cu_seqlens = nullptr, int total = 0) {
-  if (!q || !k || !v || !out) return PLX_ERR_NULL;
+               void* stream, const int* cu_seqlens = nullptr, int total = 0, float* partial = nullptr) {
+  if (!q || !k || !v || (!out && !partial)) return PLX_ERR_NULL;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return PLX_ERR_SHAPE;
   if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
   if (Hq % Hkv) return PLX_ERR_GQA;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (r && !aligned16(r)) || !aligned16(out) ||
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (r && !aligned16(r)) || (out && !aligned16(out)) ||
+      (partial && !aligned16(partial)) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (obar && !aligned16(obar)) ||
       (sbar && (reinterpret_cast<uintptr_t>(sbar) & 3u)) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
     return PLX_ERR_ALIGN;
@@ -276,8 +277,13 @@ int fwd_common(const void* q, const void* k, const void* v, const void* r, void*
   auto map_kv = [&](CUtensorMap* m, const void* base) {
     return packed ? make_map_3d_tokens(m, base, d, total, Hkv, plx::kFwdBN) : make_map_3d(m, base, d, N, pkv, plx::kFwdBN);
   };
-  if (map_q(&qm, q) != PLX_OK || map_kv(&km, k) != PLX_OK || map_kv(&vm, v) != PLX_OK || map_q(&om, out) != PLX_OK)
+  if (map_q(&qm, q) != PLX_OK || map_kv(&km, k) != PLX_OK || map_kv(&vm, v) != PLX_OK)
     return PLX_ERR_CUDA;
+  if (out) {
+    if (map_q(&om, out) != PLX_OK) return PLX_ERR_CUDA;
+  } else {
+    om = qm;  // unused: the partial-state forward writes no output tile
+  }
   if (r) {
     if (map_q(&rm, r) != PLX_OK) return PLX_ERR_CUDA;
   } else {
@@ -296,6 +302,7 @@ int fwd_common(const void* q, const void* k, const void* v, const void* r, void*
   p.cu_seqlens = cu_seqlens;
   p.total = total;
   p.lse_stride = packed ? total : N;
+  p.partial = partial;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.G = G;
   p.pair_heads = pair_heads; p.n_pairs = n_pairs; p.n_qblocks = n_qblocks;
   p.num_units = static_cast<int>(grid);
@@ -304,18 +311,28 @@ int fwd_common(const void* q, const void* k, const void* v, const void* r, void*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // persistent: one CTA per SM (the kernel's shared memory allows no more)
   const unsigned g = static_cast<unsigned>(std::min<long long>(grid, g_sm_count[dev]));
-  if (train) {
+  if (partial) {
+    constexpr int M = plx::kFwdModePartial;
     if (d == 128)
-      return r ? launch_fwd<128, true, true>(qm, rm, km, vm, om, am, p, g, st)
-               : launch_fwd<128, false, true>(qm, rm, km, vm, om, am, p, g, st);
-    return r ? launch_fwd<64, true, true>(qm, rm, km, vm, om, am, p, g, st)
-             : launch_fwd<64, false, true>(qm, rm, km, vm, om, am, p, g, st);
+      return r ? launch_fwd<128, true, M>(qm, rm, km, vm, om, am, p, g, st)
+               : launch_fwd<128, false, M>(qm, rm, km, vm, om, am, p, g, st);
+    return r ? launch_fwd<64, true, M>(qm, rm, km, vm, om, am, p, g, st)
+             : launch_fwd<64, false, M>(qm, rm, km, vm, om, am, p, g, st);
   }
+  if (train) {
+    constexpr int M = plx::kFwdModeTrain;
+    if (d == 128)
+      return r ? launch_fwd<128, true, M>(qm, rm, km, vm, om, am, p, g, st)
+               : launch_fwd<128, false, M>(qm, rm, km, vm, om, am, p, g, st);
+    return r ? launch_fwd<64, true, M>(qm, rm, km, vm, om, am, p, g, st)
+             : launch_fwd<64, false, M>(qm, rm, km, vm, om, am, p, g, st);
+  }
+  constexpr int M = plx::kFwdModeOut;
   if (d == 128)
-    return r ? launch_fwd<128, true, false>(qm, rm, km, vm, om, am, p, g, st)
-             : launch_fwd<128, false, false>(qm, rm, km, vm, om, am, p, g, st);
-  return r ? launch_fwd<64, true, false>(qm, rm, km, vm, om, am, p, g, st)
-           : launch_fwd<64, false, false>(qm, rm, km, vm, om, am, p, g, st);
+    return r ? launch_fwd<128, true, M>(qm, rm, km, vm, om, am, p, g, st)
+             : launch_fwd<128, false, M>(qm, rm, km, vm, om, am, p, g, st);
+  return r ? launch_fwd<64, true, M>(qm, rm, km, vm, om, am, p, g, st)
+           : launch_fwd<64, false, M>(qm, rm, km, vm, om, am, p, g, st);
 }
 
 }  // namespace
@@ -340,6 +357,20 @@ int plx_fwd_varlen(const void* q, const void* k, const void* v, const void* r, v
   if (!cu_seqlens) return PLX_ERR_NULL;
   return fwd_common(q, k, v, r, out, lse, nullptr, nullptr, B, Hq, Hkv, max_seqlen, d, causal, scale, stream,
                     cu_seqlens, total);
+}
+
+size_t plx_fwd_partial_size(int B, int Hq, int N, int d) {
+  if (B < 1 || Hq < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  return static_cast<size_t>(B) * Hq * N * (2 * d + 4) * sizeof(float);
+}
+
+int plx_fwd_partial(const void* q, const void* k, const void* v, const void* r, float* partial, size_t partial_bytes,
+                    int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  if (!partial) return PLX_ERR_NULL;
+  const size_t need = plx_fwd_partial_size(B, Hq, N, d);
+  if (need != 0 && partial_bytes < need) return PLX_ERR_WORKSPACE;  // bad shapes: fwd_common reports them
+  return fwd_common(q, k, v, r, nullptr, nullptr, nullptr, nullptr, B, Hq, Hkv, N, d, causal, scale, stream, nullptr,
+                    0, partial);
 }
 
 int plx_decode_paged(const void* q, const void* r, const void* kpool, const void* vpool,
@@ -617,14 +648,15 @@ int plx_decode_partial(const void* q, const void* r, const void* kcache, const v
                        partial, partial_bytes, stream, true, key_offset);
 }
 
-int plx_decode_merge(const float* partials, int ranks, int B, int Hq, int d, int num_splits, void* out, float* lse,
-                     void* stream) {
+// out / lse of `rows` rows from `ranks` blocks of partial states, each block
+// [rows, num_splits, 2d + 4] (the split-KV combine over ranks x splits)
+static int merge_common(const float* partials, int ranks, long long rows, int d, int num_splits, void* out, float* lse,
+                        void* stream) {
   if (!partials || !out) return PLX_ERR_NULL;
-  if (ranks < 1 || B < 1 || Hq < 1 || num_splits < 1) return PLX_ERR_SHAPE;
+  if (ranks < 1 || rows < 1 || num_splits < 1) return PLX_ERR_SHAPE;
   if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
   if (!aligned16(partials) || !aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return PLX_ERR_ALIGN;
-  const long long rows = static_cast<long long>(B) * Hq;
   if (rows > 0x7fffffffLL) return PLX_ERR_SHAPE;
   int dev = 0;
   int rc = check_arch(&dev);
@@ -638,6 +670,18 @@ int plx_decode_merge(const float* partials, int ranks, int B, int Hq, int d, int
     plx::plx_decode_combine_kernel<64><<<static_cast<unsigned>(rows), 64, 0, st>>>(
         partials, static_cast<__nv_bfloat16*>(out), lse, num_splits, ranks, rank_stride);
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
+int plx_decode_merge(const float* partials, int ranks, int B, int Hq, int d, int num_splits, void* out, float* lse,
+                     void* stream) {
+  if (B < 1 || Hq < 1) return (!partials || !out) ? PLX_ERR_NULL : PLX_ERR_SHAPE;
+  return merge_common(partials, ranks, static_cast<long long>(B) * Hq, d, num_splits, out, lse, stream);
+}
+
+int plx_fwd_merge(const float* partials, int ranks, int B, int Hq, int N, int d, void* out, float* lse,
+                  void* stream) {
+  if (B < 1 || Hq < 1 || N < 1) return (!partials || !out) ? PLX_ERR_NULL : PLX_ERR_SHAPE;
+  return merge_common(partials, ranks, static_cast<long long>(B) * Hq * N, d, 1, out, lse, stream);
 }
 
 int plx_check_device_status(void* stream) {

@@ -99,9 +99,17 @@ struct FwdParams {
   const int* cu_seqlens;
   int total;
   long long lse_stride;  // N (fixed length) or total (packed)
+  // partial-state forward only: [B, Hq, N, 2D + 4] fp32, per query row the
+  // record m (log2 units), l, c, pad, O1[D], O2[D] of the split-KV merge
+  float* partial;
 };
 
-template <int D, bool HAS_R, bool SAVE_AUX>
+// What the softmax warps write per unit: the output (and lse), the output plus
+// o_bar and s_bar for the backward, or the unnormalised partial state of each
+// row over this call's keys (context-parallel prefill merges those).
+constexpr int kFwdModeOut = 0, kFwdModeTrain = 1, kFwdModePartial = 2;
+
+template <int D, bool HAS_R, int MODE>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap rmap,
                const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
@@ -109,6 +117,7 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                const FwdParams p) {
   using Cfg = FwdCfg<D>;
   constexpr int NS = Cfg::kStages;
+  constexpr bool SAVE_AUX = MODE == kFwdModeTrain;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
@@ -519,6 +528,47 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       c_lo += __shfl_xor_sync(0xffffffffu, c_lo, 2);
       c_hi += __shfl_xor_sync(0xffffffffu, c_hi, 1);
       c_hi += __shfl_xor_sync(0xffffffffu, c_hi, 2);
+      if constexpr (MODE == kFwdModePartial) {
+        // This warp's 16 rows as partial states over this call's keys: O1 and
+        // O2 straight from tensor memory (relative to m, as accumulated),
+        // m = -inf for a row that saw no key.  Fixed-length layout only.
+        constexpr int PF = 2 * D + 4;
+        const size_t plane = static_cast<size_t>(qplane_of(w, t));
+        const bool live_lo = q_lo < w.N, live_hi = q_hi < w.N;
+        float* rec_lo = p.partial + (plane * p.N + static_cast<size_t>(live_lo ? q_lo : 0)) * PF;
+        float* rec_hi = p.partial + (plane * p.N + static_cast<size_t>(live_hi ? q_hi : 0)) * PF;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t o1[16], o2[16];
+          tc::ld_16x256b_x4(to1 + 32 * ch, o1);
+          tc::ld_16x256b_x4(to2 + 32 * ch, o2);
+          tc::wait_ld();
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg) {
+            const int dcol = 32 * ch + 8 * gg + 2 * c4;
+            if (live_lo) {
+              *reinterpret_cast<float2*>(rec_lo + 4 + dcol) =
+                  make_float2(__uint_as_float(o1[4 * gg]), __uint_as_float(o1[4 * gg + 1]));
+              *reinterpret_cast<float2*>(rec_lo + 4 + D + dcol) =
+                  make_float2(__uint_as_float(o2[4 * gg]), __uint_as_float(o2[4 * gg + 1]));
+            }
+            if (live_hi) {
+              *reinterpret_cast<float2*>(rec_hi + 4 + dcol) =
+                  make_float2(__uint_as_float(o1[4 * gg + 2]), __uint_as_float(o1[4 * gg + 3]));
+              *reinterpret_cast<float2*>(rec_hi + 4 + D + dcol) =
+                  make_float2(__uint_as_float(o2[4 * gg + 2]), __uint_as_float(o2[4 * gg + 3]));
+            }
+          }
+        }
+        // O has been read: the next unit's first value MMA may overwrite it
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&o_free[t]));
+        if (c4 == 0) {
+          if (live_lo) *reinterpret_cast<float4*>(rec_lo) = make_float4(m_lo, l_lo, c_lo, 0.f);
+          if (live_hi) *reinterpret_cast<float4*>(rec_hi) = make_float4(m_hi, l_hi, c_hi, 0.f);
+        }
+      } else {
       const float inv_lo = l_lo > 0.f ? 1.f / l_lo : 0.f;
       const float inv_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
       const float sb_lo = c_lo * inv_lo, sb_hi = c_hi * inv_hi;  // s_bar = c / l
@@ -636,6 +686,7 @@ plx_fwd_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           bulk_commit();
         }
       }
+      }  // output epilogue
       kv += w.nkv;
       ++n_unit;
     }

@@ -37,6 +37,12 @@ _lib.plx_fwd_varlen.restype = _I
 _lib.plx_fwd_varlen.argtypes = [_P] * 7 + [_I] * 7 + [_F, _P]
 _lib.plx_fwd_train.restype = _I
 _lib.plx_fwd_train.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
+_lib.plx_fwd_partial_size.restype = _SZ
+_lib.plx_fwd_partial_size.argtypes = [_I] * 4
+_lib.plx_fwd_partial.restype = _I
+_lib.plx_fwd_partial.argtypes = [_P] * 5 + [_SZ] + [_I] * 6 + [_F, _P]
+_lib.plx_fwd_merge.restype = _I
+_lib.plx_fwd_merge.argtypes = [_P] + [_I] * 5 + [_P, _P, _P]
 _lib.plx_bwd_workspace_size.restype = _SZ
 _lib.plx_bwd_workspace_size.argtypes = [_I, _I, _I, _I, _I]
 _lib.plx_bwd.restype = _I
@@ -143,6 +149,53 @@ def plx_fwd(q, k, v, r=None, causal=True, scale=None, out=None, lse=None, return
                       1 if causal else 0, float(scale), _stream(stream))
     if st != PLX_OK:
         raise PlxError(st, "plx_fwd")
+    return out, lse
+
+
+def plx_fwd_partial_size(B, Hq, N, d) -> int:
+    return int(_lib.plx_fwd_partial_size(B, Hq, N, d))
+
+
+def plx_fwd_partial(q, k, v, r=None, causal=True, scale=None, partial=None, stream=None):
+    """Partial states of the queries q against one chunk of keys k, v.
+
+    q, r [B, Hq, N, d], k/v [B, Hkv, N, d] bf16 CUDA.  Returns partial
+    [B, Hq, N, 2d + 4] fp32: per row m (log2 units), l, c, pad, O1[d], O2[d].
+    """
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    if r is not None:
+        _check(r, "r", torch.bfloat16, 4)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape or (r is not None and r.shape != q.shape):
+        raise ValueError("shape mismatch between q, k, v, r")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if partial is None:
+        partial = torch.empty((B, Hq, N, 2 * d + 4), device=q.device, dtype=torch.float32)
+    else:
+        _check(partial, "partial", torch.float32, 4)
+    st = _lib.plx_fwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(partial), partial.numel() * 4, B, Hq, Hkv, N,
+                              d, 1 if causal else 0, float(scale), _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_fwd_partial")
+    return partial
+
+
+def plx_fwd_merge(partials, out=None, lse=None, return_lse=True, stream=None):
+    """Merge blocks of partial states [blocks, B, Hq, N, 2d + 4] into (out, lse)."""
+    _check(partials, "partials", torch.float32, 5)
+    blocks, B, Hq, N, pf = partials.shape
+    d = (pf - 4) // 2
+    if out is None:
+        out = torch.empty((B, Hq, N, d), device=partials.device, dtype=torch.bfloat16)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, N), device=partials.device, dtype=torch.float32)
+    st = _lib.plx_fwd_merge(_ptr(partials), blocks, B, Hq, N, d, _ptr(out), _ptr(lse), _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_fwd_merge")
     return out, lse
 
 

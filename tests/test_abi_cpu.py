@@ -28,6 +28,7 @@ def declared_entry_points():
 def test_header_declares_the_boundary():
     names = declared_entry_points()
     for n in ["plx_fwd", "plx_fwd_train", "plx_bwd", "plx_bwd_workspace_size", "plx_decode_paged", "plx_kv_append", "plx_kv_append_paged", "plx_fwd_varlen", "plx_decode_partial", "plx_decode_merge", "plx_decode_partial_size",
+              "plx_fwd_partial", "plx_fwd_partial_size", "plx_fwd_merge",
               "plx_decode", "plx_decode_workspace_size", "plx_decode_num_splits",
               "plx_check_device_status", "plx_status_string", "plx_version", "plx_selftest_wait_timeout"]:
         assert n in names
@@ -232,3 +233,24 @@ def test_partial_and_merge_argument_errors(plx):
     assert mg(P(A), 2, 1, 2, 64, 0, P(A), P(A), None) == plx.PLX_ERR_SHAPE
     assert mg(P(A), 2, 1, 2, 80, 1, P(A), P(A), None) == plx.PLX_ERR_HEADDIM
     assert mg(P(A + 4), 2, 1, 2, 64, 1, P(A), P(A), None) == plx.PLX_ERR_ALIGN
+
+
+def test_prefill_partial_and_merge_argument_errors(plx):
+    fp = plx.lib.plx_fwd_partial
+    need = plx.plx_fwd_partial_size(1, 2, 64, 64)
+    assert need == 1 * 2 * 64 * (2 * 64 + 4) * 4
+    assert plx.plx_fwd_partial_size(1, 2, 64, 96) == 0 and plx.plx_fwd_partial_size(0, 2, 64, 64) == 0
+    qkv = [P(A), P(A), P(A), P(None)]
+    assert fp(*qkv, P(None), need, 1, 2, 1, 64, 64, 1, 0.125, None) == plx.PLX_ERR_NULL
+    assert fp(*qkv, P(A), need - 4, 1, 2, 1, 64, 64, 1, 0.125, None) == plx.PLX_ERR_WORKSPACE
+    assert fp(P(A), P(None), P(A), P(None), P(A), need, 1, 2, 1, 64, 64, 1, 0.125, None) == plx.PLX_ERR_NULL
+    assert fp(*qkv, P(A), need, 1, 2, 1, 64, 96, 1, 0.125, None) == plx.PLX_ERR_HEADDIM
+    assert fp(*qkv, P(A), 1 << 40, 1, 3, 2, 64, 64, 1, 0.125, None) == plx.PLX_ERR_GQA
+    assert fp(*qkv, P(A + 4), need, 1, 2, 1, 64, 64, 1, 0.125, None) == plx.PLX_ERR_ALIGN
+    assert fp(*qkv, P(A), need, 1, 2, 1, 0, 64, 1, 0.125, None) == plx.PLX_ERR_SHAPE
+    mg = plx.lib.plx_fwd_merge
+    assert mg(P(None), 2, 1, 2, 64, 64, P(A), P(A), None) == plx.PLX_ERR_NULL
+    assert mg(P(A), 0, 1, 2, 64, 64, P(A), P(A), None) == plx.PLX_ERR_SHAPE
+    assert mg(P(A), 2, 1, 2, 0, 64, P(A), P(A), None) == plx.PLX_ERR_SHAPE
+    assert mg(P(A), 2, 1, 2, 64, 80, P(A), P(A), None) == plx.PLX_ERR_HEADDIM
+    assert mg(P(A + 4), 2, 1, 2, 64, 64, P(A), P(A), None) == plx.PLX_ERR_ALIGN
