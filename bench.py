@@ -430,6 +430,9 @@ def run_gpu(args, world, rank, local):
     # ---- context-parallel decode, ranks emulated as slices on this GPU (timed on its own)
     cpd = run_cp(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes)
 
+    # ---- context-parallel prefill, the last rank emulated on this GPU (timed on its own)
+    cpp = run_cp_prefill(plx, args, dev, stream, local, tf_peak, peak_src)
+
     # ---- packed variable-length prefill with the same token count (timed on its own)
     varlen = run_varlen(plx, args, dev, stream, world, local, tf_peak, peak_src, tf_key)
 
@@ -467,6 +470,7 @@ def run_gpu(args, world, rank, local):
             "decode_paged": paged,
             "prefill_varlen": varlen,
             "decode_cp_emulated": cpd,
+            "prefill_cp_emulated": cpp,
             "backward": bwd,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
@@ -555,6 +559,57 @@ def run_cp(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes, ranks=8):
             "exchange_bytes_per_rank": part.numel() * 4,
             "note": "per-rank step time = partial + all-gather of exchange_bytes_per_rank + merge; the "
                     "all-gather is not measured (one GPU per run)"}
+
+
+def run_cp_prefill(plx, args, dev, stream, local, tf_peak, peak_src, ranks=4):
+    """The per-rank costs of context-parallel prefill for the prefill workload
+    cut into `ranks` chunks along the sequence, measured on this one GPU for
+    the last rank, which has the most blocks: its queries against its own
+    chunk (causal) and every earlier chunk (in full), then the merge."""
+    import torch
+    B, Hq, Hkv, d = PRE["B"], PRE["Hq"], PRE["Hkv"], PRE["d"]
+    C = PRE["N"] // ranks
+    g = torch.Generator(device=dev).manual_seed(400 + local)
+    q = torch.randn(B, Hq, C, d, generator=g, device=dev).bfloat16()
+    r = (0.1 * torch.randn(B, Hq, C, d, generator=g, device=dev)).bfloat16()
+    ks = torch.randn(ranks, B, Hkv, C, d, generator=g, device=dev).bfloat16()
+    vs = torch.randn(ranks, B, Hkv, C, d, generator=g, device=dev).bfloat16()
+    parts = torch.empty(ranks, B, Hq, C, 2 * d + 4, dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, C, dtype=torch.float32, device=dev)
+    last = ranks - 1
+
+    def blocks():
+        for j in range(ranks):
+            plx.plx_fwd_partial(q, ks[j], vs[j], r, causal=(j == last), partial=parts[j], stream=stream)
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n
+
+    n = max(1, min(args.steps, 20))
+    t_blocks = timed(blocks, n)
+    t_merge = timed(lambda: plx.plx_fwd_merge(parts, out=out, lse=lse, stream=stream), n)
+    st = plx.plx_check_device_status(stream)
+    if st != plx.PLX_OK:
+        raise RuntimeError(f"device status after the context-parallel prefill legs: {plx.plx_status_string(st)}")
+    flops = 8 * d * (C * (C + 1) // 2 + last * C * C) * B * Hq  # the last rank's (query, key) pairs
+    return {"workload": f"causal prefill B={B} N={PRE['N']} Hq={Hq} Hkv={Hkv} d={d} cut into {ranks} chunks of {C} "
+                        f"(one per rank); the last rank (most blocks) emulated on one GPU",
+            "ranks": ranks, "blocks_ms_last_rank": t_blocks, "merge_ms": t_merge,
+            "tflops_blocks": flops / (t_blocks * 1e-3) / 1e12, "frac_of_peak": flops / (t_blocks * 1e-3) / 1e12 / tf_peak,
+            "peak_source": peak_src,
+            "exchange_bytes_per_rank": 2 * B * Hkv * C * d * 2,
+            "note": "per-rank step time = all-gather of the key / value chunks + blocks + merge; the all-gather "
+                    "is not measured (one GPU per run); earlier ranks have fewer blocks"}
 
 
 VARLEN_LENS = [4096, 1, 2048, 777, 1024, 3000, 64, 65, 512, 1500, 4000, 129, 333, 2500, 100, 900,
