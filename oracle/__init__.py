@@ -1,3 +1,4 @@
 """fp64 CPU oracle for the Parallax attention forward pass and its gradients (test infrastructure only)."""
 from .plx_oracle import *  # noqa: F401,F403
 from .plx_oracle_bwd import *  # noqa: F401,F403
+from .plx_oracle_stream import *  # noqa: F401,F403
