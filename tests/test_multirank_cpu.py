@@ -74,3 +74,24 @@ def test_work_counts():
     assert abs(bench.prefill_flops(8, 16, 4096, 128) / 1e12 - 1.0998) < 1e-3
     assert bench.prefill_flops(1, 1, 3, 2, causal=False) == 8 * 2 * 9
     assert bench.decode_flops(16, 128, [4096] * 64) == 8 * 128 * 16 * 4096 * 64
+
+
+def test_traffic_figures_only_for_the_captured_sources(monkeypatch):
+    """The DRAM traffic in the bench line comes from profiles/ncu_traffic.json
+    only while the kernel's source files hash to the captured value."""
+    sys.path.insert(0, ROOT)
+    import bench
+    keys = ("prefill", "decode", "backward")
+    for k in keys:
+        v = bench.load_traffic(k)
+        assert v is None or v > 0
+    monkeypatch.setattr(bench, "source_hash", lambda k: "0" * 16)
+    assert all(bench.load_traffic(k) is None for k in keys)
+
+
+def test_backward_flop_count():
+    """16d per causal pair: twice the forward's 8d."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.backward_flops(8, 16, 4096, 128) == 2 * bench.prefill_flops(8, 16, 4096, 128)
+    assert bench.backward_flops(1, 1, 3, 2, causal=False) == 16 * 2 * 9
