@@ -62,12 +62,14 @@ def context_parallel_decode(q, kslice, vslice, seqlens, r=None, scale=None, num_
     return plx.plx_decode_merge(gathered, return_lse=return_lse, stream=stream)
 
 
-def context_parallel_prefill(q, k, v, r=None, scale=None, group=None, return_lse=True, stream=None):
-    """Causal prefill with every sequence cut into consecutive chunks over the ranks of `group`.
+def context_parallel_prefill(q, k, v, r=None, causal=True, scale=None, group=None, return_lse=True, stream=None):
+    """Prefill with every sequence cut into consecutive chunks over the ranks of `group`.
 
     q, r [B, Hq, C, d]; k, v [B, Hkv, C, d] bf16: this rank's chunk, positions
-    rank * C .. rank * C + C - 1 (the same C on every rank).  Returns this
-    rank's (out [B, Hq, C, d], lse [B, Hq, C]).
+    rank * C .. rank * C + C - 1 (the same C on every rank).  causal: the
+    queries attend their own chunk causally and the earlier chunks in full;
+    otherwise every chunk in full.  Returns this rank's (out [B, Hq, C, d],
+    lse [B, Hq, C]).
     """
     from . import plx
 
@@ -75,7 +77,9 @@ def context_parallel_prefill(q, k, v, r=None, scale=None, group=None, return_lse
     ks = gather_partials(k, group)  # [world, B, Hkv, C, d]
     vs = gather_partials(v, group)
     B, Hq, C, d = q.shape
-    partials = torch.empty((rank + 1, B, Hq, C, 2 * d + 4), dtype=torch.float32, device=q.device)
-    for j in range(rank + 1):
-        plx.plx_fwd_partial(q, ks[j], vs[j], r, causal=(j == rank), scale=scale, partial=partials[j], stream=stream)
+    blocks = rank + 1 if causal else ks.shape[0]
+    partials = torch.empty((blocks, B, Hq, C, 2 * d + 4), dtype=torch.float32, device=q.device)
+    for j in range(blocks):
+        plx.plx_fwd_partial(q, ks[j], vs[j], r, causal=(causal and j == rank), scale=scale, partial=partials[j],
+                            stream=stream)
     return plx.plx_fwd_merge(partials, return_lse=return_lse, stream=stream)

@@ -85,7 +85,9 @@ def _worker_prefill(rank, world, port, q):
         k = torch.full((B, Hkv, C, d), 10.0 * (rank + 1))
         v = torch.full((B, Hkv, C, d), 100.0 * (rank + 1))
         out, _ = cp.context_parallel_prefill(qq, k, v)
-        q.put((rank, calls, out.tolist()))
+        n_causal = len(calls)
+        out_full, _ = cp.context_parallel_prefill(qq, k, v, causal=False)
+        q.put((rank, calls[:n_causal], out.tolist(), calls[n_causal:], out_full.tolist()))
     finally:
         dist.destroy_process_group()
 
@@ -102,5 +104,6 @@ def test_two_gloo_ranks_prefill_blocks():
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
     res = sorted(q.get(timeout=5) for _ in range(2))
     shape = (1, 2, 4, 2 * 8 + 4)
-    assert res[0] == (0, [(True, 10.0, 100.0, shape)], [10.0])
-    assert res[1] == (1, [(False, 10.0, 100.0, shape), (True, 20.0, 200.0, shape)], [10.0, 20.0])
+    full = [(False, 10.0, 100.0, shape), (False, 20.0, 200.0, shape)]
+    assert res[0] == (0, [(True, 10.0, 100.0, shape)], [10.0], full, [10.0, 20.0])
+    assert res[1] == (1, [(False, 10.0, 100.0, shape), (True, 20.0, 200.0, shape)], [10.0, 20.0], full, [10.0, 20.0])
