@@ -321,7 +321,7 @@ def run_reference(args, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
         "config": bench_config(world),
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_threads(), "nproc": os.cpu_count(), "kind": "oracle",
                          "sample": f"decode only: {per_step} of the {DEC['B']} batch entries (x {DEC['Hq']} heads x "
                                    f"{DEC['S']} keys) per step, effective-weight fp64 form"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -444,7 +444,7 @@ def run_gpu(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         qh, kh, vh, rh, slh = (t.cpu() for t in (q, kc, vc, r, sl))
         n, secs, nb = oracle_decode_sample(qh, rh, kh, vh, slh, budget_s=10.0)
-        cpu = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+        cpu = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": cpu_threads(), "nproc": os.cpu_count(), "kind": "oracle",
                "sample": f"{n} (b) entries of the B={DEC['B']} decode step, cycling (each: all {DEC['Hq']} "
                          f"heads x {DEC['S']} keys), effective-weight fp64 form, {secs:.1f} s",
                "explicit_tiny_prefill_s": oracle_explicit_tiny()}

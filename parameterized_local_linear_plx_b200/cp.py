@@ -11,10 +11,11 @@ every sequence.
 Prefill: rank r holds positions r * C .. (r + 1) * C - 1 of the queries,
 probes, keys and values.  The ranks all-gather the key and value chunks (the
 exchange step: 2 * B * Hkv * C * d bf16 per rank); rank r then computes the
-partial states of its queries against its own chunk (causal) and against
-each earlier chunk (in full), plx_fwd_partial, and merges the r + 1 blocks
-(plx_fwd_merge).  Later ranks do more blocks: the causal work is not
-balanced across ranks.
+partial states of its queries block by block with plx_fwd_partial and merges
+them with plx_fwd_merge.  Causal: its own chunk (causal) and each earlier
+chunk (in full), r + 1 blocks, so later ranks do more blocks and the causal
+work is not balanced across ranks.  Non-causal: every chunk in full, `world`
+blocks on every rank.
 
 The arithmetic runs in the library's kernels; this module only plans the
 slices and moves the data.

@@ -23,7 +23,9 @@ def plx():
     return m
 
 
-def emulate(plx, q, k, v, r, ranks):
+def emulate(plx, q, k, v, r, ranks, causal=True):
+    """causal: rank rk merges its own chunk (causal) and the earlier chunks (in
+    full), rk + 1 blocks; otherwise every chunk in full, `ranks` blocks."""
     N = q.shape[2]
     C = N // ranks
 
@@ -34,8 +36,9 @@ def emulate(plx, q, k, v, r, ranks):
     for rk in range(ranks):
         qr = chunk(q, rk)
         rr = None if r is None else chunk(r, rk)
-        parts = torch.stack([plx.plx_fwd_partial(qr, chunk(k, j), chunk(v, j), rr, causal=(j == rk))
-                             for j in range(rk + 1)])
+        blocks = rk + 1 if causal else ranks
+        parts = torch.stack([plx.plx_fwd_partial(qr, chunk(k, j), chunk(v, j), rr, causal=(causal and j == rk))
+                             for j in range(blocks)])
         o, l = plx.plx_fwd_merge(parts)
         outs.append(o)
         lses.append(l)
@@ -60,6 +63,18 @@ def test_chunks_match_prefill_and_oracle(plx, ranks, d):
     close_to_prefill(plx, out, lse, q, k, v, r)
     ro, rl = oracle.prefill_effective(q.cpu(), k.cpu(), v.cpu(), r.cpu(), True)
     assert_close(out, ro, lse, rl, f"cp prefill ranks={ranks} d={d}")
+
+
+@pytest.mark.parametrize("ranks", [2, 3, 4])
+@pytest.mark.parametrize("d", [64, 128])
+def test_noncausal_chunks_match_prefill_and_oracle(plx, ranks, d):
+    """Every rank merges all `ranks` chunks in full; chunks of 96 rows."""
+    B, Hq, Hkv, C = 2, 4, 2, 96
+    q, k, v, r = inputs.prefill_inputs(B, Hq, Hkv, ranks * C, d, seed=70 + 10 * ranks + d, device="cuda")
+    out, lse = emulate(plx, q, k, v, r, ranks, causal=False)
+    close_to_prefill(plx, out, lse, q, k, v, r, causal=False)
+    ro, rl = oracle.prefill_effective(q.cpu(), k.cpu(), v.cpu(), r.cpu(), False)
+    assert_close(out, ro, lse, rl, f"cp prefill non-causal ranks={ranks} d={d}")
 
 
 def test_rho_none_and_odd_group(plx):

@@ -14,6 +14,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from parity import assert_close
 from parameterized_local_linear_plx_b200 import inputs
 
@@ -60,6 +61,8 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row(plx):
         torch.cuda.synchronize()
         assert plx.plx_check_device_status() == plx.PLX_OK
         assert_close(out, ref_o, lse, ref_l, f"noalloc vs decode {c}")
+        or_o, or_l = oracle.decode_effective(q.cpu(), r.cpu(), kc.cpu(), vc.cpu(), sl.cpu())
+        assert_close(out, or_o, lse, or_l, f"noalloc vs oracle {c}")
 
 
 def test_noalloc_rejects_requests_above_its_scratch(plx):
