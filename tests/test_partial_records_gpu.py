@@ -88,8 +88,14 @@ def test_decode_records(plx):
     qn, kn, vn, rn = f64(q), f64(kc), f64(vc), f64(r)
     scale = 1.0 / np.sqrt(d)
     G = Hq // Hkv
+    # one record per (b, h): compared over all B * Hq rows at once, as every
+    # parity test compares over the whole tensor (c/l of a single row is one
+    # scalar, whose relative error alone says nothing when it is near zero)
+    ref = [np.empty((B, Hq, d)), np.empty((B, Hq, d)), np.empty((B, Hq)), np.empty((B, Hq))]
     for b in range(B):
         n = int(sl[b])
         for h in range(Hq):
             st = oracle.chunk_state(qn[b, h], rn[b, h], kn[b, h // G, :n], vn[b, h // G, :n], scale)
-            compare(tuple(x[b, h] for x in dev), normalised_oracle(st), f"decode record b={b} h={h}")
+            for x, y in zip(ref, normalised_oracle(st)):
+                x[b, h] = y
+    compare(dev, tuple(ref), "decode records")
