@@ -2,7 +2,7 @@
 """Benchmark of the Parallax forward pass (decode + causal prefill) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--sweep] [--compute-matched]
+                    [--sweep] [--no-decode-configs] [--small]
 
 One step = one pass of the whole hot path over one batch of synthetic input:
   * decode: one plx_decode call on a Qwen3-0.6B-shaped layer, B=64, context
@@ -358,7 +358,7 @@ def run_gpu(args, world, rank, local):
     pout = torch.empty_like(pq)
     plse = torch.empty(PRE["B"], PRE["Hq"], PRE["N"], dtype=torch.float32, device=dev)
     n_splits = plx.plx_decode_num_splits(DEC["B"], DEC["Hq"], DEC["Hkv"], DEC["S"], DEC["d"])
-    launches_per_step = (2 if n_splits > 1 else 1) + 1
+    launches_per_step = 2 + 1  # decode split + combine, prefill
 
     def step(ev=None):
         if ev is not None:
@@ -436,9 +436,20 @@ def run_gpu(args, world, rank, local):
     # ---- packed variable-length prefill with the same token count (timed on its own)
     varlen = run_varlen(plx, args, dev, stream, world, local, tf_peak, peak_src, tf_key)
 
+    # ---- prefill end to end: inputs from pinned host memory, out and lse back
+    e2e_pre = run_e2e_prefill(plx, args, dev, stream, world, pq, pk, pv, pr)
+
+    # ---- the q/k/v/rho projection in front of the attention (timed on its own)
+    proj = run_projection(plx, args, dev, stream, world, tf_peak, f"{peak_src} {tf_key}")
+
     # ---- training backward of the prefill shape (timed on its own; not part of the step)
     bwd = run_backward(plx, args, dev, stream, world, local, pq, pk, pv, pr, peaks, peak_src)
 
+    # ---- every decode configuration (sweep, B=1/16, compute-matched), timed on its own, rank 0 at N=1
+    dcfg = None
+    if world == 1 and not args.no_decode_configs:
+        torch.cuda.empty_cache()
+        dcfg = decode_configs(plx, args, dev, hbm)
     # ---- CPU baseline: the oracle on this host, rank 0, N=1 only
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -457,7 +468,7 @@ def run_gpu(args, world, rank, local):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": bench_config(world),
             "decode": {"gbs": value, "us_per_step": dec_avg * 1e3, "us_median": statistics.median(dec_ms) * 1e3,
-                       "bytes_per_step": d_bytes, "splits": n_splits,
+                       "bytes_per_step": d_bytes, "partitions": n_splits,
                        "tflops": world * d_flops / (dec_avg * 1e-3) / 1e12},
             "prefill": {"tflops": prefill_tflops, "ms_per_step": pre_avg, "ms_median": statistics.median(pre_ms),
                         "flops_per_step": p_flops,
@@ -467,11 +478,14 @@ def run_gpu(args, world, rank, local):
             "roofline": roof_pre,
             "roofline_decode": roof_dec,
             "e2e": e2e,
+            "e2e_prefill": e2e_pre,
+            "projection": proj,
             "decode_paged": paged,
             "prefill_varlen": varlen,
             "decode_cp_emulated": cpd,
             "prefill_cp_emulated": cpp,
             "backward": bwd,
+            "decode_configs": dcfg,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
@@ -718,6 +732,113 @@ def run_backward(plx, args, dev, stream, world, local, pq, pk, pv, pr, peaks, pe
     }
 
 
+PROJ = dict(d_model=1024)  # Qwen3-0.6B hidden size
+
+
+def run_projection(plx, args, dev, stream, world, tf_peak, peak_src):
+    """plx_qkvr_proj at the prefill shape (tokens B*N = 32768, d_model = 1024,
+    W = [W_Q; W_K; W_V; W_R] of 6144 rows) and plx_qkvr_proj_decode at the
+    decode shape (B = 64 new tokens, k and v appended into a context-4096
+    cache); CUDA events around each call, max over ranks."""
+    import torch
+    B, N, Hq, Hkv, d = PRE["B"], PRE["N"], PRE["Hq"], PRE["Hkv"], PRE["d"]
+    dm = PROJ["d_model"]
+    nout = (2 * Hq + 2 * Hkv) * d
+    g = torch.Generator(device=dev).manual_seed(500)
+    x = torch.randn(B * N, dm, generator=g, device=dev).bfloat16()
+    w = (torch.randn(nout, dm, generator=g, device=dev) / dm ** 0.5).bfloat16()
+    q = torch.empty(B, Hq, N, d, dtype=torch.bfloat16, device=dev)
+    r = torch.empty_like(q)
+    k = torch.empty(B, Hkv, N, d, dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        for a, b in evs:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        return max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / n, world, dev)
+
+    n = max(1, min(args.steps, 20))
+    ms = timed(lambda: plx.plx_qkvr_proj(x, w, B, N, Hq, Hkv, d, q=q, k=k, v=v, r=r, stream=stream), n)
+    flops = 2 * B * N * dm * nout
+    achieved = flops / (ms * 1e-3) / 1e12
+    # decode step: 64 new tokens appended into a [64, 8, 4096, 128] cache at row 4000
+    Bd, S = DEC["B"], DEC["S"]
+    xd = torch.randn(Bd, dm, generator=g, device=dev).bfloat16()
+    kc = torch.zeros(Bd, Hkv, S, d, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    sl = torch.full((Bd,), S - 96, dtype=torch.int32, device=dev)
+    sl2 = torch.empty_like(sl)
+    qd = torch.empty(Bd, Hq, d, dtype=torch.bfloat16, device=dev)
+    rd = torch.empty_like(qd)
+    us_dec = 1e3 * timed(lambda: plx.plx_qkvr_proj_decode(xd, w, kc, vc, sl, Hq, seqlens_out=sl2, q=qd, r=rd,
+                                                          stream=stream), n)
+    st = plx.plx_check_device_status(stream)
+    if st != plx.PLX_OK:
+        raise RuntimeError(f"device status after the projection: {plx.plx_status_string(st)}")
+    w_bytes = nout * dm * 2
+    return {"workload": f"q/k/v/rho projection x W^T, x [{B * N}, {dm}], W [{nout}, {dm}] ([W_Q; W_K; W_V; W_R]), "
+                        f"outputs scattered to [B, H, N, d]; decode: {Bd} tokens, k/v appended into the cache",
+            "tflops": world * achieved, "ms_per_step": ms, "flops_per_step": flops,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
+                         "frac": achieved / tf_peak, "peak_source": peak_src},
+            "decode_us": us_dec,
+            "decode_gbs_weights": w_bytes / (us_dec * 1e-6) / 1e9,
+            "decode_note": "at 64 tokens the step is bound by reading W once (HBM); gbs counts the weight bytes"}
+
+
+def run_e2e_prefill(plx, args, dev, stream, world, pq, pk, pv, pr):
+    """plx_fwd measured with the step's q, k, v, r copied from pinned host
+    memory and out, lse copied back, all inside the timed region (one H2D
+    and one D2H copy per step, of packed buffers)."""
+    import torch
+    nq, nk = pq.numel() * 2, pk.numel() * 2
+    nout = pq.numel() * 2
+    nlse = PRE["B"] * PRE["Hq"] * PRE["N"] * 4
+    h_in = torch.empty(2 * nq + 2 * nk, dtype=torch.uint8).pin_memory()
+    offs = [0, nq, nq + nk, nq + 2 * nk]
+    for t, o, nb in ((pq, offs[0], nq), (pk, offs[1], nk), (pv, offs[2], nk), (pr, offs[3], nq)):
+        h_in[o:o + nb].view(torch.bfloat16).view(t.shape).copy_(t.cpu())
+    d_in = torch.empty_like(h_in, device=dev)
+    dq = d_in[offs[0]:offs[0] + nq].view(torch.bfloat16).view(pq.shape)
+    dk = d_in[offs[1]:offs[1] + nk].view(torch.bfloat16).view(pk.shape)
+    dv = d_in[offs[2]:offs[2] + nk].view(torch.bfloat16).view(pv.shape)
+    dr = d_in[offs[3]:offs[3] + nq].view(torch.bfloat16).view(pq.shape)
+    d_res = torch.empty(nout + nlse, dtype=torch.uint8, device=dev)
+    dout = d_res[:nout].view(torch.bfloat16).view(pq.shape)
+    dlse = d_res[nout:].view(torch.float32).view(PRE["B"], PRE["Hq"], PRE["N"])
+    h_res = torch.empty(nout + nlse, dtype=torch.uint8).pin_memory()
+
+    def one():
+        d_in.copy_(h_in, non_blocking=True)
+        plx.plx_fwd(dq, dk, dv, dr, causal=True, out=dout, lse=dlse, stream=stream)
+        h_res.copy_(d_res, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize(dev)
+    steps = max(1, min(args.steps, 10))
+    barrier(world, dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        one()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
+    flops = prefill_flops(PRE["B"], PRE["Hq"], PRE["N"], PRE["d"], True)
+    return {"value": world * flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h_in.numel(),
+            "d2h_bytes_per_step": h_res.numel(), "ms_per_step": ms}
+
+
 def run_e2e(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes):
     """Decode measured through plx_decode with the step's inputs (q, r,
     seqlens) copied from pinned host memory and its result (out, lse) read
@@ -763,75 +884,127 @@ def run_e2e(plx, args, dev, stream, world, q, kc, vc, r, sl, d_bytes):
             "d2h_bytes_per_step": h_res.numel(), "us_per_step": ms * 1e3}
 
 
-# ------------------------------------------------------------------ extra reports
-def run_sweep(args):
-    """Decode sweep: B x context with ragged seqlens in [ctx/2, ctx]; one JSON line per point."""
+# ------------------------------------------------------------------ decode configurations
+SWEEP_B = (1, 8, 64, 256, 1024, 2048)
+SWEEP_CTX = (128, 1024, 4096, 16384, 32768)
+SWEEP_CAP = 150e9  # bytes of KV cache above which a sweep point is skipped
+
+
+def time_decode_point(plx, torch, dev, pool_k, pool_v, B, ctx, d, seqlens_mode, seed, use_r=True, iters=10):
+    """Median CUDA-event time of one plx_decode call (split + combine) on a
+    [B, 8, ctx, d] cache viewed from the start of the pools; q, r ~ N(0,1),
+    N(0, 0.1^2); seqlens "equal" or "ragged" (uniform in [ctx/2, ctx]).  The
+    L2 is flushed before every timed call when the cache is under 4x its size."""
+    Hq, Hkv = 16, 8
+    n = B * Hkv * ctx * d
+    kc = pool_k[:n].view(B, Hkv, ctx, d)
+    vc = pool_v[:n].view(B, Hkv, ctx, d)
+    g = torch.Generator(device=dev).manual_seed(seed)
+    q = torch.randn(B, Hq, d, generator=g, device=dev).bfloat16()
+    r = (0.1 * torch.randn(B, Hq, d, generator=g, device=dev)).bfloat16() if use_r else None
+    if seqlens_mode == "equal":
+        sl = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+    else:
+        sl = torch.randint(ctx // 2, ctx + 1, (B,), generator=g, device=dev, dtype=torch.int32)
+    ws = torch.empty(plx.plx_decode_workspace_size(B, Hq, Hkv, ctx, d, 0), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    alloc = 2 * n * 2
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if alloc < 4 * L2_BYTES else None
+    for _ in range(5):
+        plx.plx_decode(q, kc, vc, sl, r, out=out, lse=lse, workspace=ws)
+    # calls enqueued back to back (flush, event, call, event, ...) and one
+    # synchronize at the end: each call's events time its GPU work, while the
+    # host enqueues the next one (host-side cost is reported separately)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        if flush is not None:
+            flush.zero_()
+        a.record()
+        plx.plx_decode(q, kc, vc, sl, r, out=out, lse=lse, workspace=ws)
+        b.record()
+    torch.cuda.synchronize()
+    ts = [a.elapsed_time(b) for a, b in evs]
+    st = plx.plx_check_device_status()
+    if st != plx.PLX_OK:
+        raise RuntimeError(f"device status after decode point ({B}, {ctx}): {plx.plx_status_string(st)}")
+    ms = statistics.median(ts)
+    nb = decode_bytes(B, Hq, Hkv, d, sl.tolist())
+    return {"B": B, "ctx": ctx, "d": d, "seqlens": seqlens_mode, "us": ms * 1e3, "bytes": nb,
+            "gbs": nb / (ms * 1e-3) / 1e9, "kv_alloc_gb": alloc / 1e9, "flushed_l2": flush is not None}
+
+
+def decode_configs(plx, args, dev, hbm):
+    """Every decode configuration of the workload list, timed on this GPU:
+    the Qwen3-0.6B-shaped layer at B = 1 and 16 (B = 64 is the bench's own
+    decode), the sweep B x context with ragged lengths (points whose KV cache
+    exceeds 150 GB skipped), and the compute-matched pair (Parallax at d = 64
+    against the softmax-only path at d = 128, B = 128, context 32768).  One
+    pair of K/V pools sized for the largest point is drawn once and viewed
+    for every point."""
     import torch
-    from parameterized_local_linear_plx_b200 import build, inputs
-    build.build()
-    from parameterized_local_linear_plx_b200 import plx
-    dev = torch.device("cuda", 0)
-    for B in (1, 8, 64, 256, 1024, 2048):
-        for ctx in (128, 1024, 4096, 16384, 32768):
-            alloc = B * ctx * 8 * 2 * 128 * 2
-            if alloc > 150e9:
-                print(json.dumps({"sweep": [B, ctx], "skipped": "KV cache above 150 GB"}), flush=True)
+    elems = 0
+    for B in SWEEP_B:
+        for ctx in SWEEP_CTX:
+            if B * ctx * 8 * 2 * 128 * 2 <= SWEEP_CAP:
+                elems = max(elems, B * 8 * ctx * 128)
+    free, _ = torch.cuda.mem_get_info(dev)
+    if 2 * elems * 2 > free - (4 << 30):
+        return {"skipped": f"needs {4 * elems / 1e9:.0f} GB of free device memory, {free / 1e9:.0f} GB free"}
+    pool_k = torch.empty(elems, dtype=torch.bfloat16, device=dev)
+    pool_v = torch.empty(elems, dtype=torch.bfloat16, device=dev)
+    g = torch.Generator(device=dev).manual_seed(1234)
+    step = 1 << 28
+    for pool in (pool_k, pool_v):
+        for i0 in range(0, elems, step):
+            i1 = min(elems, i0 + step)
+            pool[i0:i1].copy_(torch.randn(i1 - i0, generator=g, device=dev))
+    iters = 10 if not args.small else 3
+    res = {"peak_hbm_gbs": hbm, "spec_hbm_gbs": 8000.0,
+           "timing": f"median of {iters} calls enqueued back to back, CUDA events around each call, 5 warm-up; "
+                     f"L2 flushed before each call when the cache is under 4x L2"}
+    res["config2"] = []
+    for B in (1, 16):
+        pt = time_decode_point(plx, torch, dev, pool_k, pool_v, B, 4096, 128, "equal", seed=B, iters=iters)
+        pt["frac_of_hbm"] = pt["gbs"] / hbm
+        pt["frac_of_spec"] = pt["gbs"] / 8000.0
+        res["config2"].append(pt)
+    res["sweep"] = []
+    for B in SWEEP_B:
+        for ctx in SWEEP_CTX:
+            if B * ctx * 8 * 2 * 128 * 2 > SWEEP_CAP:
+                res["sweep"].append({"B": B, "ctx": ctx, "skipped": "KV cache above 150 GB"})
                 continue
-            q, kc, vc, r, sl = inputs.decode_inputs(B, 16, 8, ctx, 128, seed=0, seqlens="ragged", device=dev)
-            ws = torch.empty(max(16, plx.plx_decode_workspace_size(B, 16, 8, ctx, 128, 0)), dtype=torch.uint8,
-                             device=dev)
-            out = torch.empty_like(q)
-            lse = torch.empty(B, 16, dtype=torch.float32, device=dev)
-            flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if alloc < 4 * L2_BYTES else None
-            for _ in range(5):
-                plx.plx_decode(q, kc, vc, sl, r, out=out, lse=lse, workspace=ws)
-            ts = []
-            for _ in range(20):
-                if flush is not None:
-                    flush.zero_()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record()
-                plx.plx_decode(q, kc, vc, sl, r, out=out, lse=lse, workspace=ws)
-                b.record()
-                torch.cuda.synchronize()
-                ts.append(a.elapsed_time(b))
-            ms = statistics.median(ts)
-            nb = decode_bytes(B, 16, 8, 128, sl.tolist())
-            print(json.dumps({"sweep": [B, ctx], "us": ms * 1e3, "gbs": nb / (ms * 1e-3) / 1e9, "bytes": nb,
-                              "splits": plx.plx_decode_num_splits(B, 16, 8, ctx, 128)}), flush=True)
-            del q, kc, vc, r, sl, ws, out, lse, flush
-            torch.cuda.empty_cache()
+            pt = time_decode_point(plx, torch, dev, pool_k, pool_v, B, ctx, 128, "ragged", seed=B * 7 + ctx,
+                                   iters=iters)
+            pt["frac_of_hbm"] = pt["gbs"] / hbm
+            pt["frac_of_spec"] = pt["gbs"] / 8000.0
+            pt["bar_applies"] = pt["bytes"] >= 100e6  # ~100 MB and up: not launch-bound
+            res["sweep"].append(pt)
+    cm = {}
+    for name, d, use_r in (("parallax_d64", 64, True), ("softmax_d128", 128, False)):
+        cm[name] = time_decode_point(plx, torch, dev, pool_k, pool_v, 128, 32768, d, "equal", seed=5, use_r=use_r,
+                                     iters=iters)
+    cm["speedup_parallax_d64_over_softmax_d128"] = cm["softmax_d128"]["us"] / cm["parallax_d64"]["us"]
+    res["compute_matched"] = cm
+    big = [p for p in res["sweep"] if p.get("bar_applies")]
+    res["sweep_min_frac_of_spec_at_100MB_and_up"] = min(p["frac_of_spec"] for p in big) if big else None
+    del pool_k, pool_v
+    torch.cuda.empty_cache()
+    return res
 
 
-def run_compute_matched(args):
-    """Parallax at d=64 vs the library's softmax-only path (r = NULL) at d=128,
-    B=128, context 32768, Hq=16, Hkv=8."""
+def run_sweep(args):
+    """--sweep: the decode configurations as one JSON line."""
     import torch
-    from parameterized_local_linear_plx_b200 import build, inputs
+    from parameterized_local_linear_plx_b200 import build
     build.build()
     from parameterized_local_linear_plx_b200 import plx
     dev = torch.device("cuda", 0)
-    res = {}
-    for name, d, use_r in (("parallax_d64", 64, True), ("softmax_d128", 128, False)):
-        q, kc, vc, r, sl = inputs.decode_inputs(128, 16, 8, 32768, d, seed=0, device=dev)
-        for _ in range(5):
-            plx.plx_decode(q, kc, vc, sl, r if use_r else None)
-        ts = []
-        for _ in range(20):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            plx.plx_decode(q, kc, vc, sl, r if use_r else None)
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        ms = statistics.median(ts)
-        nb = decode_bytes(128, 16, 8, d, sl.tolist())
-        res[name] = {"us": ms * 1e3, "gbs": nb / (ms * 1e-3) / 1e9, "gflop": decode_flops(16, d, sl.tolist()) / 1e9
-                     * (1 if use_r else 0.5)}
-        del q, kc, vc, r, sl
-        torch.cuda.empty_cache()
-    res["speedup_parallax_d64_over_softmax_d128"] = res["softmax_d128"]["us"] / res["parallax_d64"]["us"]
-    print(json.dumps({"compute_matched": res}), flush=True)
+    peaks, _ = load_peaks()
+    print(json.dumps({"decode_configs": decode_configs(plx, args, dev, float(peaks.get("hbm_gbs", 6650.0)))}),
+          flush=True)
 
 
 def main():
@@ -843,8 +1016,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--small", action="store_true",
                     help="profiling-size workload: decode B=16, prefill B=2 (both still larger than L2)")
-    ap.add_argument("--sweep", action="store_true", help="decode sweep lines instead of the bench line")
-    ap.add_argument("--compute-matched", action="store_true", help="compute-matched decode comparison")
+    ap.add_argument("--sweep", action="store_true", help="only the decode configurations (sweep, B=1/16, "
+                    "compute-matched) as one JSON line")
+    ap.add_argument("--no-decode-configs", action="store_true", help="leave the decode configurations out of the "
+                    "bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -858,8 +1033,6 @@ def main():
         return run_reference(args, world, rank)
     if args.sweep:
         return run_sweep(args)
-    if args.compute_matched:
-        return run_compute_matched(args)
     if world > 1:
         import datetime
 

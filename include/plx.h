@@ -323,6 +323,60 @@ int plx_kv_append_paged(const void* knew, const void* vnew, void* kpool, void* v
                         void* stream);
 
 /*
+ * The projection in front of the attention.  The pages make the probe rho one
+ * more learned projection of the layer input, beside q, k and v
+ * (news.chathome.org, "Parallax: ...", section "What is Parallax"; gist.science,
+ * "Technical overview: Parallax ...", "Method: Parallax / Core mechanism").  The
+ * four weights are stacked along the output dimension,
+ *
+ *     w = [W_Q; W_K; W_V; W_R]   [Nout, d_model] bf16, row-major (a row per
+ *                                output feature), Nout = (2 Hq + 2 Hkv) d,
+ *                                rows: Hq*d of W_Q, Hkv*d of W_K, Hkv*d of W_V,
+ *                                Hq*d of W_R (head-major, d per head);
+ *                                with r == NULL the W_R rows are absent,
+ *                                Nout = (Hq + 2 Hkv) d,
+ *
+ * and one GEMM y = x w^T (bf16 operands, fp32 accumulation, bf16 results on
+ * tcgen05 tensor cores) gives all four; its epilogue writes every head's d
+ * columns straight into the layout the attention reads.  No bias, no
+ * normalisation, no positional rotation: the pages name none.  One kernel on
+ * `stream`; no workspace.
+ *
+ * plx_qkvr_proj -- prefill: x [B * N, d_model] bf16 (token m = b N + t);
+ *   writes q, r [B, Hq, N, d] and k, v [B, Hkv, N, d] (r may be NULL).
+ * Requirements: B, N >= 1; d_model >= 8 and a multiple of 8; d in {64, 128};
+ * Hq % Hkv == 0; pointers 16-byte aligned.  Errors: PLX_ERR_NULL,
+ * PLX_ERR_SHAPE, PLX_ERR_HEADDIM, PLX_ERR_GQA, PLX_ERR_ALIGN, PLX_ERR_CUDA.
+ */
+int plx_qkvr_proj(const void* x, const void* w, void* q, void* k, void* v, void* r,
+                  int B, int N, int d_model, int Hq, int Hkv, int d, void* stream);
+
+/*
+ * plx_qkvr_proj_decode -- one decode step's projection with the KV append
+ * fused in: x [B, d_model] bf16 holds each sequence's new token; writes
+ * q, r [B, Hq, d] and the token's k, v of every KV head into
+ * kcache, vcache [B, Hkv, S_max, d] at row seqlens[b].  An entry with
+ * seqlens[b] < 0 or >= S_max gets no k, v.  seqlens_out (DEVICE int32 [B],
+ * may be NULL; must not be seqlens) receives seqlens[b] + 1 where the token
+ * was written and seqlens[b] elsewhere: the lengths the decode step then
+ * reads.  Requirements and errors as plx_qkvr_proj, plus S_max >= 1.
+ */
+int plx_qkvr_proj_decode(const void* x, const void* w, void* q, void* r, void* kcache, void* vcache,
+                         const int32_t* seqlens, int32_t* seqlens_out, int B, int d_model, int Hq, int Hkv,
+                         int S_max, int d, void* stream);
+
+/*
+ * plx_qkvr_proj_decode_paged -- plx_qkvr_proj_decode for the page pools of
+ * plx_decode_paged: k, v go to row seqlens[b] % page_size of page
+ * block_table[b * max_pages + seqlens[b] / page_size]; nothing is written for
+ * a slot past max_pages * page_size or a page id outside [0, num_pages).
+ */
+int plx_qkvr_proj_decode_paged(const void* x, const void* w, void* q, void* r, void* kpool, void* vpool,
+                               const int32_t* block_table, const int32_t* seqlens, int32_t* seqlens_out, int B,
+                               int d_model, int Hq, int Hkv, int num_pages, int page_size, int max_pages, int d,
+                               void* stream);
+
+/*
  * Context-parallel decode: the KV cache of each sequence is split along the
  * sequence over `ranks` GPUs (rank r holds a contiguous slice of the keys).
  * Each rank computes the partial state of its slice with
@@ -365,7 +419,7 @@ int plx_decode_partial(const void* q, const void* r, const void* kcache, const v
  *   out [B, Hq, d] bf16; lse [B, Hq] fp32 (NULL: skipped)
  * A row with no live key in any rank gives out = 0, lse = -inf.
  */
-int plx_decode_merge(const float* partials, int ranks, int B, int Hq, int d, int num_splits,
+int plx_decode_merge(const float* partials, int ranks, int B, int Hq, int d,
                      void* out, float* lse, void* stream);
 
 /*

@@ -1,10 +1,10 @@
 """Context parallelism over torch.distributed: one rank per GPU, each holding
 a contiguous slice of every sequence.
 
-Decode: every rank computes the partial states of its slice of the KV cache
-(plx_decode_partial), the ranks all-gather them in rank order (the one
-exchange step: B * Hq * splits * (2d + 4) fp32 per rank, over NCCL on
-NVLink), and every rank merges them (plx_decode_merge).  The slices follow
+Decode: every rank computes the state record of its slice of the KV cache
+per (b, h) (plx_decode_partial), the ranks all-gather them in rank order (the
+one exchange step: B * Hq * (2d + 4) fp32 per rank, over NCCL on NVLink), and
+every rank merges them (plx_decode_merge).  The slices follow
 one another: rank r holds keys r * slice_len .. (r + 1) * slice_len - 1 of
 every sequence.
 
@@ -50,8 +50,8 @@ def context_parallel_decode(q, kslice, vslice, seqlens, r=None, scale=None, num_
     q, r [B, Hq, d] bf16 (the same on every rank); kslice, vslice
     [B, Hkv, slice_len, d] bf16: this rank's slice; seqlens [B] int32: the full
     lengths (the same on every rank).  Every rank returns the full (out, lse).
-    num_splits must resolve to the same count on every rank (0: automatic,
-    which depends on the shapes only).
+    num_splits: the work partitions of this rank's decode kernel (0:
+    automatic); ranks may differ, since each sends one record per (b, h).
     """
     from . import plx
 

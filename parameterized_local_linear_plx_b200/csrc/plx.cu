@@ -16,11 +16,11 @@
 #include "plx_bwd.cuh"
 #include "plx_decode.cuh"
 #include "plx_fwd.cuh"
+#include "plx_proj.cuh"
 
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kSmCount = 148;  // B200
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -66,8 +66,46 @@ int get_encoder() {
 // A bf16 tensor [planes, rows, D] (D contiguous) as a 3-D TMA map with a
 // box of {64 elements, box_rows, 1} and 128-byte swizzle.  Loads past `rows`
 // (inside a plane) are zero-filled, so ragged tails never read a neighbour.
-int make_map_3d(CUtensorMap* map, const void* base, int D, long long rows, long long planes,
-                int box_rows) {
+// Encoded maps are cached per (base, D, rows, planes, box_rows): a decode
+// step at a steady shape re-encodes nothing (the encode is host work on the
+// critical path of a small call).  A map holds only the address, extents and
+// strides, so a cached entry stays valid for any buffer at that address.
+struct MapKey {
+  const void* base;
+  long long rows, planes;
+  int D, box_rows;
+};
+constexpr int kMapCache = 64;
+MapKey g_map_keys[kMapCache];
+CUtensorMap g_map_vals[kMapCache];
+int g_map_next = 0;
+std::mutex g_map_mu;
+
+int encode_map_3d(CUtensorMap* map, const void* base, int D, long long rows, long long planes, int box_rows);
+
+int make_map_3d(CUtensorMap* map, const void* base, int D, long long rows, long long planes, int box_rows) {
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    for (int i = 0; i < kMapCache; ++i) {
+      const MapKey& k = g_map_keys[i];
+      if (k.base == base && k.base != nullptr && k.rows == rows && k.planes == planes && k.D == D &&
+          k.box_rows == box_rows) {
+        *map = g_map_vals[i];
+        return PLX_OK;
+      }
+    }
+  }
+  const int rc = encode_map_3d(map, base, D, rows, planes, box_rows);
+  if (rc == PLX_OK) {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    g_map_keys[g_map_next] = MapKey{base, rows, planes, D, box_rows};
+    g_map_vals[g_map_next] = *map;
+    g_map_next = (g_map_next + 1) % kMapCache;
+  }
+  return rc;
+}
+
+int encode_map_3d(CUtensorMap* map, const void* base, int D, long long rows, long long planes, int box_rows) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(planes)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2u,
@@ -97,6 +135,20 @@ int make_map_3d_tokens(CUtensorMap* map, const void* base, int D, long long rows
   return rc == CUDA_SUCCESS ? PLX_OK : PLX_ERR_CUDA;
 }
 
+// A row-major bf16 matrix [rows, cols] as a 2-D TMA map with a box of
+// {64 columns, box_rows rows} and 128-byte swizzle; loads past either extent
+// are zero-filled.
+int make_map_2d(CUtensorMap* map, const void* base, long long cols, long long rows, int box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2u};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult rc = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS ? PLX_OK : PLX_ERR_CUDA;
+}
+
 // Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
 template <typename K>
 int ensure_smem(K kernel, int bytes, bool* done) {
@@ -108,65 +160,120 @@ int ensure_smem(K kernel, int bytes, bool* done) {
 }
 
 // ---------------------------------------------------------------- decode
-struct SplitPlan {
-  int splits, chunk;
-};
+// The decode split kernel runs P persistent CTAs (two per SM by default) over
+// the key tiles of the whole batch; its scratch holds two partial-state slots
+// per CTA (rows_per_slot rows each) and one int4 per CTA for the combine.
+size_t align256(size_t n) { return (n + 255) / 256 * 256; }
 
-SplitPlan plan_splits(int B, int Hq, int Hkv, int S_max, int num_splits) {
-  const int G = Hq / Hkv;
-  const int n_hg = (G + 7) / 8;
-  const long long units = static_cast<long long>(B) * Hkv * n_hg;
-  int splits = num_splits;
-  if (splits <= 0) {
-    const long long target = 4LL * 2 * kSmCount;  // about four waves of two CTAs per SM
-    long long s = (target + units - 1) / units;
-    const long long max_s = (S_max + 127) / 128;  // chunks of at least 128 keys
-    if (s > max_s) s = max_s;
-    if (s < 1) s = 1;
-    splits = static_cast<int>(s);
-  }
-  if (splits > S_max) splits = S_max;
-  int chunk = (S_max + splits - 1) / splits;
-  chunk = (chunk + plx::kDecTileKeys - 1) / plx::kDecTileKeys * plx::kDecTileKeys;
-  splits = (S_max + chunk - 1) / chunk;
-  return {splits, chunk};
+int sm_count_or_default() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+    return sms;
+  return 148;  // B200
 }
 
-size_t workspace_bytes_for(int B, int Hq, int d, int splits) {
-  if (splits <= 1) return 0;
-  return static_cast<size_t>(B) * Hq * splits * (2 * d + 4) * sizeof(float);
+int decode_ctas(int num_splits) { return num_splits > 0 ? num_splits : 2 * sm_count_or_default(); }
+
+int rows_per_slot(int Hq, int Hkv) { return std::min(Hq / Hkv, 8); }
+
+size_t decode_scratch_bytes(int Hq, int Hkv, int d, int P) {
+  return align256(static_cast<size_t>(2) * P * rows_per_slot(Hq, Hkv) * (2 * d + 4) * sizeof(float));
+}
+
+// Two plans share the decode kernel.  The balanced plan (persistent CTAs over
+// equal ranges of the batch's tile list) wins when the batch has few (b, kv
+// head) segments, or short ones; with many long segments the chunked plan
+// (one CTA per chunk of a segment, like a split-KV grid, several waves)
+// streams the cache faster.  Measured crossover: 128 segments or more, of
+// more than 256 keys.
+constexpr long long kChunkedMinSegments = 128;
+constexpr int kChunkedMinKeys = 256;
+
+struct DecodePlan {
+  bool chunked;
+  int P;            // CTAs of the decode kernel
+  int splits;       // chunked: parts per segment
+  int chunk_tiles;  // chunked: tiles per part
+  size_t ws_bytes;  // workspace the plan needs
+};
+
+DecodePlan plan_decode(int B, int Hq, int Hkv, int S_max, int d, int num_splits, bool records) {
+  DecodePlan pl{};
+  const int n_hg = (Hq / Hkv + 7) / 8;
+  const long long segs = static_cast<long long>(B) * Hkv * n_hg;
+  if (num_splits == 0 && !records && segs >= kChunkedMinSegments && S_max > kChunkedMinKeys && B <= 65535 &&
+      static_cast<long long>(Hkv) * n_hg <= 65535) {
+    // about four waves of two CTAs per SM, chunks of at least 128 keys
+    const long long target = 4LL * 2 * sm_count_or_default();
+    long long sp = (target + segs - 1) / segs;
+    const long long max_sp = (S_max + 127) / 128;
+    sp = std::max(1LL, std::min(sp, max_sp));
+    const int keys = static_cast<int>((S_max + sp - 1) / sp);
+    pl.chunked = true;
+    pl.chunk_tiles = (keys + plx::kDecTileKeys - 1) / plx::kDecTileKeys;
+    pl.splits = (S_max + pl.chunk_tiles * plx::kDecTileKeys - 1) / (pl.chunk_tiles * plx::kDecTileKeys);
+    pl.P = static_cast<int>(std::min<long long>(segs * pl.splits, 0x7fffffffLL));
+    pl.ws_bytes = pl.splits > 1 ? align256(static_cast<size_t>(B) * Hq * pl.splits * (2 * d + 4) * sizeof(float)) : 0;
+    return pl;
+  }
+  pl.chunked = false;
+  pl.P = decode_ctas(num_splits);
+  pl.ws_bytes = decode_scratch_bytes(Hq, Hkv, d, pl.P);
+  return pl;
 }
 
 template <int D, bool HAS_R, bool PAGED>
-int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const plx::DecodeParams& p, int n_hg,
+int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const plx::DecodeParams& p, int P,
                   cudaStream_t st) {
   using Cfg = plx::DecodeCfg<D>;
-  static bool done[kMaxDevices];
+  static bool done[kMaxDevices], done_chunk[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  auto kern = plx::plx_decode_split_kernel<D, HAS_R, PAGED>;
-  if (ensure_smem(kern, Cfg::kSmemBytes, &done[dev]) != PLX_OK) return PLX_ERR_CUDA;
-  dim3 grid(p.splits, p.Hkv * n_hg, p.B);
-  kern<<<grid, plx::kDecThreads, Cfg::kSmemBytes, st>>>(km, vm, p);
-  if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
-  if (p.splits > 1 && !p.partial_out) {
-    // programmatic dependent launch: the combine is scheduled as the split
-    // CTAs finish, and griddepcontrol.wait inside it orders it after them
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(p.B * p.Hq));
-    cfg.blockDim = dim3(D);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const float* ws = p.ws;
-    if (cudaLaunchKernelEx(&cfg, plx::plx_decode_combine_kernel<D>, ws, p.out, p.lse, p.splits, 1,
-                           static_cast<size_t>(0)) != cudaSuccess)
-      return PLX_ERR_CUDA;
+  if (p.chunk_tiles > 0) {
+    auto kern = plx::plx_decode_chunk_kernel<D, HAS_R, PAGED>;
+    if (ensure_smem(kern, Cfg::kChunkSmemBytes, &done_chunk[dev]) != PLX_OK) return PLX_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(p.splits), static_cast<unsigned>(p.Hkv * p.n_hgroups),
+                    static_cast<unsigned>(p.B));
+    kern<<<grid, plx::kDecThreads, Cfg::kChunkSmemBytes, st>>>(km, vm, p);
+    if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+    if (p.splits == 1) return PLX_OK;  // every segment was finished whole
+  } else {
+    auto kern = plx::plx_decode_split_kernel<D, HAS_R, PAGED>;
+    if (ensure_smem(kern, Cfg::kSmemBytes, &done[dev]) != PLX_OK) return PLX_ERR_CUDA;
+    kern<<<static_cast<unsigned>(P), plx::kDecThreads, Cfg::kSmemBytes, st>>>(km, vm, p);
+    if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
   }
+  // programmatic dependent launch: the second kernel's CTAs are scheduled
+  // while the decode grid runs, and griddepcontrol.wait inside it orders its
+  // reads after that grid's completion
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  if (p.chunk_tiles > 0) {
+    // the parts of every row: [B * Hq rows, splits, 2D + 4] merged one warp per row
+    const long long rows = static_cast<long long>(p.B) * p.Hq;
+    const long long threads = rows * (D / 4);
+    cfg.gridDim = dim3(static_cast<unsigned>((threads + 255) / 256));
+    cfg.blockDim = dim3(256);
+    const long long rf = 2 * D + 4;
+    if (cudaLaunchKernelEx(&cfg, plx::plx_record_merge_kernel<D>, static_cast<const float*>(p.ws), p.splits, rows,
+                           p.out, p.lse, rf, rf * p.splits) != cudaSuccess)
+      return PLX_ERR_CUDA;
+    return PLX_OK;
+  }
+  // balanced plan: one combine CTA per SM (each can be resident beside the
+  // split CTAs), at most a few split CTAs' jobs each
+  const int sms = sm_count_or_default();
+  const int cgrid = std::max(std::min(P, sms), (P + 3) / 4);
+  cfg.gridDim = dim3(static_cast<unsigned>(cgrid));
+  cfg.blockDim = dim3(plx::kDecCombineThreads);
+  if (cudaLaunchKernelEx(&cfg, plx::plx_decode_combine_kernel<D>, p, P) != cudaSuccess) return PLX_ERR_CUDA;
   return PLX_OK;
 }
 
@@ -380,7 +487,7 @@ int plx_decode_paged(const void* q, const void* r, const void* kpool, const void
   if (!q || !kpool || !vpool || !block_table || !seqlens || !out) return PLX_ERR_NULL;
   if (B < 1 || Hq < 1 || Hkv < 1 || num_pages < 1 || max_pages < 1 || num_splits < 0) return PLX_ERR_SHAPE;
   if (page_size < 16 || page_size > 4096 || (page_size & (page_size - 1))) return PLX_ERR_SHAPE;
-  if (B > 65535 || static_cast<long long>(max_pages) * page_size > 0x7fffffffLL ||
+  if (static_cast<long long>(max_pages) * page_size > 0x7fffffffLL ||
       static_cast<long long>(num_pages) * Hkv > 0x7fffffffLL)
     return PLX_ERR_SHAPE;
   if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
@@ -390,15 +497,14 @@ int plx_decode_paged(const void* q, const void* r, const void* kpool, const void
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return PLX_ERR_ALIGN;
   const int S_max = max_pages * page_size;
-  const SplitPlan plan = plan_splits(B, Hq, Hkv, S_max, num_splits);
-  const size_t need = workspace_bytes_for(B, Hq, d, plan.splits);
-  if (need > 0) {
-    if (!workspace || workspace_bytes < need) return PLX_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return PLX_ERR_ALIGN;
-  }
+  const DecodePlan plan = plan_decode(B, Hq, Hkv, S_max, d, num_splits, false);
+  const int P = plan.P;
+  if (plan.ws_bytes > 0 && (!workspace || workspace_bytes < plan.ws_bytes)) return PLX_ERR_WORKSPACE;
+  if (plan.ws_bytes > 0 && !aligned16(workspace)) return PLX_ERR_ALIGN;
   const int G = Hq / Hkv;
   const int n_hg = (G + 7) / 8;
-  if (static_cast<long long>(Hkv) * n_hg > 65535) return PLX_ERR_SHAPE;
+  if (static_cast<long long>(B) * Hkv * n_hg * ((S_max + plx::kDecTileKeys - 1) / plx::kDecTileKeys) > 0x7fffffffLL)
+    return PLX_ERR_SHAPE;
   int dev = 0;
   int rc = check_arch(&dev);
   if (rc != PLX_OK) return rc;
@@ -418,7 +524,6 @@ int plx_decode_paged(const void* q, const void* r, const void* kpool, const void
   p.seqlens = seqlens;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  p.ws = static_cast<float*>(workspace);
   p.block_table = block_table;
   p.num_pages = num_pages;
   p.max_pages = max_pages;
@@ -428,11 +533,14 @@ int plx_decode_paged(const void* q, const void* r, const void* kpool, const void
   p.page_shift = shift;
   p.box_rows = box_rows;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.S_max = S_max; p.G = G; p.n_hgroups = n_hg;
-  p.splits = plan.splits; p.chunk = plan.chunk;
+  p.rps = rows_per_slot(Hq, Hkv);
+  p.ws = static_cast<float*>(workspace);
+  p.chunk_tiles = plan.chunked ? plan.chunk_tiles : 0;
+  p.splits = plan.chunked ? plan.splits : 0;
   p.scale_log2 = scale * plx::kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 128) return r ? launch_decode<128, true, true>(km, vm, p, n_hg, st) : launch_decode<128, false, true>(km, vm, p, n_hg, st);
-  return r ? launch_decode<64, true, true>(km, vm, p, n_hg, st) : launch_decode<64, false, true>(km, vm, p, n_hg, st);
+  if (d == 128) return r ? launch_decode<128, true, true>(km, vm, p, P, st) : launch_decode<128, false, true>(km, vm, p, P, st);
+  return r ? launch_decode<64, true, true>(km, vm, p, P, st) : launch_decode<64, false, true>(km, vm, p, P, st);
 }
 
 }  // extern "C"
@@ -554,45 +662,40 @@ int plx_bwd(const void* q, const void* k, const void* v, const void* r, const vo
 }
 
 int plx_decode_num_splits(int B, int Hq, int Hkv, int S_max, int d) {
-  (void)d;
-  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv) return 1;
-  return plan_splits(B, Hq, Hkv, S_max, 0).splits;
+  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128)) return decode_ctas(0);
+  return plan_decode(B, Hq, Hkv, S_max, d, 0, false).P;
 }
 
 size_t plx_decode_workspace_size(int B, int Hq, int Hkv, int S_max, int d, int num_splits) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128)) return 0;
-  return workspace_bytes_for(B, Hq, d, plan_splits(B, Hq, Hkv, S_max, num_splits).splits);
+  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128) || num_splits < 0) return 0;
+  return plan_decode(B, Hq, Hkv, S_max, d, num_splits, false).ws_bytes;
 }
 
 }  // extern "C"
 
 namespace {
 
-// plx_decode, or (partial_out) plx_decode_partial: the same validation and
-// launch; partial_out writes every split's partial state to `workspace` and
-// never runs the combine.
+// plx_decode, or (rec_out) plx_decode_partial: the same validation and
+// launches; rec_out receives one state record per (b, h) instead of out/lse.
 int decode_common(const void* q, const void* r, const void* kcache, const void* vcache, const int32_t* seqlens,
-                  void* out, float* lse, int B, int Hq, int Hkv, int S_max, int d, float scale, int num_splits,
-                  void* workspace, size_t workspace_bytes, void* stream, bool partial_out, int key_offset = 0) {
-  if (!q || !kcache || !vcache || !seqlens || (!out && !partial_out)) return PLX_ERR_NULL;
+                  void* out, float* lse, float* rec_out, int B, int Hq, int Hkv, int S_max, int d, float scale,
+                  int num_splits, void* workspace, size_t workspace_bytes, void* stream, int key_offset = 0) {
+  if (!q || !kcache || !vcache || !seqlens || (!out && !rec_out)) return PLX_ERR_NULL;
   if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || num_splits < 0) return PLX_ERR_SHAPE;
-  if (B > 65535) return PLX_ERR_SHAPE;
   if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
   if (Hq % Hkv) return PLX_ERR_GQA;
   if (!aligned16(q) || (r && !aligned16(r)) || !aligned16(kcache) || !aligned16(vcache) ||
-      (out && !aligned16(out)) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+      (out && !aligned16(out)) || (rec_out && !aligned16(rec_out)) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return PLX_ERR_ALIGN;
-  const SplitPlan plan = plan_splits(B, Hq, Hkv, S_max, num_splits);
-  const size_t need = partial_out ? static_cast<size_t>(B) * Hq * plan.splits * (2 * d + 4) * sizeof(float)
-                                  : workspace_bytes_for(B, Hq, d, plan.splits);
-  if (need > 0) {
-    if (!workspace || workspace_bytes < need) return PLX_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return PLX_ERR_ALIGN;
-  }
+  const DecodePlan plan = plan_decode(B, Hq, Hkv, S_max, d, num_splits, rec_out != nullptr);
+  const int P = plan.P;
+  if (plan.ws_bytes > 0 && (!workspace || workspace_bytes < plan.ws_bytes)) return PLX_ERR_WORKSPACE;
+  if (plan.ws_bytes > 0 && !aligned16(workspace)) return PLX_ERR_ALIGN;
   const int G = Hq / Hkv;
   const int n_hg = (G + 7) / 8;
-  if (static_cast<long long>(Hkv) * n_hg > 65535) return PLX_ERR_SHAPE;
+  if (static_cast<long long>(B) * Hkv * n_hg * ((S_max + plx::kDecTileKeys - 1) / plx::kDecTileKeys) > 0x7fffffffLL)
+    return PLX_ERR_SHAPE;
   int dev = 0;
   int rc = check_arch(&dev);
   if (rc != PLX_OK) return rc;
@@ -609,16 +712,18 @@ int decode_common(const void* q, const void* r, const void* kcache, const void* 
   p.r = static_cast<const __nv_bfloat16*>(r);
   p.seqlens = seqlens;
   p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = partial_out ? nullptr : lse;
-  p.ws = static_cast<float*>(workspace);
+  p.lse = rec_out ? nullptr : lse;
+  p.rec_out = rec_out;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.S_max = S_max; p.G = G; p.n_hgroups = n_hg;
-  p.splits = plan.splits; p.chunk = plan.chunk;
-  p.partial_out = partial_out ? 1 : 0;
+  p.rps = rows_per_slot(Hq, Hkv);
+  p.ws = static_cast<float*>(workspace);
+  p.chunk_tiles = plan.chunked ? plan.chunk_tiles : 0;
+  p.splits = plan.chunked ? plan.splits : 0;
   p.key_offset = key_offset;
   p.scale_log2 = scale * plx::kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 128) return r ? launch_decode<128, true, false>(km, vm, p, n_hg, st) : launch_decode<128, false, false>(km, vm, p, n_hg, st);
-  return r ? launch_decode<64, true, false>(km, vm, p, n_hg, st) : launch_decode<64, false, false>(km, vm, p, n_hg, st);
+  if (d == 128) return r ? launch_decode<128, true, false>(km, vm, p, P, st) : launch_decode<128, false, false>(km, vm, p, P, st);
+  return r ? launch_decode<64, true, false>(km, vm, p, P, st) : launch_decode<64, false, false>(km, vm, p, P, st);
 }
 
 }  // namespace
@@ -629,14 +734,14 @@ int plx_decode(const void* q, const void* r, const void* kcache, const void* vca
                const int32_t* seqlens, void* out, float* lse, int B, int Hq, int Hkv, int S_max,
                int d, float scale, int num_splits, void* workspace, size_t workspace_bytes,
                void* stream) {
-  return decode_common(q, r, kcache, vcache, seqlens, out, lse, B, Hq, Hkv, S_max, d, scale, num_splits,
-                       workspace, workspace_bytes, stream, false);
+  return decode_common(q, r, kcache, vcache, seqlens, out, lse, nullptr, B, Hq, Hkv, S_max, d, scale, num_splits,
+                       workspace, workspace_bytes, stream);
 }
 
 size_t plx_decode_partial_size(int B, int Hq, int Hkv, int S_max, int d, int num_splits) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128) || num_splits < 0) return 0;
-  return static_cast<size_t>(B) * Hq * plan_splits(B, Hq, Hkv, S_max, num_splits).splits * (2 * d + 4) *
-         sizeof(float);
+  return align256(static_cast<size_t>(B) * Hq * (2 * d + 4) * sizeof(float)) +
+         decode_scratch_bytes(Hq, Hkv, d, decode_ctas(num_splits));
 }
 
 int plx_decode_partial(const void* q, const void* r, const void* kcache, const void* vcache,
@@ -644,44 +749,48 @@ int plx_decode_partial(const void* q, const void* r, const void* kcache, const v
                        float scale, int num_splits, float* partial, size_t partial_bytes, void* stream) {
   if (!partial) return PLX_ERR_NULL;
   if (key_offset < 0) return PLX_ERR_SHAPE;
-  return decode_common(q, r, kcache, vcache, seqlens, nullptr, nullptr, B, Hq, Hkv, S_max, d, scale, num_splits,
-                       partial, partial_bytes, stream, true, key_offset);
+  const size_t need = plx_decode_partial_size(B, Hq, Hkv, S_max, d, num_splits);
+  if (need != 0 && partial_bytes < need) return PLX_ERR_WORKSPACE;  // bad shapes: decode_common reports them
+  const size_t rec_bytes = align256(static_cast<size_t>(B > 0 ? B : 0) * (Hq > 0 ? Hq : 0) * (2 * d + 4) * sizeof(float));
+  return decode_common(q, r, kcache, vcache, seqlens, nullptr, nullptr, partial, B, Hq, Hkv, S_max, d, scale,
+                       num_splits, reinterpret_cast<char*>(partial) + rec_bytes,
+                       partial_bytes > rec_bytes ? partial_bytes - rec_bytes : 0, stream, key_offset);
 }
 
-// out / lse of `rows` rows from `ranks` blocks of partial states, each block
-// [rows, num_splits, 2d + 4] (the split-KV combine over ranks x splits)
-static int merge_common(const float* partials, int ranks, long long rows, int d, int num_splits, void* out, float* lse,
-                        void* stream) {
-  if (!partials || !out) return PLX_ERR_NULL;
-  if (ranks < 1 || rows < 1 || num_splits < 1) return PLX_ERR_SHAPE;
+// out / lse of `rows` rows from `blocks` blocks of state records, each block
+// [rows, 2d + 4] (the merge over context-parallel ranks or key chunks)
+static int merge_common(const float* recs, int blocks, long long rows, int d, void* out, float* lse, void* stream) {
+  if (!recs || !out) return PLX_ERR_NULL;
+  if (blocks < 1 || rows < 1) return PLX_ERR_SHAPE;
   if (d != 64 && d != 128) return PLX_ERR_HEADDIM;
-  if (!aligned16(partials) || !aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+  if (!aligned16(recs) || (reinterpret_cast<uintptr_t>(out) & 7u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return PLX_ERR_ALIGN;
-  if (rows > 0x7fffffffLL) return PLX_ERR_SHAPE;
+  const long long threads = rows * (d / 4);
+  if ((threads + 255) / 256 > 0x7fffffffLL) return PLX_ERR_SHAPE;
   int dev = 0;
   int rc = check_arch(&dev);
   if (rc != PLX_OK) return rc;
-  const size_t rank_stride = static_cast<size_t>(rows) * num_splits * (2 * d + 4);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
+  const long long rf = 2 * d + 4;
   if (d == 128)
-    plx::plx_decode_combine_kernel<128><<<static_cast<unsigned>(rows), 128, 0, st>>>(
-        partials, static_cast<__nv_bfloat16*>(out), lse, num_splits, ranks, rank_stride);
+    plx::plx_record_merge_kernel<128><<<grid, 256, 0, st>>>(recs, blocks, rows, static_cast<__nv_bfloat16*>(out), lse,
+                                                           rows * rf, rf);
   else
-    plx::plx_decode_combine_kernel<64><<<static_cast<unsigned>(rows), 64, 0, st>>>(
-        partials, static_cast<__nv_bfloat16*>(out), lse, num_splits, ranks, rank_stride);
+    plx::plx_record_merge_kernel<64><<<grid, 256, 0, st>>>(recs, blocks, rows, static_cast<__nv_bfloat16*>(out), lse,
+                                                          rows * rf, rf);
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
-int plx_decode_merge(const float* partials, int ranks, int B, int Hq, int d, int num_splits, void* out, float* lse,
-                     void* stream) {
+int plx_decode_merge(const float* partials, int ranks, int B, int Hq, int d, void* out, float* lse, void* stream) {
   if (B < 1 || Hq < 1) return (!partials || !out) ? PLX_ERR_NULL : PLX_ERR_SHAPE;
-  return merge_common(partials, ranks, static_cast<long long>(B) * Hq, d, num_splits, out, lse, stream);
+  return merge_common(partials, ranks, static_cast<long long>(B) * Hq, d, out, lse, stream);
 }
 
 int plx_fwd_merge(const float* partials, int ranks, int B, int Hq, int N, int d, void* out, float* lse,
                   void* stream) {
   if (B < 1 || Hq < 1 || N < 1) return (!partials || !out) ? PLX_ERR_NULL : PLX_ERR_SHAPE;
-  return merge_common(partials, ranks, static_cast<long long>(B) * Hq * N, d, 1, out, lse, stream);
+  return merge_common(partials, ranks, static_cast<long long>(B) * Hq * N, d, out, lse, stream);
 }
 
 int plx_check_device_status(void* stream) {
@@ -758,3 +867,125 @@ extern "C" int plx_decode_noalloc(const void* q, const void* r, const void* kcac
   return plx_decode(q, r, kcache, vcache, seqlens, out, lse, B, Hq, Hkv, S_max, d, scale, num_splits,
                     scratch, PLX_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+// ------------------------------------------------------------------ q, k, v, rho projection
+namespace {
+
+int proj_common(const void* x, const void* w, plx::ProjParams& p, int M, int d_model, void* stream) {
+  if (!x || !w) return PLX_ERR_NULL;
+  if (M < 1 || d_model < 8 || d_model % 8 || p.Hq < 1 || p.Hkv < 1) return PLX_ERR_SHAPE;
+  if (p.d != 64 && p.d != 128) return PLX_ERR_HEADDIM;
+  if (p.Hq % p.Hkv) return PLX_ERR_GQA;
+  if (!aligned16(x) || !aligned16(w)) return PLX_ERR_ALIGN;
+  const long long nout = static_cast<long long>(2 * p.Hkv + (p.r ? 2 : 1) * p.Hq) * p.d;
+  const long long m_tiles = (M + plx::kPjBM - 1) / plx::kPjBM;
+  long long n_tiles = (nout + 63) / 64;
+  if (m_tiles * n_tiles > 0x7fffffffLL || static_cast<long long>(M) * nout > (1LL << 40)) return PLX_ERR_SHAPE;
+  int dev = 0;
+  int rc = check_arch(&dev);
+  if (rc != PLX_OK) return rc;
+  if ((rc = get_encoder()) != PLX_OK) return rc;
+  // few rows (a decode step): narrow tiles, so that more CTAs share the weight stream
+  const bool narrow = M <= plx::kPjBM;
+  const int bn = narrow ? 64 : 256;
+  n_tiles = (nout + bn - 1) / bn;
+  CUtensorMap xm, wm;
+  if (make_map_2d(&xm, x, d_model, M, plx::kPjBM) != PLX_OK || make_map_2d(&wm, w, d_model, nout, bn) != PLX_OK)
+    return PLX_ERR_CUDA;
+  p.M = M;
+  p.K = d_model;
+  p.Nout = static_cast<int>(nout);
+  p.m_tiles = static_cast<int>(m_tiles);
+  p.n_tiles = static_cast<int>(n_tiles);
+  p.num_tiles = static_cast<int>(m_tiles * n_tiles);
+  p.k_steps = (d_model + plx::kPjBK - 1) / plx::kPjBK;
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(p.num_tiles, g_sm_count[dev]));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (narrow) {
+    static bool done[kMaxDevices];
+    auto kern = plx::plx_proj_kernel<64>;
+    if (ensure_smem(kern, plx::ProjCfg<64>::kSmemBytes, &done[dev]) != PLX_OK) return PLX_ERR_CUDA;
+    kern<<<grid, plx::kPjThreads, plx::ProjCfg<64>::kSmemBytes, st>>>(xm, wm, p);
+  } else {
+    static bool done[kMaxDevices];
+    auto kern = plx::plx_proj_kernel<256>;
+    if (ensure_smem(kern, plx::ProjCfg<256>::kSmemBytes, &done[dev]) != PLX_OK) return PLX_ERR_CUDA;
+    kern<<<grid, plx::kPjThreads, plx::ProjCfg<256>::kSmemBytes, st>>>(xm, wm, p);
+  }
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int plx_qkvr_proj(const void* x, const void* w, void* q, void* k, void* v, void* r, int B, int N, int d_model,
+                  int Hq, int Hkv, int d, void* stream) {
+  if (!q || !k || !v) return PLX_ERR_NULL;
+  if (B < 1 || N < 1) return PLX_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (r && !aligned16(r))) return PLX_ERR_ALIGN;
+  if (static_cast<long long>(B) * N > 0x7fffffffLL) return PLX_ERR_SHAPE;
+  plx::ProjParams p{};
+  p.q = static_cast<__nv_bfloat16*>(q);
+  p.k = static_cast<__nv_bfloat16*>(k);
+  p.v = static_cast<__nv_bfloat16*>(v);
+  p.r = static_cast<__nv_bfloat16*>(r);
+  p.N = N; p.Hq = Hq; p.Hkv = Hkv; p.d = d;
+  return proj_common(x, w, p, B * N, d_model, stream);
+}
+
+int plx_qkvr_proj_decode(const void* x, const void* w, void* q, void* r, void* kcache, void* vcache,
+                         const int32_t* seqlens, int32_t* seqlens_out, int B, int d_model, int Hq, int Hkv,
+                         int S_max, int d, void* stream) {
+  if (!q || !kcache || !vcache || !seqlens) return PLX_ERR_NULL;
+  if (B < 1 || S_max < 1) return PLX_ERR_SHAPE;
+  if (seqlens_out && static_cast<const void*>(seqlens_out) == static_cast<const void*>(seqlens)) return PLX_ERR_SHAPE;
+  if (!aligned16(q) || (r && !aligned16(r)) || !aligned16(kcache) || !aligned16(vcache) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(seqlens_out) & 3u))
+    return PLX_ERR_ALIGN;
+  plx::ProjParams p{};
+  p.q = static_cast<__nv_bfloat16*>(q);
+  p.r = static_cast<__nv_bfloat16*>(r);
+  p.decode = 1;
+  p.kcache = static_cast<__nv_bfloat16*>(kcache);
+  p.vcache = static_cast<__nv_bfloat16*>(vcache);
+  p.S_max = S_max;
+  p.seqlens = seqlens;
+  p.seqlens_out = seqlens_out;
+  p.N = 1; p.Hq = Hq; p.Hkv = Hkv; p.d = d;
+  return proj_common(x, w, p, B, d_model, stream);
+}
+
+int plx_qkvr_proj_decode_paged(const void* x, const void* w, void* q, void* r, void* kpool, void* vpool,
+                               const int32_t* block_table, const int32_t* seqlens, int32_t* seqlens_out, int B,
+                               int d_model, int Hq, int Hkv, int num_pages, int page_size, int max_pages, int d,
+                               void* stream) {
+  if (!q || !kpool || !vpool || !seqlens || !block_table) return PLX_ERR_NULL;
+  if (B < 1 || num_pages < 1 || max_pages < 1) return PLX_ERR_SHAPE;
+  if (page_size < 16 || page_size > 4096 || (page_size & (page_size - 1))) return PLX_ERR_SHAPE;
+  if (static_cast<long long>(max_pages) * page_size > 0x7fffffffLL) return PLX_ERR_SHAPE;
+  if (seqlens_out && static_cast<const void*>(seqlens_out) == static_cast<const void*>(seqlens)) return PLX_ERR_SHAPE;
+  if (!aligned16(q) || (r && !aligned16(r)) || !aligned16(kpool) || !aligned16(vpool) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(seqlens_out) & 3u) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u))
+    return PLX_ERR_ALIGN;
+  plx::ProjParams p{};
+  p.q = static_cast<__nv_bfloat16*>(q);
+  p.r = static_cast<__nv_bfloat16*>(r);
+  p.decode = 1;
+  p.kcache = static_cast<__nv_bfloat16*>(kpool);
+  p.vcache = static_cast<__nv_bfloat16*>(vpool);
+  p.seqlens = seqlens;
+  p.seqlens_out = seqlens_out;
+  p.block_table = block_table;
+  p.num_pages = num_pages;
+  p.page_size = page_size;
+  int shift = 0;
+  while ((1 << shift) < page_size) ++shift;
+  p.page_shift = shift;
+  p.max_pages = max_pages;
+  p.N = 1; p.Hq = Hq; p.Hkv = Hkv; p.d = d;
+  return proj_common(x, w, p, B, d_model, stream);
+}
+
+}  // extern "C"

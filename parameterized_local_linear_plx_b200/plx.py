@@ -10,6 +10,7 @@ no fallback implementation.
 from __future__ import annotations
 
 import ctypes
+import functools
 import math
 import os
 
@@ -59,12 +60,18 @@ _lib.plx_kv_append.restype = _I
 _lib.plx_kv_append.argtypes = [_P] * 5 + [_I] * 5 + [_P]
 _lib.plx_kv_append_paged.restype = _I
 _lib.plx_kv_append_paged.argtypes = [_P] * 6 + [_I] * 7 + [_P]
+_lib.plx_qkvr_proj.restype = _I
+_lib.plx_qkvr_proj.argtypes = [_P] * 6 + [_I] * 6 + [_P]
+_lib.plx_qkvr_proj_decode.restype = _I
+_lib.plx_qkvr_proj_decode.argtypes = [_P] * 8 + [_I] * 6 + [_P]
+_lib.plx_qkvr_proj_decode_paged.restype = _I
+_lib.plx_qkvr_proj_decode_paged.argtypes = [_P] * 9 + [_I] * 8 + [_P]
 _lib.plx_decode_partial_size.restype = _SZ
 _lib.plx_decode_partial_size.argtypes = [_I] * 6
 _lib.plx_decode_partial.restype = _I
 _lib.plx_decode_partial.argtypes = [_P] * 5 + [_I] * 6 + [_F, _I, _P, _SZ, _P]
 _lib.plx_decode_merge.restype = _I
-_lib.plx_decode_merge.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P]
+_lib.plx_decode_merge.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P]
 _lib.plx_decode_noalloc.restype = _I
 _lib.plx_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]
 _lib.plx_check_device_status.restype = _I
@@ -296,7 +303,14 @@ def plx_bwd(q, k, v, r, out, dout, lse, obar, sbar=None, causal=True, scale=None
 
 
 def plx_decode_num_splits(B, Hq, Hkv, S_max, d) -> int:
+    """The number of work partitions (persistent CTAs) plx_decode uses with num_splits = 0."""
     return _lib.plx_decode_num_splits(B, Hq, Hkv, S_max, d)
+
+
+@functools.lru_cache(maxsize=256)
+def _decode_ws_size(B, Hq, Hkv, S_max, d, num_splits, dev):
+    # cached per shape so that a steady decode loop makes one library call per step
+    return int(_lib.plx_decode_workspace_size(B, Hq, Hkv, S_max, d, num_splits))
 
 
 def plx_decode_workspace_size(B, Hq, Hkv, S_max, d, num_splits=0) -> int:
@@ -325,10 +339,10 @@ def plx_decode(q, kcache, vcache, seqlens, r=None, scale=None, num_splits=0, out
         out = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
-    need = plx_decode_workspace_size(B, Hq, Hkv, S_max, d, num_splits)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if workspace is None:
+        need = _decode_ws_size(B, Hq, Hkv, S_max, d, int(num_splits), q.device.index)
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    ws_bytes = workspace.numel() * workspace.element_size()
     st = _lib.plx_decode(_ptr(q), _ptr(r), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(out), _ptr(lse),
                          B, Hq, Hkv, S_max, d, float(scale), int(num_splits), _ptr(workspace), ws_bytes,
                          _stream(stream))
@@ -361,10 +375,10 @@ def plx_decode_paged(q, kpool, vpool, block_table, seqlens, r=None, scale=None, 
         out = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
-    need = plx_decode_workspace_size(B, Hq, Hkv, max_pages * page_size, d, num_splits)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if workspace is None:
+        need = _decode_ws_size(B, Hq, Hkv, max_pages * page_size, d, int(num_splits), q.device.index)
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    ws_bytes = workspace.numel() * workspace.element_size()
     st = _lib.plx_decode_paged(_ptr(q), _ptr(r), _ptr(kpool), _ptr(vpool), _ptr(block_table), _ptr(seqlens),
                                _ptr(out), _ptr(lse), B, Hq, Hkv, num_pages, page_size, max_pages, d, float(scale),
                                int(num_splits), _ptr(workspace), ws_bytes, _stream(stream))
@@ -413,15 +427,104 @@ def plx_kv_append_paged(knew, vnew, kpool, vpool, block_table, seqlens, advance=
         raise PlxError(st, "plx_kv_append_paged")
 
 
+def _proj_shapes(x, w, Hq, Hkv, d, with_r):
+    _check(x, "x", torch.bfloat16, 2)
+    _check(w, "w", torch.bfloat16, 2)
+    nout = (2 * Hkv + (2 if with_r else 1) * Hq) * d
+    if w.shape != (nout, x.shape[1]):
+        raise ValueError(f"w must be [{nout}, {x.shape[1]}] ([W_Q; W_K; W_V{'; W_R' if with_r else ''}]), "
+                         f"got {tuple(w.shape)}")
+
+
+def plx_qkvr_proj(x, w, B, N, Hq, Hkv, d, with_r=True, q=None, k=None, v=None, r=None, stream=None):
+    """q, k, v, rho of every token from one GEMM: x [B*N, d_model] bf16 (token
+    m = b*N + t), w = [W_Q; W_K; W_V; W_R] [Nout, d_model] bf16.  Returns
+    (q [B, Hq, N, d], k [B, Hkv, N, d], v, r [B, Hq, N, d] or None)."""
+    _proj_shapes(x, w, Hq, Hkv, d, with_r)
+    if x.shape[0] != B * N:
+        raise ValueError("x must have B * N rows")
+    dev = x.device
+    q = torch.empty((B, Hq, N, d), device=dev, dtype=torch.bfloat16) if q is None else q
+    k = torch.empty((B, Hkv, N, d), device=dev, dtype=torch.bfloat16) if k is None else k
+    v = torch.empty((B, Hkv, N, d), device=dev, dtype=torch.bfloat16) if v is None else v
+    if with_r and r is None:
+        r = torch.empty((B, Hq, N, d), device=dev, dtype=torch.bfloat16)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")) + (((r, "r"),) if with_r else ()):
+        _check(t, n, torch.bfloat16, 4)
+    st = _lib.plx_qkvr_proj(_ptr(x), _ptr(w), _ptr(q), _ptr(k), _ptr(v), _ptr(r if with_r else None), B, N,
+                            x.shape[1], Hq, Hkv, d, _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_qkvr_proj")
+    return q, k, v, (r if with_r else None)
+
+
+def plx_qkvr_proj_decode(x, w, kcache, vcache, seqlens, Hq, with_r=True, seqlens_out=None, q=None, r=None,
+                         stream=None):
+    """One decode step's projection with the KV append fused in: x [B, d_model]
+    bf16 (each sequence's new token); k, v go into kcache / vcache
+    [B, Hkv, S_max, d] at row seqlens[b].  Returns (q [B, Hq, d], r or None,
+    seqlens_out [B] int32 = seqlens + 1 where the token was written)."""
+    _check(kcache, "kcache", torch.bfloat16, 4)
+    _check(vcache, "vcache", torch.bfloat16, 4)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    B = x.shape[0]
+    Hkv, S_max, d = kcache.shape[1], kcache.shape[2], kcache.shape[3]
+    _proj_shapes(x, w, Hq, Hkv, d, with_r)
+    if kcache.shape[0] != B or vcache.shape != kcache.shape or seqlens.shape != (B,):
+        raise ValueError("shape mismatch between x, caches, seqlens")
+    dev = x.device
+    q = torch.empty((B, Hq, d), device=dev, dtype=torch.bfloat16) if q is None else q
+    if with_r and r is None:
+        r = torch.empty((B, Hq, d), device=dev, dtype=torch.bfloat16)
+    if seqlens_out is None:
+        seqlens_out = torch.empty_like(seqlens)
+    st = _lib.plx_qkvr_proj_decode(_ptr(x), _ptr(w), _ptr(q), _ptr(r if with_r else None), _ptr(kcache),
+                                   _ptr(vcache), _ptr(seqlens), _ptr(seqlens_out), B, x.shape[1], Hq, Hkv, S_max, d,
+                                   _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_qkvr_proj_decode")
+    return q, (r if with_r else None), seqlens_out
+
+
+def plx_qkvr_proj_decode_paged(x, w, kpool, vpool, block_table, seqlens, Hq, with_r=True, seqlens_out=None, q=None,
+                               r=None, stream=None):
+    """plx_qkvr_proj_decode for page pools [num_pages, Hkv, page_size, d] and a
+    block table [B, max_pages] int32."""
+    _check(kpool, "kpool", torch.bfloat16, 4)
+    _check(vpool, "vpool", torch.bfloat16, 4)
+    _check(block_table, "block_table", torch.int32, 2)
+    _check(seqlens, "seqlens", torch.int32, 1)
+    B = x.shape[0]
+    num_pages, Hkv, page_size, d = kpool.shape
+    _proj_shapes(x, w, Hq, Hkv, d, with_r)
+    if vpool.shape != kpool.shape or block_table.shape[0] != B or seqlens.shape != (B,):
+        raise ValueError("shape mismatch between x, pools, block_table, seqlens")
+    dev = x.device
+    q = torch.empty((B, Hq, d), device=dev, dtype=torch.bfloat16) if q is None else q
+    if with_r and r is None:
+        r = torch.empty((B, Hq, d), device=dev, dtype=torch.bfloat16)
+    if seqlens_out is None:
+        seqlens_out = torch.empty_like(seqlens)
+    st = _lib.plx_qkvr_proj_decode_paged(_ptr(x), _ptr(w), _ptr(q), _ptr(r if with_r else None), _ptr(kpool),
+                                         _ptr(vpool), _ptr(block_table), _ptr(seqlens), _ptr(seqlens_out), B,
+                                         x.shape[1], Hq, Hkv, num_pages, page_size, block_table.shape[1], d,
+                                         _stream(stream))
+    if st != PLX_OK:
+        raise PlxError(st, "plx_qkvr_proj_decode_paged")
+    return q, (r if with_r else None), seqlens_out
+
+
 def plx_decode_partial_size(B, Hq, Hkv, S_max, d, num_splits=0) -> int:
     return int(_lib.plx_decode_partial_size(B, Hq, Hkv, S_max, d, num_splits))
 
 
 def plx_decode_partial(q, kcache, vcache, seqlens, r=None, key_offset=0, scale=None, num_splits=0, partial=None,
                        stream=None):
-    """Partial states of a slice of the keys (keys key_offset .. key_offset + S_max - 1
-    of each sequence; seqlens are the full lengths): fp32 [B, Hq, splits, 2d + 4]
-    (m in log2 units, l, c, pad, O1[d], O2[d])."""
+    """The state record of a slice of the keys (keys key_offset .. key_offset + S_max - 1
+    of each sequence; seqlens are the full lengths) per (b, h): fp32 [B, Hq, 2d + 4]
+    (m in log2 units, l, c, pad, O1[d], O2[d]).  The records are the head of a
+    buffer of plx_decode_partial_size bytes whose tail is the kernels' scratch;
+    `partial` may be a record view returned by an earlier call (its buffer is reused)."""
     _check(q, "q", torch.bfloat16, 3)
     _check(kcache, "kcache", torch.bfloat16, 4)
     _check(vcache, "vcache", torch.bfloat16, 4)
@@ -434,29 +537,32 @@ def plx_decode_partial(q, kcache, vcache, seqlens, r=None, key_offset=0, scale=N
         raise ValueError("shape mismatch between q, caches, seqlens")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    # the split count the kernel uses (a requested count is rounded to whole 64-key chunks)
-    splits = plx_decode_partial_size(B, Hq, Hkv, S_max, d, num_splits) // (B * Hq * (2 * d + 4) * 4)
+    need = plx_decode_partial_size(B, Hq, Hkv, S_max, d, num_splits)
     if partial is None:
-        partial = torch.empty((B, Hq, splits, 2 * d + 4), device=q.device, dtype=torch.float32)
+        buf = torch.empty((need + 3) // 4, device=q.device, dtype=torch.float32)
+        partial = buf[:B * Hq * (2 * d + 4)].view(B, Hq, 2 * d + 4)
+    else:
+        _check(partial, "partial", torch.float32, 3)
+        if partial.shape != (B, Hq, 2 * d + 4):
+            raise ValueError("partial must be [B, Hq, 2d + 4]")
+    avail = partial.untyped_storage().nbytes() - partial.storage_offset() * 4
     st = _lib.plx_decode_partial(_ptr(q), _ptr(r), _ptr(kcache), _ptr(vcache), _ptr(seqlens), int(key_offset), B, Hq,
-                                 Hkv, S_max, d,
-                                 float(scale), int(num_splits), _ptr(partial),
-                                 partial.numel() * partial.element_size(), _stream(stream))
+                                 Hkv, S_max, d, float(scale), int(num_splits), _ptr(partial), avail, _stream(stream))
     if st != PLX_OK:
         raise PlxError(st, "plx_decode_partial")
     return partial
 
 
 def plx_decode_merge(partials, out=None, lse=None, return_lse=True, stream=None):
-    """Merge gathered partials [ranks, B, Hq, splits, 2d + 4] into (out, lse)."""
-    _check(partials, "partials", torch.float32, 5)
-    ranks, B, Hq, splits, pf = partials.shape
+    """Merge gathered state records [ranks, B, Hq, 2d + 4] into (out, lse)."""
+    _check(partials, "partials", torch.float32, 4)
+    ranks, B, Hq, pf = partials.shape
     d = (pf - 4) // 2
     if out is None:
         out = torch.empty((B, Hq, d), device=partials.device, dtype=torch.bfloat16)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), device=partials.device, dtype=torch.float32)
-    st = _lib.plx_decode_merge(_ptr(partials), ranks, B, Hq, d, splits, _ptr(out), _ptr(lse), _stream(stream))
+    st = _lib.plx_decode_merge(_ptr(partials), ranks, B, Hq, d, _ptr(out), _ptr(lse), _stream(stream))
     if st != PLX_OK:
         raise PlxError(st, "plx_decode_merge")
     return out, lse

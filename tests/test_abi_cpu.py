@@ -98,7 +98,7 @@ def test_decode_argument_errors(plx):
     assert dec(plx, Hq=5, Hkv=2) == plx.PLX_ERR_GQA
     assert dec(plx, vc=A + 4) == plx.PLX_ERR_ALIGN
     assert dec(plx, sl=A + 2) == plx.PLX_ERR_ALIGN
-    # two splits need a workspace
+    # every call needs the workspace (partial states of the partitions)
     assert dec(plx, S=256, splits=2) == plx.PLX_ERR_WORKSPACE
     need = plx.plx_decode_workspace_size(1, 2, 1, 256, 64, 2)
     assert dec(plx, S=256, splits=2, ws=A, wsb=need - 1) == plx.PLX_ERR_WORKSPACE
@@ -106,19 +106,35 @@ def test_decode_argument_errors(plx):
 
 
 def test_split_planning(plx):
-    # one split needs no workspace
-    assert plx.plx_decode_workspace_size(4, 16, 8, 1000, 128, 1) == 0
-    # explicit count: (2d + 4) floats per (b, h, split)
-    assert plx.plx_decode_workspace_size(2, 4, 2, 1024, 128, 4) == 2 * 4 * 4 * (2 * 128 + 4) * 4
-    # the automatic count is at least one and never gives chunks below 128 keys
-    for B, S in [(1, 128), (1, 4096), (16, 4096), (64, 4096), (2048, 16384)]:
-        n = plx.plx_decode_num_splits(B, 16, 8, S, 128)
-        assert 1 <= n <= max(1, (S + 127) // 128)
-    assert plx.plx_decode_num_splits(1, 16, 8, 4096, 128) > 1
-    assert plx.plx_decode_num_splits(2048, 16, 8, 16384, 128) == 1
-    # bad shapes: count 1, size 0
-    assert plx.plx_decode_num_splits(0, 16, 8, 4096, 128) == 1
+    # P partitions (persistent CTAs): two partial slots of min(G, 8) rows of
+    # (2d + 4) floats per partition, padded to 256 bytes; B and S_max do not enter
+    up = lambda n: (n + 255) // 256 * 256
+    for (Hq, Hkv, d, P) in [(4, 2, 128, 4), (16, 8, 128, 296), (8, 2, 64, 7), (16, 1, 128, 3)]:
+        want = up(2 * P * min(Hq // Hkv, 8) * (2 * d + 4) * 4)
+        assert plx.plx_decode_workspace_size(2, Hq, Hkv, 1024, d, P) == want
+        assert plx.plx_decode_workspace_size(64, Hq, Hkv, 32768, d, P) == want
+    # automatic plan, few segments (b, kv head): two balanced partitions per SM
+    n = plx.plx_decode_num_splits(1, 16, 8, 4096, 128)
+    assert n >= 2 and n % 2 == 0
+    assert plx.plx_decode_num_splits(8, 16, 8, 32768, 128) == n  # 64 segments
+    assert plx.plx_decode_workspace_size(1, 16, 8, 4096, 128, 0) == plx.plx_decode_workspace_size(1, 16, 8, 4096, 128, n)
+    # automatic plan, many segments: chunks of whole 64-key tiles, about four
+    # waves of two CTAs per SM, chunks of at least 128 keys; one record of
+    # (2d + 4) floats per (b, h, chunk) when a segment has several chunks
+    sms = n // 2
+    for B, S in [(64, 4096), (256, 1024), (2048, 16384), (1024, 512)]:
+        segs = B * 8
+        sp = max(1, min(-(-4 * 2 * sms // segs), (S + 127) // 128))
+        tiles = -(-(-(-S // sp)) // 64)
+        splits = -(-S // (tiles * 64))
+        assert plx.plx_decode_num_splits(B, 16, 8, S, 128) == segs * splits
+        assert plx.plx_decode_workspace_size(B, 16, 8, S, 128, 0) == (up(B * 16 * splits * 260 * 4) if splits > 1 else 0)
+    assert plx.plx_decode_num_splits(2048, 16, 8, 16384, 128) == 2048 * 8  # one chunk per segment: no workspace
+    # short segments keep the balanced plan whatever their number
+    assert plx.plx_decode_num_splits(2048, 16, 8, 256, 128) == n
+    # bad shapes: size 0
     assert plx.plx_decode_workspace_size(1, 3, 2, 128, 128, 2) == 0
+    assert plx.plx_decode_workspace_size(1, 2, 1, 128, 128, -1) == 0
 
 
 def fwdt(plx, q=A, k=A, v=A, r=A, out=A, lse=A, obar=A, sbar=A, B=1, Hq=2, Hkv=1, N=8, d=64):
@@ -221,18 +237,21 @@ def test_partial_and_merge_argument_errors(plx):
     dp = plx.lib.plx_decode_partial
     ok = lambda **kw: [P(kw.get(n, A)) for n in ("q", "r", "kc", "vc", "sl")]
     need = plx.plx_decode_partial_size(1, 2, 1, 64, 64, 1)
-    assert need == 1 * 2 * 1 * (2 * 64 + 4) * 4
+    # the records [B, Hq, 2d + 4] fp32, then the workspace of one partition
+    up = lambda n: (n + 255) // 256 * 256
+    assert need == up(1 * 2 * (2 * 64 + 4) * 4) + plx.plx_decode_workspace_size(1, 2, 1, 64, 64, 1)
     assert dp(*ok(), 0, 1, 2, 1, 64, 64, 0.125, 1, P(None), need, None) == plx.PLX_ERR_NULL
     assert dp(*ok(), -1, 1, 2, 1, 64, 64, 0.125, 1, P(A), need, None) == plx.PLX_ERR_SHAPE
     assert dp(*ok(), 0, 1, 2, 1, 64, 64, 0.125, 1, P(A), need - 4, None) == plx.PLX_ERR_WORKSPACE
     assert dp(*ok(kc=None), 0, 1, 2, 1, 64, 64, 0.125, 1, P(A), need, None) == plx.PLX_ERR_NULL
     assert dp(*ok(), 0, 1, 2, 1, 64, 96, 0.125, 1, P(A), need, None) == plx.PLX_ERR_HEADDIM
     mg = plx.lib.plx_decode_merge
-    assert mg(P(None), 2, 1, 2, 64, 1, P(A), P(A), None) == plx.PLX_ERR_NULL
-    assert mg(P(A), 0, 1, 2, 64, 1, P(A), P(A), None) == plx.PLX_ERR_SHAPE
-    assert mg(P(A), 2, 1, 2, 64, 0, P(A), P(A), None) == plx.PLX_ERR_SHAPE
-    assert mg(P(A), 2, 1, 2, 80, 1, P(A), P(A), None) == plx.PLX_ERR_HEADDIM
-    assert mg(P(A + 4), 2, 1, 2, 64, 1, P(A), P(A), None) == plx.PLX_ERR_ALIGN
+    assert mg(P(None), 2, 1, 2, 64, P(A), P(A), None) == plx.PLX_ERR_NULL
+    assert mg(P(A), 0, 1, 2, 64, P(A), P(A), None) == plx.PLX_ERR_SHAPE
+    assert mg(P(A), 2, 0, 2, 64, P(A), P(A), None) == plx.PLX_ERR_SHAPE
+    assert mg(P(A), 2, 1, 2, 80, P(A), P(A), None) == plx.PLX_ERR_HEADDIM
+    assert mg(P(A + 4), 2, 1, 2, 64, P(A), P(A), None) == plx.PLX_ERR_ALIGN
+    assert mg(P(A), 2, 1, 2, 64, P(A + 4), P(A), None) == plx.PLX_ERR_ALIGN
 
 
 def test_prefill_partial_and_merge_argument_errors(plx):

@@ -33,12 +33,12 @@ def _worker(rank, world, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         from parameterized_local_linear_plx_b200 import cp
-        B, Hq, splits, d = 3, 4, 2, 8
-        # a rank's partial block, filled with values that name the rank and the position
-        part = torch.arange(B * Hq * splits * (2 * d + 4), dtype=torch.float32).reshape(B, Hq, splits, 2 * d + 4)
+        B, Hq, d = 3, 4, 8
+        # a rank's state records, filled with values that name the rank and the position
+        part = torch.arange(B * Hq * (2 * d + 4), dtype=torch.float32).reshape(B, Hq, 2 * d + 4)
         part = part + 1000.0 * rank
         g = cp.gather_partials(part)
-        q.put((rank, tuple(g.shape), [float(g[i, 0, 0, 0, 0]) for i in range(world)],
+        q.put((rank, tuple(g.shape), [float(g[i, 0, 0, 0]) for i in range(world)],
                cp.slice_start(rank, 512)))
     finally:
         dist.destroy_process_group()
@@ -55,7 +55,7 @@ def test_two_gloo_ranks_gather_rank_major():
         p.join(timeout=120)
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
     res = sorted(q.get(timeout=5) for _ in range(2))
-    assert res == [(0, (2, 3, 4, 2, 20), [0.0, 1000.0], 0), (1, (2, 3, 4, 2, 20), [0.0, 1000.0], 512)]
+    assert res == [(0, (2, 3, 4, 20), [0.0, 1000.0], 0), (1, (2, 3, 4, 20), [0.0, 1000.0], 512)]
 
 
 def _worker_prefill(rank, world, port, q):

@@ -1,4 +1,5 @@
-"""Decode (split-KV) on the GPU against the fp64 oracle, through the C ABI."""
+"""Decode (split-KV, balanced over the key tiles of the batch) on the GPU
+against the fp64 oracle, through the C ABI."""
 import numpy as np
 import pytest
 import torch
@@ -76,6 +77,44 @@ def test_decode_split_invariance(plx):
         assert_close(o, ro, l, rl, f"splits={s}")
         # different splits differ only by rounding
         assert (o.float() - ref_o.float()).abs().max().item() <= 1e-2
+
+
+@pytest.mark.parametrize("splits", [1, 3, 5, 11, 0])
+def test_decode_partitions_cross_sequences_and_head_groups(plx, splits):
+    """The work partitions cut the tile list of the whole batch anywhere: in
+    the middle of a sequence, of a head group (G = 12: groups of 8 and 4 query
+    heads per KV head), next to empty sequences.  Every cut must merge back to
+    the oracle's result."""
+    lens = [0, 5, 0, 0, 300, 64, 0, 129, 1, 0]
+    o, l, ro, rl = run(plx, len(lens), 24, 2, 320, 64, seqlens=lens, seed=40 + splits, splits=splits)
+    assert_close(o, ro, l, rl, f"partitions={splits}")
+    o, l, ro, rl = run(plx, len(lens), 24, 2, 320, 128, seqlens=lens, seed=50 + splits, splits=splits)
+    assert_close(o, ro, l, rl, f"partitions={splits} d=128")
+
+
+@pytest.mark.parametrize("B,S,d", [(40, 1000, 128), (300, 200, 128), (48, 700, 64)])
+def test_decode_many_segments(plx, B, S, d):
+    """Batches with 128 (b, kv head) segments or more: of more than 256 keys
+    they take the chunked plan (a CTA per chunk of a segment, chunk records
+    merged per row), shorter ones the balanced plan; ragged lengths with empty
+    sequences among them; sampled batch entries."""
+    q, kc, vc, r, _ = inputs.decode_inputs(B, 16, 8, S, d, seed=60 + B, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(61)
+    sl = torch.randint(0, S + 1, (B,), generator=g, device="cuda", dtype=torch.int32)
+    sl[::7] = 0
+    sl[1] = S
+    out, lse = plx.plx_decode(q, kc, vc, sl, r)
+    torch.cuda.synchronize()
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    chunked = plx.plx_decode_num_splits(B, 16, 8, S, d) >= B * 8
+    assert chunked == (S > 256)
+    pick = sorted({0, 1, 2, 7, B // 2, B - 1})
+    qc, kcc, vcc, rc, slc = (t[pick].cpu() for t in (q, kc, vc, r, sl))
+    ro, rl = oracle.decode_effective(qc, rc, kcc, vcc, slc)
+    assert_close(out[pick], ro, lse[pick], rl, f"chunked B={B} S={S} d={d}")
+    # the balanced plan (explicit partition count) gives the same result up to rounding
+    o2, l2 = plx.plx_decode(q, kc, vc, sl, r, num_splits=296)
+    assert (o2.float() - out.float()).abs().max().item() <= 1e-2
 
 
 def test_decode_r_none_equals_r_zero_and_softmax(plx):

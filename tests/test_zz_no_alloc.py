@@ -66,8 +66,8 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row(plx):
 
 
 def test_noalloc_rejects_requests_above_its_scratch(plx):
-    # B=64, 1024 splits of 64 keys: the partials would need ~1.1 GB > 16 MiB
-    B, Hq, Hkv, S, d, splits = 64, 16, 8, 65536, 128, 1024
+    # 8192 work partitions: their partial-state slots would need ~34 MB > 16 MiB
+    B, Hq, Hkv, S, d, splits = 64, 16, 8, 65536, 128, 8192
     need = plx.plx_decode_workspace_size(B, Hq, Hkv, S, d, splits)
     assert need > plx.PLX_NOALLOC_SCRATCH_BYTES
     P = ctypes.c_void_p
