@@ -415,10 +415,13 @@ def run_gpu(args, world, rank, local):
     pre_achieved = p_flops / (pre_avg * 1e-3) / 1e12
     roof_dec = {"bound": "hbm", "achieved": dec_achieved, "peak": hbm, "unit": "GB/s",
                 "frac": dec_achieved / hbm, "traffic": load_traffic("decode"),
+                "traffic_note": "scaled x4 from a B=16 ncu capture of the decode kernel",
                 "kernel": "plx_decode (split + combine), per call",
                 "peak_source": f"{peak_src} hbm_gbs"}
     roof_pre = {"bound": "tensor", "achieved": pre_achieved, "peak": tf_peak, "unit": "TFLOP/s",
                 "frac": pre_achieved / tf_peak, "traffic": load_traffic("prefill"),
+                "traffic_note": "scaled x4 from a B=2 ncu capture; a lower bound (the last writes are still "
+                                "in L2 when the capture ends)",
                 "kernel": "plx_fwd_kernel<128,true>", "peak_source": f"{peak_src} {tf_key}"}
 
     # ---- end to end through the public API: pinned host buffers, copies timed
@@ -612,6 +615,38 @@ def run_cp_prefill(plx, args, dev, stream, local, tf_peak, peak_src, ranks=4):
     n = max(1, min(args.steps, 20))
     t_blocks = timed(blocks, n)
     t_merge = timed(lambda: plx.plx_fwd_merge(parts, out=out, lse=lse, stream=stream), n)
+
+    # the zig-zag layout: 2 * ranks chunks of c = N / (2 ranks), rank r holds
+    # chunks r and 2 ranks - 1 - r; every rank's blocks and merges, timed rank by rank
+    from parameterized_local_linear_plx_b200 import cp as cpm
+    c = PRE["N"] // (2 * ranks)
+    zq = torch.randn(B, Hq, 2 * c, d, generator=g, device=dev).bfloat16()
+    zr = (0.1 * torch.randn(B, Hq, 2 * c, d, generator=g, device=dev)).bfloat16()
+    zk = torch.randn(2 * ranks, B, Hkv, c, d, generator=g, device=dev).bfloat16()
+    zv = torch.randn(2 * ranks, B, Hkv, c, d, generator=g, device=dev).bfloat16()
+    zq_h = [zq[:, :, :c].contiguous(), zq[:, :, c:].contiguous()]
+    zr_h = [zr[:, :, :c].contiguous(), zr[:, :, c:].contiguous()]
+    # slots 0 .. ranks - 1 for the early chunk's blocks (at most ranks), ranks .. 3 ranks - 1 for the late one's
+    zparts = torch.empty(3 * ranks, B, Hq, c, 2 * d + 4, dtype=torch.float32, device=dev)
+    zout = torch.empty(B, Hq, c, d, dtype=torch.bfloat16, device=dev)
+    zlse = torch.empty(B, Hq, c, dtype=torch.float32, device=dev)
+    zz = []
+    for rk in range(ranks):
+        local, remote = cpm.zigzag_blocks(rk, ranks)
+        a, b_ = cpm.zigzag_chunks(rk, ranks)
+
+        def zig(local=local, remote=remote, a=a, b_=b_):
+            used = {a: 0, b_: ranks}
+            for qc, kc, causal in local + remote:
+                h = 0 if qc == a else 1
+                plx.plx_fwd_partial(zq_h[h], zk[kc], zv[kc], zr_h[h], causal=causal, partial=zparts[used[qc]],
+                                    stream=stream)
+                used[qc] += 1
+            plx.plx_fwd_merge(zparts[:used[a]], out=zout, lse=zlse, stream=stream)
+            plx.plx_fwd_merge(zparts[ranks:used[b_]], out=zout, lse=zlse, stream=stream)
+
+        zz.append(timed(zig, n))
+    zflops = 8 * d * (2 * (c * (c + 1) // 2) + (2 * ranks - 1) * c * c) * B * Hq  # every rank's pairs
     st = plx.plx_check_device_status(stream)
     if st != plx.PLX_OK:
         raise RuntimeError(f"device status after the context-parallel prefill legs: {plx.plx_status_string(st)}")
@@ -623,7 +658,12 @@ def run_cp_prefill(plx, args, dev, stream, local, tf_peak, peak_src, ranks=4):
             "peak_source": peak_src,
             "exchange_bytes_per_rank": 2 * B * Hkv * C * d * 2,
             "note": "per-rank step time = all-gather of the key / value chunks + blocks + merge; the all-gather "
-                    "is not measured (one GPU per run); earlier ranks have fewer blocks"}
+                    "is not measured (one GPU per run); earlier ranks have fewer blocks",
+            "zigzag": {"layout": f"{2 * ranks} chunks of {c}; rank r holds chunks r and {2 * ranks - 1} - r: "
+                                 f"{2 * ranks + 1} blocks (2 causal) and 2 merges per rank",
+                       "ms_per_rank": zz, "max_over_min": max(zz) / min(zz),
+                       "tflops_slowest_rank": zflops / (max(zz) * 1e-3) / 1e12,
+                       "note": "blocks + merges per rank; the all-gather overlaps the three local blocks"}}
 
 
 VARLEN_LENS = [4096, 1, 2048, 777, 1024, 3000, 64, 65, 512, 1500, 4000, 129, 333, 2500, 100, 900,
@@ -1007,6 +1047,41 @@ def run_sweep(args):
           flush=True)
 
 
+def run_profile_small(args):
+    """--profile-small: one call of each small case the ncu summaries in
+    profiles/ capture (decode in both plans, the projection in both forms),
+    then exit; inputs larger than L2 but a few GB at most."""
+    import torch
+    from parameterized_local_linear_plx_b200 import build, inputs
+    build.build()
+    from parameterized_local_linear_plx_b200 import plx
+    dev = torch.device("cuda", 0)
+    # decode, balanced plan: B=1, context 32768, Hq=16, Hkv=8, d=128 (134 MB of KV)
+    q, kc, vc, r, sl = inputs.decode_inputs(1, 16, 8, 32768, 128, seed=0, device=dev)
+    plx.plx_decode(q, kc, vc, sl, r)
+    del kc, vc
+    # decode, chunked plan: B=64, context 4096 (1.07 GB of KV)
+    q, kc, vc, r, sl = inputs.decode_inputs(64, 16, 8, 4096, 128, seed=0, device=dev)
+    plx.plx_decode(q, kc, vc, sl, r)
+    del kc, vc
+    # projection, prefill form: 2 x 4096 tokens, d_model 1024, W [6144, 1024]
+    g = torch.Generator(device=dev).manual_seed(1)
+    x = torch.randn(8192, 1024, generator=g, device=dev).bfloat16()
+    w = (torch.randn(6144, 1024, generator=g, device=dev) / 32).bfloat16()
+    plx.plx_qkvr_proj(x, w, 2, 4096, 16, 8, 128)
+    # projection, decode form: 64 tokens appended into a [64, 8, 4096, 128] cache
+    kc = torch.zeros(64, 8, 4096, 128, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    s = torch.full((64,), 4000, dtype=torch.int32, device=dev)
+    plx.plx_qkvr_proj_decode(x[:64].contiguous(), w, kc, vc, s, 16)
+    torch.cuda.synchronize()
+    st = plx.plx_check_device_status()
+    if st != plx.PLX_OK:
+        raise RuntimeError(f"device status: {plx.plx_status_string(st)}")
+    print(json.dumps({"profile_small": "ok"}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -1020,6 +1095,8 @@ def main():
                     "compute-matched) as one JSON line")
     ap.add_argument("--no-decode-configs", action="store_true", help="leave the decode configurations out of the "
                     "bench line")
+    ap.add_argument("--profile-small", action="store_true", help="one call of each small case the ncu summaries "
+                    "capture (decode in both plans, the projection in both forms), then exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -1033,6 +1110,8 @@ def main():
         return run_reference(args, world, rank)
     if args.sweep:
         return run_sweep(args)
+    if args.profile_small:
+        return run_profile_small(args)
     if world > 1:
         import datetime
 

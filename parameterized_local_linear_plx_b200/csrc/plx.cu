@@ -173,7 +173,14 @@ int sm_count_or_default() {
   return 148;  // B200
 }
 
-int decode_ctas(int num_splits) { return num_splits > 0 ? num_splits : 2 * sm_count_or_default(); }
+// The balanced plan's default CTA count: one per SM when segments are long
+// (fewer, longer ranges: fewer partial states to merge), two per SM for
+// short segments (at most 256 keys), whose cost is per segment rather than
+// per key.  Both measured on every shape the plan serves.
+int decode_ctas(int num_splits, int S_max) {
+  if (num_splits > 0) return num_splits;
+  return (S_max <= 256 ? 2 : 1) * sm_count_or_default();
+}
 
 int rows_per_slot(int Hq, int Hkv) { return std::min(Hq / Hkv, 8); }
 
@@ -218,7 +225,7 @@ DecodePlan plan_decode(int B, int Hq, int Hkv, int S_max, int d, int num_splits,
     return pl;
   }
   pl.chunked = false;
-  pl.P = decode_ctas(num_splits);
+  pl.P = decode_ctas(num_splits, S_max);
   pl.ws_bytes = decode_scratch_bytes(Hq, Hkv, d, pl.P);
   return pl;
 }
@@ -662,7 +669,7 @@ int plx_bwd(const void* q, const void* k, const void* v, const void* r, const vo
 }
 
 int plx_decode_num_splits(int B, int Hq, int Hkv, int S_max, int d) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128)) return decode_ctas(0);
+  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128)) return decode_ctas(0, 4096);
   return plan_decode(B, Hq, Hkv, S_max, d, 0, false).P;
 }
 
@@ -741,7 +748,7 @@ int plx_decode(const void* q, const void* r, const void* kcache, const void* vca
 size_t plx_decode_partial_size(int B, int Hq, int Hkv, int S_max, int d, int num_splits) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128) || num_splits < 0) return 0;
   return align256(static_cast<size_t>(B) * Hq * (2 * d + 4) * sizeof(float)) +
-         decode_scratch_bytes(Hq, Hkv, d, decode_ctas(num_splits));
+         plan_decode(B, Hq, Hkv, S_max, d, num_splits, true).ws_bytes;
 }
 
 int plx_decode_partial(const void* q, const void* r, const void* kcache, const void* vcache,

@@ -58,6 +58,7 @@ constexpr int kDecConsumerWarps = 4; // 16 keys of each tile per warp
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
 constexpr int kDecMinTilesPerCta = 4;   // smallest range: below this a CTA's ring has nothing to overlap
 constexpr int kDecCombineThreads = 128;
+constexpr int kCombineDepth = 4;  // partial states a combine warp has in flight
 
 template <int D>
 struct DecodeCfg {
@@ -832,7 +833,7 @@ plx_decode_chunk_kernel(const __grid_constant__ CUtensorMap kmap,
 // dependent of the split kernel; small enough (128 threads, ~4 KB of shared
 // memory) to be resident beside two split CTAs on an SM.
 template <int D>
-__global__ void __launch_bounds__(kDecCombineThreads)
+__global__ void __launch_bounds__(kDecCombineThreads, 6)  // <= 85 registers: fits beside two split CTAs
 plx_decode_combine_kernel(const DecodeParams p, int P) {
   constexpr int RF = DecodeCfg<D>::kRecFloats;
   constexpr int NT = kDecCombineThreads;
@@ -901,11 +902,12 @@ plx_decode_combine_kernel(const DecodeParams p, int P) {
         float M = -INFINITY, L = 0.f, C = 0.f;
         float4 a1 = make_float4(0.f, 0.f, 0.f, 0.f), a2 = a1;
         const bool lv = lane < LANES;
-        for (int k0 = sub; k0 < n; k0 += 2 * wpr) {
-          // two partials per round, both loaded before either is merged
-          float4 h[2], x1[2], x2[2];
+        constexpr int R = kCombineDepth;
+        for (int k0 = sub; k0 < n; k0 += R * wpr) {
+          // R partials per round, all loaded before any is merged
+          float4 h[R], x1[R], x2[R];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
+          for (int u = 0; u < R; ++u) {
             const int kk = k0 + u * wpr;
             h[u] = make_float4(-INFINITY, 0.f, 0.f, 0.f);
             x1[u] = x2[u] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -920,7 +922,7 @@ plx_decode_combine_kernel(const DecodeParams p, int P) {
             }
           }
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
+          for (int u = 0; u < R; ++u) {
             const float Mn = fmaxf(M, h[u].x);
             if (Mn == -INFINITY) continue;
             const float al = ex2(M - Mn), be = ex2(h[u].x - Mn);

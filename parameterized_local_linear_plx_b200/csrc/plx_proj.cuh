@@ -253,17 +253,21 @@ plx_proj_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
           }
         }
         __syncwarp();
-        // the warp writes its 32 rows, cpr lanes per row, 16 bytes each
+        // each lane finds the destination of its own row once (the index
+        // arithmetic has runtime divisors); the warp then writes its 32 rows,
+        // cpr lanes per row, 16 bytes each, taking row pointers by shuffle
+        const int col = n0 + c0, in_head = col & (d - 1);
+        const int m_me = rbase + lane;
+        __nv_bfloat16* mine = m_me < p.M ? proj_dest(p, m_me, col - in_head) : nullptr;
+        const unsigned long long my_dst =
+            mine ? reinterpret_cast<unsigned long long>(mine + in_head) : 0ull;
+        const int rshift = __ffs(cpr) - 1;  // cpr is a power of two
         for (int idx = lane; idx < 32 * cpr; idx += 32) {
-          const int rr = idx / cpr, ch = idx % cpr;
-          const int m = rbase + rr;
-          if (m >= p.M) continue;
-          const int col = n0 + c0, in_head = col % d;
-          __nv_bfloat16* dst = proj_dest(p, m, col - in_head);
-          if (dst == nullptr) continue;
-          dst += in_head;
+          const int rr = idx >> rshift, ch = idx & (cpr - 1);
+          const unsigned long long dst = __shfl_sync(0xffffffffu, my_dst, rr);
+          if (dst == 0ull) continue;
           const uint4 w4 = *reinterpret_cast<const uint4*>(stg + rr * (cw * 2) + ((ch ^ (rr & (cpr - 1))) * 16));
-          *reinterpret_cast<uint4*>(dst + ch * 8) = w4;
+          *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(dst) + ch * 8) = w4;
         }
         __syncwarp();
       }

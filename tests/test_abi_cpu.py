@@ -113,15 +113,15 @@ def test_split_planning(plx):
         want = up(2 * P * min(Hq // Hkv, 8) * (2 * d + 4) * 4)
         assert plx.plx_decode_workspace_size(2, Hq, Hkv, 1024, d, P) == want
         assert plx.plx_decode_workspace_size(64, Hq, Hkv, 32768, d, P) == want
-    # automatic plan, few segments (b, kv head): two balanced partitions per SM
+    # automatic plan, few segments (b, kv head): one balanced partition per SM
     n = plx.plx_decode_num_splits(1, 16, 8, 4096, 128)
-    assert n >= 2 and n % 2 == 0
+    assert n >= 1
     assert plx.plx_decode_num_splits(8, 16, 8, 32768, 128) == n  # 64 segments
     assert plx.plx_decode_workspace_size(1, 16, 8, 4096, 128, 0) == plx.plx_decode_workspace_size(1, 16, 8, 4096, 128, n)
     # automatic plan, many segments: chunks of whole 64-key tiles, about four
     # waves of two CTAs per SM, chunks of at least 128 keys; one record of
     # (2d + 4) floats per (b, h, chunk) when a segment has several chunks
-    sms = n // 2
+    sms = n
     for B, S in [(64, 4096), (256, 1024), (2048, 16384), (1024, 512)]:
         segs = B * 8
         sp = max(1, min(-(-4 * 2 * sms // segs), (S + 127) // 128))
@@ -130,8 +130,9 @@ def test_split_planning(plx):
         assert plx.plx_decode_num_splits(B, 16, 8, S, 128) == segs * splits
         assert plx.plx_decode_workspace_size(B, 16, 8, S, 128, 0) == (up(B * 16 * splits * 260 * 4) if splits > 1 else 0)
     assert plx.plx_decode_num_splits(2048, 16, 8, 16384, 128) == 2048 * 8  # one chunk per segment: no workspace
-    # short segments keep the balanced plan whatever their number
-    assert plx.plx_decode_num_splits(2048, 16, 8, 256, 128) == n
+    # short segments keep the balanced plan whatever their number, with two partitions per SM
+    assert plx.plx_decode_num_splits(2048, 16, 8, 256, 128) == 2 * n
+    assert plx.plx_decode_num_splits(1, 16, 8, 128, 128) == 2 * n
     # bad shapes: size 0
     assert plx.plx_decode_workspace_size(1, 3, 2, 128, 128, 2) == 0
     assert plx.plx_decode_workspace_size(1, 2, 1, 128, 128, -1) == 0

@@ -131,3 +131,77 @@ def test_context_parallel_prefill_through_nccl_world_one(plx):
         close_to_prefill(plx, out, lse, q, k, v, r)
     finally:
         dist.destroy_process_group()
+
+
+def emulate_zigzag(plx, q, k, v, r, ranks):
+    """Every rank's zig-zag blocks (cp.zigzag_blocks) computed on this GPU from
+    chunks of the full tensors, merged per query chunk, then unsharded."""
+    from parameterized_local_linear_plx_b200 import cp
+    N = q.shape[2]
+    c = N // (2 * ranks)
+
+    def chunk(t, i):
+        return t[:, :, i * c:(i + 1) * c].contiguous()
+
+    outs, lses = [], []
+    for rk in range(ranks):
+        local, remote = cp.zigzag_blocks(rk, ranks)
+        res = {}
+        for qc in cp.zigzag_chunks(rk, ranks):
+            blocks = [(kc, causal) for qq, kc, causal in local + remote if qq == qc]
+            parts = torch.stack([plx.plx_fwd_partial(chunk(q, qc), chunk(k, kc), chunk(v, kc),
+                                                     None if r is None else chunk(r, qc), causal=causal)
+                                 for kc, causal in blocks])
+            res[qc] = plx.plx_fwd_merge(parts)
+        a, b = cp.zigzag_chunks(rk, ranks)
+        outs.append(torch.cat([res[a][0], res[b][0]], dim=2))
+        lses.append(torch.cat([res[a][1], res[b][1]], dim=2))
+    torch.cuda.synchronize()
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    return cp.zigzag_unshard(outs), cp.zigzag_unshard(lses)
+
+
+@pytest.mark.parametrize("ranks", [1, 2, 3, 4])
+@pytest.mark.parametrize("d", [64, 128])
+def test_zigzag_chunks_match_prefill_and_oracle(plx, ranks, d):
+    """Zig-zag layout, chunks of 48 rows (each ends inside a key tile)."""
+    B, Hq, Hkv, c = 2, 4, 2, 48
+    q, k, v, r = inputs.prefill_inputs(B, Hq, Hkv, 2 * ranks * c, d, seed=90 + 10 * ranks + d, device="cuda")
+    out, lse = emulate_zigzag(plx, q, k, v, r, ranks)
+    close_to_prefill(plx, out, lse, q, k, v, r)
+    ro, rl = oracle.prefill_effective(q.cpu(), k.cpu(), v.cpu(), r.cpu(), True)
+    assert_close(out, ro, lse, rl, f"zigzag ranks={ranks} d={d}")
+
+
+def test_zigzag_bench_shape(plx):
+    """Causal prefill B=1, N=4096, Hq=16, Hkv=8, d=128 over 4 emulated ranks
+    (8 chunks of 512), rho = 0 and rho."""
+    q, k, v, r = inputs.prefill_inputs(1, 16, 8, 4096, 128, seed=3, device="cuda")
+    for rr in (None, r):
+        out, lse = emulate_zigzag(plx, q, k, v, rr, 4)
+        close_to_prefill(plx, out, lse, q, k, v, rr)
+
+
+def test_zigzag_through_nccl_world_one(plx):
+    """The zig-zag orchestration (asynchronous all-gather overlapped by the
+    local blocks, remote blocks, two merges) with one rank."""
+    import datetime
+    import socket
+
+    import torch.distributed as dist
+    from parameterized_local_linear_plx_b200 import cp
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda", 0))
+    try:
+        q, k, v, r = inputs.prefill_inputs(2, 8, 2, 334, 128, seed=13, device="cuda")
+        sh = lambda t: cp.zigzag_shard(t, 0, 1)
+        out, lse = cp.context_parallel_prefill_zigzag(sh(q), sh(k), sh(v), sh(r))
+        torch.cuda.synchronize()
+        out, lse = cp.zigzag_unshard([out]), cp.zigzag_unshard([lse])
+        close_to_prefill(plx, out, lse, q, k, v, r)
+    finally:
+        dist.destroy_process_group()
