@@ -91,6 +91,7 @@ KERNEL_SOURCES = {
     "prefill": ("plx_fwd.cuh", "plx_tcgen05.cuh", "plx_ptx.cuh"),
     "decode": ("plx_decode.cuh", "plx_ptx.cuh"),
     "backward": ("plx_bwd.cuh", "plx_tcgen05.cuh", "plx_ptx.cuh"),
+    "projection": ("plx_proj.cuh", "plx_tcgen05.cuh", "plx_ptx.cuh"),
 }
 
 
@@ -829,7 +830,8 @@ def run_projection(plx, args, dev, stream, world, tf_peak, peak_src):
                         f"outputs scattered to [B, H, N, d]; decode: {Bd} tokens, k/v appended into the cache",
             "tflops": world * achieved, "ms_per_step": ms, "flops_per_step": flops,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
-                         "frac": achieved / tf_peak, "peak_source": peak_src},
+                         "frac": achieved / tf_peak, "traffic": load_traffic("projection"),
+                         "traffic_note": "scaled x4 from a 2 x 4096-token ncu capture", "peak_source": peak_src},
             "decode_us": us_dec,
             "decode_gbs_weights": w_bytes / (us_dec * 1e-6) / 1e9,
             "decode_note": "at 64 tokens the step is bound by reading W once (HBM); gbs counts the weight bytes"}
