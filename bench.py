@@ -440,6 +440,9 @@ def run_gpu(args, world, rank, local):
     # ---- packed variable-length prefill with the same token count (timed on its own)
     varlen = run_varlen(plx, args, dev, stream, world, local, tf_peak, peak_src, tf_key)
 
+    # ---- host cost of one small decode call
+    host = run_host_overhead(plx, dev, stream)
+
     # ---- prefill end to end: inputs from pinned host memory, out and lse back
     e2e_pre = run_e2e_prefill(plx, args, dev, stream, world, pq, pk, pv, pr)
 
@@ -483,6 +486,7 @@ def run_gpu(args, world, rank, local):
             "roofline_decode": roof_dec,
             "e2e": e2e,
             "e2e_prefill": e2e_pre,
+            "decode_host_overhead": host,
             "projection": proj,
             "decode_paged": paged,
             "prefill_varlen": varlen,
@@ -835,6 +839,42 @@ def run_projection(plx, args, dev, stream, world, tf_peak, peak_src):
             "decode_us": us_dec,
             "decode_gbs_weights": w_bytes / (us_dec * 1e-6) / 1e9,
             "decode_note": "at 64 tokens the step is bound by reading W once (HBM); gbs counts the weight bytes"}
+
+
+def run_host_overhead(plx, dev, stream):
+    """Host time per decode call at B=1 (context 4096): the Python binding
+    (argument checks, ctypes) and the raw C ABI through ctypes, each over 200
+    calls enqueued without synchronising (the GPU keeps up at this size, so
+    the loop measures the host's enqueue cost: checks, cached tensor maps, two
+    kernel launches)."""
+    import ctypes
+    import torch
+    q, kc, vc, r, sl = inputs_mod().decode_inputs(1, DEC["Hq"], DEC["Hkv"], DEC["S"], DEC["d"], seed=9, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(1, DEC["Hq"], dtype=torch.float32, device=dev)
+    ws = torch.empty(max(16, plx.plx_decode_workspace_size(1, DEC["Hq"], DEC["Hkv"], DEC["S"], DEC["d"], 0)),
+                     dtype=torch.uint8, device=dev)
+    P = ctypes.c_void_p
+    args_c = (P(q.data_ptr()), P(r.data_ptr()), P(kc.data_ptr()), P(vc.data_ptr()), P(sl.data_ptr()),
+              P(out.data_ptr()), P(lse.data_ptr()), 1, DEC["Hq"], DEC["Hkv"], DEC["S"], DEC["d"],
+              DEC["d"] ** -0.5, 0, P(ws.data_ptr()), ws.numel(), P(stream.cuda_stream))
+    res = {}
+    for name, fn in (("binding", lambda: plx.plx_decode(q, kc, vc, sl, r, out=out, lse=lse, workspace=ws,
+                                                       stream=stream)),
+                     ("c_abi", lambda: plx.lib.plx_decode(*args_c))):
+        for _ in range(20):
+            fn()
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        for _ in range(200):
+            fn()
+        res[f"{name}_us_per_call"] = (time.perf_counter() - t0) / 200 * 1e6
+        torch.cuda.synchronize(dev)
+    st = plx.plx_check_device_status(stream)
+    if st != plx.PLX_OK:
+        raise RuntimeError(f"device status after the host-overhead leg: {plx.plx_status_string(st)}")
+    res["workload"] = f"plx_decode B=1 ctx={DEC['S']} Hq={DEC['Hq']} Hkv={DEC['Hkv']} d={DEC['d']}, 200 calls"
+    return res
 
 
 def run_e2e_prefill(plx, args, dev, stream, world, pq, pk, pv, pr):
