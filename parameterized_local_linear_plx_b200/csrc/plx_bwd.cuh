@@ -25,8 +25,9 @@
 //     G = [dO;0] V^T (dO in the query slots of a second stacked operand and
 //     zeros in the probe slots, so g lands in the query lanes beside a), then
 //     the element-wise warps write [scale dA ; dS] in bf16 over S and one MMA
-//     [scale dA ; dS] K accumulates [dQ ; dR] in tensor memory.  G has two
-//     buffers, so the next tile's G runs during the element-wise pass.
+//     [scale dA ; dS] K accumulates [dQ ; dR] in tensor memory.  S has two
+//     buffers: the scores of tile j+1 are computed during the element-wise
+//     pass of tile j, and only G(j+1) stands between two passes.
 //   * plx_bwd_kv_kernel (dK, dV): one CTA per 128-key tile, keys as the MMA
 //     rows.  For each 64-query tile of each query head of the KV group:
 //     [A^T | S^T] = K [Q;R]^T and G^T = V dO^T; per (key, query) the
@@ -118,11 +119,12 @@ __global__ void __launch_bounds__(256) plx_bwd_pre_kernel(const __nv_bfloat16* _
 
 // ---------------------------------------------------------------- dQ, dR
 // Keys come in tiles of 128 (N = 128 score MMAs: half the instructions per key
-// of 64-key tiles).  Tensor memory holds one score buffer, two G buffers and
-// [dQ ; dR]: G of tile j+1 runs during the element-wise pass of tile j, and
-// only [dQ ; dR] of tile j and the scores of tile j+1 stand between two
-// passes.  K and V have rings of their own: V is free once G has read it, K
-// only after the [dQ ; dR] product.
+// of 64-key tiles).  Tensor memory holds two score buffers, one G buffer and
+// [dQ ; dR]: the scores of tile j+1 run during the element-wise pass of tile
+// j, and only G(j+1) (512 tensor cycles) stands between two passes; [dQ ; dR]
+// of tile j and the scores of j+2 follow it in the tensor pipe.  K and V have
+// rings of their own: V is free once G has read it, K only after the
+// [dQ ; dR] product.
 constexpr int kBwdQBN = 128;     // keys per tile of the query-side kernel
 constexpr int kBwdQKStages = 3;  // K ring
 constexpr int kBwdQVStages = 2;  // V ring
@@ -139,9 +141,9 @@ struct BwdQCfg {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kBwdQKStages * kKVBytes;
   static constexpr int kOffBar = kOffV + kBwdQVStages * kKVBytes;
-  static constexpr int kSmemBytes = kOffBar + 128 + 1024;
-  // tensor memory: S [0,128), G of tile j at 128 + 128 (j & 1), [dQ ; dR] at 384
-  static constexpr uint32_t kColS = 0, kColG = 128, kColAcc = 384, kTmemCols = 512;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  // tensor memory: S of tile j at 128 (j & 1), G at 256, [dQ ; dR] at 384
+  static constexpr uint32_t kColS = 0, kColG = 256, kColAcc = 384, kTmemCols = 512;
 };
 
 template <int D, bool HAS_R>
@@ -159,8 +161,9 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
   uint64_t* k_empty = k_full + NK;      // [NK]
   uint64_t* v_full = k_empty + NK;      // [NV]
   uint64_t* v_empty = v_full + NV;      // [NV]
-  uint64_t* s_full = v_empty + NV;      // [1] S of a key tile (and its G, issued before) in TMEM
-  uint64_t* p_ready = s_full + 1;       // [1] [dA ; dS] written (one arrival per element-wise warp)
+  uint64_t* s_full = v_empty + NV;      // [2] S of a key tile in TMEM buffer j & 1
+  uint64_t* g_full = s_full + 2;        // [1] G of a key tile in TMEM
+  uint64_t* p_ready = g_full + 1;       // [1] [dA ; dS] written (one arrival per element-wise warp)
   uint64_t* o_done = p_ready + 1;       // [1] every MMA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
 
@@ -186,7 +189,9 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       mbar_init(smem_u32(&v_full[s]), 1);
       mbar_init(smem_u32(&v_empty[s]), 1);
     }
-    mbar_init(smem_u32(s_full), 1);
+    mbar_init(smem_u32(&s_full[0]), 1);
+    mbar_init(smem_u32(&s_full[1]), 1);
+    mbar_init(smem_u32(g_full), 1);
     mbar_init(smem_u32(p_ready), kBwdElemWarps);  // one arrival per element-wise warp
     mbar_init(smem_u32(o_done), 1);
     fence_barrier_init();
@@ -273,26 +278,29 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       const uint64_t d_v = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffV), 16, 1024);
       const uint64_t d_kmn = tc::smem_desc_sw128(smem_u32(smem + Cfg::kOffK), Cfg::kKVBlock, 1024);
       // Per key tile j, in issue order (the tensor pipe runs them in that
-      // order): G(j+1) into the other G buffer; after the element-wise pass of
-      // j, [dQ ; dR] += [scale dA ; dS] K (the last reader of the score
-      // columns); then the scores of j+1.
+      // order): after the element-wise pass of j, G(j+1) (the pass of j+1 then
+      // waits only for it: its scores were computed during the pass of j),
+      // [dQ ; dR] += [scale dA ; dS] K (the last reader of S buffer j & 1),
+      // then the scores of j+2 into that buffer.
       auto issue_s = [&](int j) -> bool {
         const int s = j % NK;
         if (!mbar_wait(smem_u32(&k_full[s]), (j / NK) & 1, kErrBwdMma)) return false;
         tc::fence_after_sync();
+        const uint32_t cs = tmem + Cfg::kColS + 128 * static_cast<uint32_t>(j & 1);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t koff_a = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
           const uint64_t koff_b = static_cast<uint64_t>(((ks >> 2) * Cfg::kKVBlock + (ks & 3) * 32) >> 4);
-          tc::mma_ss(tmem + Cfg::kColS, d_qr + koff_a, d_k + s * kStageStep + koff_b, idesc_s, ks > 0 ? 1u : 0u);
+          tc::mma_ss(cs, d_qr + koff_a, d_k + s * kStageStep + koff_b, idesc_s, ks > 0 ? 1u : 0u);
         }
+        tc::commit(smem_u32(&s_full[j & 1]));
         return true;
       };
       auto issue_g = [&](int j) -> bool {
         const int s = j % NV;
         if (!mbar_wait(smem_u32(&v_full[s]), (j / NV) & 1, kErrBwdMma)) return false;
         tc::fence_after_sync();
-        const uint32_t cg = tmem + Cfg::kColG + 128 * static_cast<uint32_t>(j & 1);
+        const uint32_t cg = tmem + Cfg::kColG;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t koff_a = static_cast<uint64_t>(((ks >> 2) * Cfg::kBlock + (ks & 3) * 32) >> 4);
@@ -300,32 +308,27 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
           tc::mma_ss(cg, d_do + koff_a, d_v + s * kStageStep + koff_b, idesc_s, ks > 0 ? 1u : 0u);
         }
         tc::commit(smem_u32(&v_empty[s]));  // G is V's only reader
+        tc::commit(smem_u32(g_full));
         return true;
       };
       ok = mbar_wait(smem_u32(q_full), 0, kErrBwdMma);
-      if (ok && nkv > 0) {
-        ok = issue_g(0) && issue_s(0);
-        if (ok) tc::commit(smem_u32(s_full));
-      }
+      if (ok && nkv > 0) ok = issue_g(0) && issue_s(0) && (nkv < 2 || issue_s(1));
       for (int j = 0; j < nkv && ok; ++j) {
-        const bool more = j + 1 < nkv;
-        // G(j+1) goes to the buffer of tile j-1, whose element-wise pass is over (p_ready waited)
-        if (more && !issue_g(j + 1)) { ok = false; break; }
+        // the element-wise pass of j is over: G and S buffer j & 1 may be reused
         if (!mbar_wait(smem_u32(p_ready), j & 1, kErrBwdMma)) { ok = false; break; }
         tc::fence_after_sync();
+        if (j + 1 < nkv && !issue_g(j + 1)) { ok = false; break; }
         // A = the bf16 pairs of keys 16kk..16kk+15: warp part c wrote keys
-        // 32c..32c+31 as pairs at columns 32c..32c+15
+        // 32c..32c+31 as pairs at columns 32c..32c+15 of its S buffer
         const int sk = j % NK;
+        const uint32_t cs = tmem + Cfg::kColS + 128 * static_cast<uint32_t>(j & 1);
 #pragma unroll
         for (int kk = 0; kk < kBwdQBN / 16; ++kk)
-          tc::mma_ts(tmem + Cfg::kColAcc, tmem + Cfg::kColS + 32 * (kk >> 1) + 8 * (kk & 1),
+          tc::mma_ts(tmem + Cfg::kColAcc, cs + 32 * (kk >> 1) + 8 * (kk & 1),
                      d_kmn + sk * kStageStep + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
                      (j > 0 || kk > 0) ? 1u : 0u);
         tc::commit(smem_u32(&k_empty[sk]));
-        if (more) {
-          if (!issue_s(j + 1)) { ok = false; break; }
-          tc::commit(smem_u32(s_full));  // scores of j+1, and G(j+1) issued before
-        }
+        if (j + 2 < nkv && !issue_s(j + 2)) { ok = false; break; }
       }
       tc::commit(smem_u32(o_done));  // also on abort: every issued MMA completes before dealloc
       mbar_wait(smem_u32(o_done), 0, kErrBwdMma);
@@ -363,12 +366,13 @@ plx_bwd_q_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
     const uint64_t nd_lo = f2(-dd_lo, -dd_lo), nd_hi = f2(-dd_hi, -dd_hi);
     const uint64_t c_sl2 = f2(p.scale_log2, p.scale_log2), c_m1 = f2(-1.f, -1.f), c_sc = f2(p.scale, p.scale);
     for (int j = 0; j < nkv; ++j) {
-      const bool landed = mbar_wait_sleep(smem_u32(s_full), j & 1, kErrBwdElem);
+      const bool landed = mbar_wait_sleep(smem_u32(&s_full[j & 1]), (j >> 1) & 1, kErrBwdElem) &&
+                          mbar_wait_sleep(smem_u32(g_full), j & 1, kErrBwdElem);
       if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
       tc::fence_after_sync();
-      const uint32_t cs = Cfg::kColS + 32 * part;
+      const uint32_t cs = Cfg::kColS + 128 * static_cast<uint32_t>(j & 1) + 32 * part;
       const uint32_t ta = tmem + lane_a + cs, ts = tmem + lane_s + cs;
-      const uint32_t tg = tmem + lane_a + Cfg::kColG + 128 * static_cast<uint32_t>(j & 1) + 32 * part;
+      const uint32_t tg = tmem + lane_a + Cfg::kColG + 32 * part;
       uint32_t ra[16], rs[16], rg[16];
       tc::ld_16x256b_x4(ta, ra);
       tc::ld_16x256b_x4(ts, rs);
