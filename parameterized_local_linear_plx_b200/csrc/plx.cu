@@ -231,8 +231,8 @@ DecodePlan plan_decode(int B, int Hq, int Hkv, int S_max, int d, int num_splits,
 }
 
 template <int D, bool HAS_R, bool PAGED>
-int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const plx::DecodeParams& p, int P,
-                  cudaStream_t st) {
+int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& kt, const CUtensorMap& vt,
+                  const plx::DecodeParams& p, int P, cudaStream_t st) {
   using Cfg = plx::DecodeCfg<D>;
   static bool done[kMaxDevices], done_chunk[kMaxDevices];
   int dev = 0;
@@ -242,13 +242,13 @@ int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const plx::Decod
     if (ensure_smem(kern, Cfg::kChunkSmemBytes, &done_chunk[dev]) != PLX_OK) return PLX_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(p.splits), static_cast<unsigned>(p.Hkv * p.n_hgroups),
                     static_cast<unsigned>(p.B));
-    kern<<<grid, plx::kDecThreads, Cfg::kChunkSmemBytes, st>>>(km, vm, p);
+    kern<<<grid, plx::kDecThreads, Cfg::kChunkSmemBytes, st>>>(km, vm, kt, vt, p);
     if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
     if (p.splits == 1) return PLX_OK;  // every segment was finished whole
   } else {
     auto kern = plx::plx_decode_split_kernel<D, HAS_R, PAGED>;
     if (ensure_smem(kern, Cfg::kSmemBytes, &done[dev]) != PLX_OK) return PLX_ERR_CUDA;
-    kern<<<static_cast<unsigned>(P), plx::kDecThreads, Cfg::kSmemBytes, st>>>(km, vm, p);
+    kern<<<static_cast<unsigned>(P), plx::kDecThreads, Cfg::kSmemBytes, st>>>(km, vm, kt, vt, p);
     if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
   }
   // programmatic dependent launch: the second kernel's CTAs are scheduled
@@ -546,8 +546,12 @@ int plx_decode_paged(const void* q, const void* r, const void* kpool, const void
   p.splits = plan.chunked ? plan.splits : 0;
   p.scale_log2 = scale * plx::kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 128) return r ? launch_decode<128, true, true>(km, vm, p, P, st) : launch_decode<128, false, true>(km, vm, p, P, st);
-  return r ? launch_decode<64, true, true>(km, vm, p, P, st) : launch_decode<64, false, true>(km, vm, p, P, st);
+  // (the partial-tile maps are for contiguous caches; page parts carry their own box)
+  if (d == 128)
+    return r ? launch_decode<128, true, true>(km, vm, km, vm, p, P, st)
+             : launch_decode<128, false, true>(km, vm, km, vm, p, P, st);
+  return r ? launch_decode<64, true, true>(km, vm, km, vm, p, P, st)
+           : launch_decode<64, false, true>(km, vm, km, vm, p, P, st);
 }
 
 }  // extern "C"
@@ -708,10 +712,13 @@ int decode_common(const void* q, const void* r, const void* kcache, const void* 
   if (rc != PLX_OK) return rc;
   if ((rc = get_encoder()) != PLX_OK) return rc;
 
-  CUtensorMap km, vm;
+  // full 64-key tiles, and kDecTailRows-key parts for each sequence's last, partial tile
+  CUtensorMap km, vm, kt, vt;
   const long long planes = static_cast<long long>(B) * Hkv;
   if (make_map_3d(&km, kcache, d, S_max, planes, plx::kDecTileKeys) != PLX_OK ||
-      make_map_3d(&vm, vcache, d, S_max, planes, plx::kDecTileKeys) != PLX_OK)
+      make_map_3d(&vm, vcache, d, S_max, planes, plx::kDecTileKeys) != PLX_OK ||
+      make_map_3d(&kt, kcache, d, S_max, planes, plx::kDecTailRows) != PLX_OK ||
+      make_map_3d(&vt, vcache, d, S_max, planes, plx::kDecTailRows) != PLX_OK)
     return PLX_ERR_CUDA;
 
   plx::DecodeParams p{};
@@ -729,8 +736,11 @@ int decode_common(const void* q, const void* r, const void* kcache, const void* 
   p.key_offset = key_offset;
   p.scale_log2 = scale * plx::kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 128) return r ? launch_decode<128, true, false>(km, vm, p, P, st) : launch_decode<128, false, false>(km, vm, p, P, st);
-  return r ? launch_decode<64, true, false>(km, vm, p, P, st) : launch_decode<64, false, false>(km, vm, p, P, st);
+  if (d == 128)
+    return r ? launch_decode<128, true, false>(km, vm, kt, vt, p, P, st)
+             : launch_decode<128, false, false>(km, vm, kt, vt, p, P, st);
+  return r ? launch_decode<64, true, false>(km, vm, kt, vt, p, P, st)
+           : launch_decode<64, false, false>(km, vm, kt, vt, p, P, st);
 }
 
 }  // namespace

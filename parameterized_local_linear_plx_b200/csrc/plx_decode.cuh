@@ -57,6 +57,7 @@ constexpr int kDecTileKeys = 64;     // keys per pipeline stage
 constexpr int kDecConsumerWarps = 4; // 16 keys of each tile per warp
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
 constexpr int kDecMinTilesPerCta = 4;   // smallest range: below this a CTA's ring has nothing to overlap
+constexpr int kDecTailRows = 16;     // a sequence's last, partial tile is loaded in parts of this many keys
 constexpr int kDecCombineThreads = 128;
 constexpr int kCombineDepth = 4;  // partial states a combine warp has in flight
 
@@ -117,6 +118,77 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
                : "memory");
+}
+
+// Consumer: o += [P ; P*S] V over this warp's 16 keys of the stage's V tile
+// (transposed ldmatrix: b0 / b2 hold keys qc*2, qc*2+1 of the first eight,
+// b1 / b3 the same of the second eight, lower key in the low half).
+template <int D>
+__device__ __forceinline__ void value_mma(float (&o)[D / 8][4], const uint32_t (&pa)[4], uint32_t vbase, int vkey,
+                                          int mi) {
+#pragma unroll
+  for (int jp = 0; jp < D / 16; ++jp) {
+    const int chunk = (2 * jp + (mi >> 1)) & 7;
+    const uint32_t addr = vbase + (jp >> 2) * (kDecTileKeys * 128) + sw128(vkey, chunk);
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4_t(addr, b0, b1, b2, b3);
+    mma_bf16_16816(o[2 * jp], pa, b0, b1);
+    mma_bf16_16816(o[2 * jp + 1], pa, b2, b3);
+  }
+}
+
+// The same with the value rows of keys >= kend zeroed in the fragments, so
+// that a zero weight times whatever those rows hold (Inf, NaN) adds nothing.
+// key_lo = the key of this thread's first fragment element.
+template <int D>
+__device__ __forceinline__ void value_mma_masked(float (&o)[D / 8][4], const uint32_t (&pa)[4], uint32_t vbase,
+                                                 int vkey, int mi, int key_lo, int kend) {
+  const uint32_t m_lo = (key_lo < kend ? 0x0000ffffu : 0u) | (key_lo + 1 < kend ? 0xffff0000u : 0u);
+  const uint32_t m_hi = (key_lo + 8 < kend ? 0x0000ffffu : 0u) | (key_lo + 9 < kend ? 0xffff0000u : 0u);
+#pragma unroll
+  for (int jp = 0; jp < D / 16; ++jp) {
+    const int chunk = (2 * jp + (mi >> 1)) & 7;
+    const uint32_t addr = vbase + (jp >> 2) * (kDecTileKeys * 128) + sw128(vkey, chunk);
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4_t(addr, b0, b1, b2, b3);
+    b0 &= m_lo; b1 &= m_hi; b2 &= m_lo; b3 &= m_hi;
+    mma_bf16_16816(o[2 * jp], pa, b0, b1);
+    mma_bf16_16816(o[2 * jp + 1], pa, b2, b3);
+  }
+}
+
+// Producer: the K and V tile of keys key0 .. key0 + 63 of plane kvrow into
+// kdst / vdst (128-byte swizzled, D / 64 column halves of 64 rows each),
+// completing on `bar`, which also expects `extra` bytes of other copies.  A
+// tile with fewer than 64 live keys (the sequence's last) is loaded in
+// kDecTailRows-key parts through the maps kmap_t / vmap_t, only as far as the
+// live keys reach: the rows past them keep whatever the stage held before,
+// which the consumers mask out.  A part's 16 x 128-byte boxes start on 2 KB
+// boundaries, so the swizzle pattern of every row is the full tile's.
+template <int D>
+__device__ __forceinline__ void load_kv_tile(const CUtensorMap* kmap, const CUtensorMap* vmap, const CUtensorMap* kmap_t,
+                                             const CUtensorMap* vmap_t, uint32_t kdst, uint32_t vdst, uint32_t bar,
+                                             int key0, int live_from_key0, int kvrow, uint32_t extra) {
+  constexpr int kHalves = D / 64;
+  if (live_from_key0 >= kDecTileKeys) {
+    mbar_arrive_expect_tx(bar, 2u * kDecTileKeys * D * 2 + extra);
+#pragma unroll
+    for (int hf = 0; hf < kHalves; ++hf) {
+      tma_load_3d(kmap, kdst + hf * (kDecTileKeys * 128), bar, hf * 64, key0, kvrow);
+      tma_load_3d(vmap, vdst + hf * (kDecTileKeys * 128), bar, hf * 64, key0, kvrow);
+    }
+    return;
+  }
+  const int parts = (live_from_key0 + kDecTailRows - 1) / kDecTailRows;  // 1 .. 4
+  mbar_arrive_expect_tx(bar, static_cast<uint32_t>(parts) * (2u * kDecTailRows * D * 2) + extra);
+  for (int part = 0; part < parts; ++part) {
+    const uint32_t off = static_cast<uint32_t>(part * kDecTailRows * 128);
+#pragma unroll
+    for (int hf = 0; hf < kHalves; ++hf) {
+      tma_load_3d(kmap_t, kdst + hf * (kDecTileKeys * 128) + off, bar, hf * 64, key0 + part * kDecTailRows, kvrow);
+      tma_load_3d(vmap_t, vdst + hf * (kDecTileKeys * 128) + off, bar, hf * 64, key0 + part * kDecTailRows, kvrow);
+    }
+  }
 }
 
 // Position in the tile list: segment (b, j = g * n_hgroups + hg), tile i of
@@ -214,7 +286,9 @@ __device__ __forceinline__ int dec_tpc(int T, int P) { return max((T + P - 1) / 
 template <int D, bool HAS_R, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, 2)
 plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
-                        const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
+                        const __grid_constant__ CUtensorMap vmap,
+                        const __grid_constant__ CUtensorMap kmap_t,
+                        const __grid_constant__ CUtensorMap vmap_t, const DecodeParams p) {
   using Cfg = DecodeCfg<D>;
   constexpr int NS = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -284,17 +358,14 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
             break;
           }
           const uint32_t fb = smem_u32(&full_bar[s]);
-          mbar_arrive_expect_tx(fb, Cfg::kKVBytes + (u == 0 ? qr_bytes : 0u));
           const uint32_t kdst = smem_u32(smem + s * Cfg::kStageBytes);
           const uint32_t vdst = kdst + Cfg::kTileBytes;
           const int key0 = (cur.i + u) * kDecTileKeys;
           if (!PAGED) {
-#pragma unroll
-            for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-              tma_load_3d(&kmap, kdst + hf * (kDecTileKeys * 128), fb, hf * 64, key0, kvrow);
-              tma_load_3d(&vmap, vdst + hf * (kDecTileKeys * 128), fb, hf * 64, key0, kvrow);
-            }
+            load_kv_tile<D>(&kmap, &vmap, &kmap_t, &vmap_t, kdst, vdst, fb, key0, cur.live - key0, kvrow,
+                            u == 0 ? qr_bytes : 0u);
           } else {
+            mbar_arrive_expect_tx(fb, Cfg::kKVBytes + (u == 0 ? qr_bytes : 0u));
             // one load per page part of the tile: plane = page * Hkv + g, row within the page
             for (int part = 0; part * p.box_rows < kDecTileKeys; ++part) {
               const int key = key0 + part * p.box_rows;
@@ -399,13 +470,16 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 
       // ---- shared online softmax over both branches
       const int key_lo = (i0 + u) * kDecTileKeys + warp * 16 + qc * 2;  // key of acc[0][0]
-      float x[4];
+      // Keys past the sequence (the tail of its last tile) take no part,
+      // whatever their rows hold: -inf scores, zero rho.k, zero value rows.
+      float x[4], sv[4];
 #pragma unroll
       for (int nn = 0; nn < 2; ++nn)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int key = key_lo + nn * 8 + e;
-          x[nn * 2 + e] = key < kend ? acc[nn][e] * p.scale_log2 : -INFINITY;
+          const bool in = key_lo + nn * 8 + e < kend;
+          x[nn * 2 + e] = in ? acc[nn][e] * p.scale_log2 : -INFINITY;
+          sv[nn * 2 + e] = in ? acc[nn][2 + e] : 0.f;  // rho.k, same keys
         }
       float tmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
       tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
@@ -416,7 +490,6 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
       float pr[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) pr[e] = ex2(x[e] - m_use);
-      const float sv[4] = {acc[0][2], acc[0][3], acc[1][2], acc[1][3]};  // rho.k, same keys
       float ps[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) ps[e] = HAS_R ? pr[e] * sv[e] : 0.f;
@@ -439,15 +512,10 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
       }
 
       // ---- value product with the stacked [P ; P*S] operand
-#pragma unroll
-      for (int jp = 0; jp < D / 16; ++jp) {
-        const int chunk = (2 * jp + (mi >> 1)) & 7;
-        const uint32_t addr = vbase + (jp >> 2) * (kDecTileKeys * 128) + sw128(vkey, chunk);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(addr, b0, b1, b2, b3);
-        mma_bf16_16816(o[2 * jp], pa, b0, b1);
-        mma_bf16_16816(o[2 * jp + 1], pa, b2, b3);
-      }
+      if (key_lo - qc * 2 + 16 <= kend)  // warp-uniform: all 16 keys of this warp are live
+        value_mma<D>(o, pa, vbase, vkey, mi);
+      else
+        value_mma_masked<D>(o, pa, vbase, vkey, mi, key_lo, kend);
       if (u + 1 < n) {
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
@@ -540,7 +608,9 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 template <int D, bool HAS_R, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, 2)
 plx_decode_chunk_kernel(const __grid_constant__ CUtensorMap kmap,
-                        const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
+                        const __grid_constant__ CUtensorMap vmap,
+                        const __grid_constant__ CUtensorMap kmap_t,
+                        const __grid_constant__ CUtensorMap vmap_t, const DecodeParams p) {
   using Cfg = DecodeCfg<D>;
   constexpr int NS = Cfg::kStages;
   constexpr int kStride = Cfg::kKVBytes;  // stage stride: K and V tiles only
@@ -609,17 +679,13 @@ plx_decode_chunk_kernel(const __grid_constant__ CUtensorMap kmap,
           if (!mbar_wait(smem_u32(&empty_bar[s]), ((t / NS) - 1) & 1, kErrDecodeEmpty)) { ok = false; break; }
         }
         const uint32_t fb = smem_u32(&full_bar[s]);
-        mbar_arrive_expect_tx(fb, kStride);
         const uint32_t kdst = smem_u32(smem + s * kStride);
         const uint32_t vdst = kdst + Cfg::kTileBytes;
         const int key0 = kbeg + t * kDecTileKeys;
         if (!PAGED) {
-#pragma unroll
-          for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-            tma_load_3d(&kmap, kdst + hf * (kDecTileKeys * 128), fb, hf * 64, key0, kvrow);
-            tma_load_3d(&vmap, vdst + hf * (kDecTileKeys * 128), fb, hf * 64, key0, kvrow);
-          }
+          load_kv_tile<D>(&kmap, &vmap, &kmap_t, &vmap_t, kdst, vdst, fb, key0, kend - key0, kvrow, 0u);
         } else {
+          mbar_arrive_expect_tx(fb, kStride);
           // one load per page part of the tile: plane = page * Hkv + g, row within the page
           for (int part = 0; part * p.box_rows < kDecTileKeys; ++part) {
             const int key = key0 + part * p.box_rows;
@@ -707,13 +773,15 @@ plx_decode_chunk_kernel(const __grid_constant__ CUtensorMap kmap,
 
     // ---- shared online softmax over both branches
     const int key_lo = kbeg + t * kDecTileKeys + warp * 16 + qc * 2;  // key of acc[0][0]
-    float x[4];
+    // keys past the sequence take no part, whatever their rows hold
+    float x[4], sv[4];
 #pragma unroll
     for (int n = 0; n < 2; ++n)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int key = key_lo + n * 8 + e;
-        x[n * 2 + e] = key < kend ? acc[n][e] * p.scale_log2 : -INFINITY;
+        const bool in = key_lo + n * 8 + e < kend;
+        x[n * 2 + e] = in ? acc[n][e] * p.scale_log2 : -INFINITY;
+        sv[n * 2 + e] = in ? acc[n][2 + e] : 0.f;  // rho.k, same keys
       }
     float tmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
@@ -724,7 +792,6 @@ plx_decode_chunk_kernel(const __grid_constant__ CUtensorMap kmap,
     float pr[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) pr[i] = ex2(x[i] - m_use);
-    const float sv[4] = {acc[0][2], acc[0][3], acc[1][2], acc[1][3]};  // rho.k, same keys
     float ps[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) ps[i] = HAS_R ? pr[i] * sv[i] : 0.f;
@@ -747,15 +814,10 @@ plx_decode_chunk_kernel(const __grid_constant__ CUtensorMap kmap,
     }
 
     // ---- value product with the stacked [P ; P*S] operand
-#pragma unroll
-    for (int jp = 0; jp < D / 16; ++jp) {
-      const int chunk = (2 * jp + (mi >> 1)) & 7;
-      const uint32_t addr = vbase + (jp >> 2) * (kDecTileKeys * 128) + sw128(vkey, chunk);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(addr, b0, b1, b2, b3);
-      mma_bf16_16816(o[2 * jp], pa, b0, b1);
-      mma_bf16_16816(o[2 * jp + 1], pa, b2, b3);
-    }
+    if (key_lo - qc * 2 + 16 <= kend)  // warp-uniform: all 16 keys of this warp are live
+      value_mma<D>(o, pa, vbase, vkey, mi);
+    else
+      value_mma_masked<D>(o, pa, vbase, vkey, mi, key_lo, kend);
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
   }

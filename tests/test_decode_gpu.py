@@ -195,3 +195,81 @@ def test_decode_largest_sweep_point(plx):
     assert_close(out[pick], ro, lse[pick], rl, "largest sweep point")
     del q, kc, vc, r, sl
     torch.cuda.empty_cache()
+
+
+def _poison_tail(cache, seqlens):
+    """A copy of cache [B, Hkv, S_max, d] whose rows at or past seqlens[b]
+    hold NaN, +Inf and -Inf in turn (what an uninitialised cache may hold)."""
+    bad = cache.clone()
+    vals = (float("nan"), float("inf"), float("-inf"))
+    for b, s in enumerate(seqlens.tolist()):
+        s = max(0, min(int(s), cache.shape[2]))
+        for row in range(s, cache.shape[2]):
+            bad[b, :, row] = vals[row % 3]
+    return bad
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,S,d,splits", [
+    (3, 4, 2, 200, 128, 0),      # balanced plan, tails inside 16-key parts
+    (3, 4, 2, 200, 64, 3),       # explicit partitions
+    (5, 8, 1, 130, 128, 1),      # one partition over every segment
+    (40, 16, 8, 1000, 128, 0),   # chunked plan (320 segments of > 256 keys)
+])
+def test_decode_ignores_cache_rows_past_the_sequence(plx, B, Hq, Hkv, S, d, splits):
+    """Keys past the sequence take no part whatever their rows hold: NaN and
+    Inf there change no bit of out or lse."""
+    rng = np.random.default_rng(B * 1000 + S)
+    lens = [S] + [int(x) for x in rng.integers(1, S, size=B - 1)]
+    lens[-1] = 65 if S > 65 else lens[-1]  # one key into a new tile
+    q, kc, vc, r, sl = inputs.decode_inputs(B, Hq, Hkv, S, d, seed=S + d, seqlens=lens)
+    dev = "cuda"
+    out0, lse0 = plx.plx_decode(q.to(dev), kc.to(dev), vc.to(dev), sl.to(dev), r.to(dev), num_splits=splits)
+    kb, vb = _poison_tail(kc, sl), _poison_tail(vc, sl)
+    out1, lse1 = plx.plx_decode(q.to(dev), kb.to(dev), vb.to(dev), sl.to(dev), r.to(dev), num_splits=splits)
+    torch.cuda.synchronize()
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    assert torch.equal(out0, out1) and torch.equal(lse0, lse1)
+    ro, rl = oracle.decode_effective(q, r, kc, vc, sl)
+    assert_close(out1.float().cpu().numpy(), ro, lse1.cpu().numpy(), rl, f"poisoned tail B={B} S={S} d={d}")
+
+
+def test_decode_paged_ignores_page_rows_past_the_sequence(plx):
+    """The same on a paged cache: the rows of a sequence's last page past its
+    length hold NaN / Inf."""
+    B, Hq, Hkv, mp, ps, d = 4, 8, 2, 5, 64, 128
+    q, kp, vp, r, table, _ = inputs.paged_decode_inputs(B, Hq, Hkv, mp, ps, d, seed=41)
+    sl = torch.tensor([mp * ps, 1, 100, 257], dtype=torch.int32)
+    kc, vc = inputs.gather_pages(kp, table), inputs.gather_pages(vp, table)
+    kb, vb = kp.clone(), vp.clone()
+    vals = (float("nan"), float("inf"), float("-inf"))
+    for b in range(B):
+        for key in range(int(sl[b]), mp * ps):
+            page = int(table[b, key // ps])
+            kb[page, :, key % ps] = vals[key % 3]
+            vb[page, :, key % ps] = vals[(key + 1) % 3]
+    dev = "cuda"
+    args = (table.to(dev), sl.to(dev), r.to(dev))
+    out0, lse0 = plx.plx_decode_paged(q.to(dev), kp.to(dev), vp.to(dev), *args)
+    out1, lse1 = plx.plx_decode_paged(q.to(dev), kb.to(dev), vb.to(dev), *args)
+    torch.cuda.synchronize()
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    assert torch.equal(out0, out1) and torch.equal(lse0, lse1)
+    ro, rl = oracle.decode_effective(q, r, kc, vc, sl)
+    assert_close(out1.float().cpu().numpy(), ro, lse1.cpu().numpy(), rl, "paged poisoned tail")
+
+
+def test_decode_records_ignore_cache_rows_past_the_sequence(plx):
+    """The context-parallel form (state records of a key slice) with the
+    slice's rows past each sequence poisoned: records identical bit for bit."""
+    B, Hq, Hkv, S, d, off = 3, 4, 2, 150, 128, 100
+    lens = [off + S, off + 70, off + 1]
+    q, kc, vc, r, _ = inputs.decode_inputs(B, Hq, Hkv, S, d, seed=77)
+    sl = torch.tensor(lens, dtype=torch.int32)
+    kb, vb = _poison_tail(kc, sl - off), _poison_tail(vc, sl - off)
+    dev = "cuda"
+    rec0 = plx.plx_decode_partial(q.to(dev), kc.to(dev), vc.to(dev), sl.to(dev), r.to(dev), key_offset=off).clone()
+    rec1 = plx.plx_decode_partial(q.to(dev), kb.to(dev), vb.to(dev), sl.to(dev), r.to(dev), key_offset=off).clone()
+    torch.cuda.synchronize()
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    assert torch.isfinite(rec1).all()
+    assert torch.equal(rec0, rec1)
