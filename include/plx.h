@@ -248,13 +248,19 @@ size_t plx_decode_workspace_size(int B, int Hq, int Hkv, int S_max, int d, int n
  *                                       out = 0 and lse = -inf)
  *   out     [B, Hq, d]           bf16   output (written)
  *   lse     [B, Hq]              fp32   (NULL: skipped)
- *   num_splits: key chunks per (b, kv head); 0 = automatic.  With more than
- *     one split the partial states (m, l, c, O1, O2) go to `workspace` and a
- *     second kernel merges them; the result does not depend on the count
- *     beyond rounding.
+ *   num_splits: 0 = automatic.  A positive count asks for the balanced plan
+ *     with that many persistent CTAs, which take equal ranges of the batch's
+ *     64-key tiles; a (b, kv head) stream cut by a range boundary leaves a
+ *     partial state (m, l, c, O1, O2) per CTA in `workspace`, and a second
+ *     kernel merges them.  The automatic choice may instead take the chunked
+ *     plan (a split-KV grid and a merge kernel) for many long streams.  The
+ *     result does not depend on the plan or the count beyond rounding.
  *   workspace / workspace_bytes: caller-owned device scratch of at least
  *     plx_decode_workspace_size(...) bytes, 16-byte aligned (may be NULL when
- *     that size is 0).  Its contents are overwritten.
+ *     that size is 0).  Its contents are overwritten; it need not start at
+ *     zero.  Calls that overlap on the GPU must not share one.
+ *   Cache rows at or past seqlens[b] are never used and may hold anything
+ *   (NaN and Inf included).
  *
  * Requirements: B, Hq, Hkv, S_max >= 1; d in {64, 128}; Hq % Hkv == 0.
  */

@@ -273,3 +273,40 @@ def test_decode_records_ignore_cache_rows_past_the_sequence(plx):
     assert plx.plx_check_device_status() == plx.PLX_OK
     assert torch.isfinite(rec1).all()
     assert torch.equal(rec0, rec1)
+
+
+def test_decode_dirty_workspace_and_graph_replay(plx):
+    """A workspace full of garbage gives the right answer (nothing in it needs
+    to start at zero), and a CUDA graph that replays the same call (the
+    balanced plan's two kernels, the second a programmatic dependent) gives
+    it again, bit for bit."""
+    B, Hq, Hkv, S, d, splits = 3, 8, 2, 1000, 128, 11
+    q, kc, vc, r, sl = inputs.decode_inputs(B, Hq, Hkv, S, d, seed=90, seqlens=[1000, 333, 777])
+    dev = "cuda"
+    q, kc, vc, r, sl_d = q.to(dev), kc.to(dev), vc.to(dev), r.to(dev), sl.to(dev)
+    need = plx.plx_decode_workspace_size(B, Hq, Hkv, S, d, splits)
+    ws = torch.full((need,), 0xAB, dtype=torch.uint8, device=dev)
+    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    plx.plx_decode(q, kc, vc, sl_d, r, num_splits=splits, out=out, lse=lse, workspace=ws)
+    torch.cuda.synchronize()
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    ro, rl = oracle.decode_effective(q.cpu(), r.cpu(), kc.cpu(), vc.cpu(), sl)
+    assert_close(out.float().cpu().numpy(), ro, lse.cpu().numpy(), rl, "dirty workspace")
+    want_o, want_l = out.clone(), lse.clone()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        plx.plx_decode(q, kc, vc, sl_d, r, num_splits=splits, out=out, lse=lse, workspace=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(g):
+        plx.plx_decode(q, kc, vc, sl_d, r, num_splits=splits, out=out, lse=lse, workspace=ws)
+    for _ in range(3):
+        out.zero_()
+        lse.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, want_o) and torch.equal(lse, want_l)
+    assert plx.plx_check_device_status() == plx.PLX_OK
+    del g
