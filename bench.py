@@ -973,15 +973,29 @@ SWEEP_CAP = 150e9  # bytes of KV cache above which a sweep point is skipped
 
 
 def time_decode_point(plx, torch, dev, pool_k, pool_v, B, ctx, d, seqlens_mode, seed, use_r=True, iters=10):
-    """Median CUDA-event time of one plx_decode call (split + combine) on a
-    [B, 8, ctx, d] cache viewed from the start of the pools; q, r ~ N(0,1),
-    N(0, 0.1^2); seqlens "equal" or "ragged" (uniform in [ctx/2, ctx]).  The
-    L2 is emptied before every timed call (a read of twice its size) when
-    the cache is under twice its size."""
+    """Per-call time of plx_decode (split + combine, or chunk + merge) on a
+    [B, 8, ctx, d] cache viewed from the pools; q, r ~ N(0,1), N(0, 0.1^2);
+    seqlens "equal" or "ragged" (uniform in [ctx/2, ctx]).
+
+    us: calls enqueued back to back between one pair of CUDA events (three
+    rounds, the median), each call on its own copy of the cache, rotating
+    over enough copies (adjacent views of the pools) that at least twice the
+    L2's size of other cache bytes is read between two uses of a copy; a
+    cache of 2x L2 or more is its own rotation.  This is the steady per-call
+    cost of a stream of decode calls from HBM.
+    us_single: one call between its own pair of events after the L2 was
+    emptied (a read of twice its size) -- the cold single-call latency; each
+    timing event costs the GPU ~2.6 us before the next kernel starts, which
+    this figure carries."""
     Hq, Hkv = 16, 8
     n = B * Hkv * ctx * d
-    kc = pool_k[:n].view(B, Hkv, ctx, d)
-    vc = pool_v[:n].view(B, Hkv, ctx, d)
+    alloc = 2 * n * 2
+    copies = 1 if alloc >= 2 * L2_BYTES else -(-2 * L2_BYTES // alloc) + 1
+    copies = max(1, min(copies, pool_k.numel() // n))
+    rotate_ok = copies * alloc >= 2 * L2_BYTES or alloc >= 2 * L2_BYTES
+    views = [(pool_k[i * n:(i + 1) * n].view(B, Hkv, ctx, d), pool_v[i * n:(i + 1) * n].view(B, Hkv, ctx, d))
+             for i in range(copies)]
+    kc, vc = views[0]
     g = torch.Generator(device=dev).manual_seed(seed)
     q = torch.randn(B, Hq, d, generator=g, device=dev).bfloat16()
     r = (0.1 * torch.randn(B, Hq, d, generator=g, device=dev)).bfloat16() if use_r else None
@@ -989,21 +1003,30 @@ def time_decode_point(plx, torch, dev, pool_k, pool_v, B, ctx, d, seqlens_mode, 
         sl = torch.full((B,), ctx, dtype=torch.int32, device=dev)
     else:
         sl = torch.randint(ctx // 2, ctx + 1, (B,), generator=g, device=dev, dtype=torch.int32)
-    ws = torch.empty(plx.plx_decode_workspace_size(B, Hq, Hkv, ctx, d, 0), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(16, plx.plx_decode_workspace_size(B, Hq, Hkv, ctx, d, 0)), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
-    alloc = 2 * n * 2
-    # the L2 is emptied before each call of a small point by READING a buffer
-    # twice its size (writing one would leave dirty lines whose write-back
-    # then competes with the call being timed); caches of at least 2x L2 need
-    # no flush: a call streams through more than the L2 holds
+    for i in range(max(5, copies)):
+        kv = views[i % copies]
+        plx.plx_decode(q, kv[0], kv[1], sl, r, out=out, lse=lse, workspace=ws)
+    # back to back over the rotation
+    calls = copies * max(1, -(-max(iters, 20) // copies))
+    per_call = []
+    for _ in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for i in range(calls):
+            kv = views[i % copies]
+            plx.plx_decode(q, kv[0], kv[1], sl, r, out=out, lse=lse, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        per_call.append(a.elapsed_time(b) / calls)
+    # single calls after emptying the L2 by READING a buffer twice its size
+    # (writing one would leave dirty lines whose write-back then competes
+    # with the call being timed); caches of at least 2x L2 need no flush
     flush_src = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if alloc < 2 * L2_BYTES else None
     flush_dst = torch.empty((), dtype=torch.float32, device=dev)
-    for _ in range(5):
-        plx.plx_decode(q, kc, vc, sl, r, out=out, lse=lse, workspace=ws)
-    # calls enqueued back to back (flush, event, call, event, ...) and one
-    # synchronize at the end: each call's events time its GPU work, while the
-    # host enqueues the next one (host-side cost is reported separately)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
     torch.cuda.synchronize()
     for a, b in evs:
@@ -1013,14 +1036,16 @@ def time_decode_point(plx, torch, dev, pool_k, pool_v, B, ctx, d, seqlens_mode, 
         plx.plx_decode(q, kc, vc, sl, r, out=out, lse=lse, workspace=ws)
         b.record()
     torch.cuda.synchronize()
-    ts = [a.elapsed_time(b) for a, b in evs]
     st = plx.plx_check_device_status()
     if st != plx.PLX_OK:
         raise RuntimeError(f"device status after decode point ({B}, {ctx}): {plx.plx_status_string(st)}")
-    ms = statistics.median(ts)
+    ms_single = statistics.median(a.elapsed_time(b) for a, b in evs)
+    ms = statistics.median(per_call) if rotate_ok else ms_single
     nb = decode_bytes(B, Hq, Hkv, d, sl.tolist())
     return {"B": B, "ctx": ctx, "d": d, "seqlens": seqlens_mode, "us": ms * 1e3, "bytes": nb,
-            "gbs": nb / (ms * 1e-3) / 1e9, "kv_alloc_gb": alloc / 1e9, "flushed_l2": flush_src is not None}
+            "gbs": nb / (ms * 1e-3) / 1e9, "us_single": ms_single * 1e3,
+            "gbs_single": nb / (ms_single * 1e-3) / 1e9, "kv_alloc_gb": alloc / 1e9,
+            "rotation_copies": copies if rotate_ok else None, "flushed_l2_single": flush_src is not None}
 
 
 def decode_configs(plx, args, dev, hbm):
@@ -1050,8 +1075,12 @@ def decode_configs(plx, args, dev, hbm):
             pool[i0:i1].copy_(torch.randn(i1 - i0, generator=g, device=dev))
     iters = 10 if not args.small else 3
     res = {"peak_hbm_gbs": hbm, "spec_hbm_gbs": 8000.0,
-           "timing": f"median of {iters} calls enqueued back to back, CUDA events around each call, 5 warm-up; "
-                     f"L2 emptied (a read of 2x its size) before each call when the cache is under 2x L2"}
+           "timing": "us: per call, calls enqueued back to back between one pair of CUDA events (median of 3 "
+                     "rounds of >= 20 calls), each call on its own copy of the KV cache, rotating over enough "
+                     "copies that >= 2x L2 of other cache bytes is read between two uses of a copy (a cache of "
+                     "2x L2 or more is its own rotation); us_single: one call between its own events after a "
+                     "2x-L2 read emptied the L2 (median of the calls), which includes the ~2.6 us a timing "
+                     "event costs the GPU before the next kernel"}
     res["config2"] = []
     for B in (1, 16):
         pt = time_decode_point(plx, torch, dev, pool_k, pool_v, B, 4096, 128, "equal", seed=B, iters=iters)

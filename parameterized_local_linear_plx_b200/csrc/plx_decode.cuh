@@ -313,6 +313,13 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     }
     fence_barrier_init();
   }
+  if (tid == kDecConsumerWarps * 32) {
+    // the descriptors' fetch overlaps the range search below
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&vmap);
+    tma_prefetch_desc(&kmap_t);
+    tma_prefetch_desc(&vmap_t);
+  }
   // ---- this CTA's range of the tile list (scratch: stage 0, before any load)
   int* scratch = reinterpret_cast<int*>(smem);
   DecCursor cur;
@@ -341,8 +348,6 @@ plx_decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
   if (warp == kDecConsumerWarps) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&kmap);
-      tma_prefetch_desc(&vmap);
       bool ok = true;
       int k = 0;  // tiles issued
       for (int t = t_begin; t < t_end && ok;) {
