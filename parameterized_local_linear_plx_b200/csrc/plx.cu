@@ -196,19 +196,29 @@ size_t decode_scratch_bytes(int Hq, int Hkv, int d, int P) {
 // more than 256 keys.
 constexpr long long kChunkedMinSegments = 128;
 constexpr int kChunkedMinKeys = 256;
+// The segment plan (one warp streams each whole segment, one kernel, no
+// partial states) for contiguous caches whose segments are all short.
+constexpr int kSegMaxKeys = 256;
 
 struct DecodePlan {
   bool chunked;
+  bool seg;         // segment plan
   int P;            // CTAs of the decode kernel
   int splits;       // chunked: parts per segment
   int chunk_tiles;  // chunked: tiles per part
   size_t ws_bytes;  // workspace the plan needs
 };
 
-DecodePlan plan_decode(int B, int Hq, int Hkv, int S_max, int d, int num_splits, bool records) {
+DecodePlan plan_decode(int B, int Hq, int Hkv, int S_max, int d, int num_splits, bool records, bool paged) {
   DecodePlan pl{};
   const int n_hg = (Hq / Hkv + 7) / 8;
   const long long segs = static_cast<long long>(B) * Hkv * n_hg;
+  if (num_splits == 0 && !paged && S_max <= kSegMaxKeys && segs <= 0x7fffffffLL) {
+    pl.seg = true;
+    pl.P = static_cast<int>(std::min<long long>((segs + plx::kSegWarps - 1) / plx::kSegWarps, sm_count_or_default()));
+    pl.ws_bytes = 0;
+    return pl;
+  }
   if (num_splits == 0 && !records && segs >= kChunkedMinSegments && S_max > kChunkedMinKeys && B <= 65535 &&
       static_cast<long long>(Hkv) * n_hg <= 65535) {
     // about four waves of two CTAs per SM, chunks of at least 128 keys
@@ -232,11 +242,22 @@ DecodePlan plan_decode(int B, int Hq, int Hkv, int S_max, int d, int num_splits,
 
 template <int D, bool HAS_R, bool PAGED>
 int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& kt, const CUtensorMap& vt,
-                  const plx::DecodeParams& p, int P, cudaStream_t st) {
+                  const CUtensorMap* k32, const CUtensorMap* v32, const plx::DecodeParams& p,
+                  const DecodePlan& plan, cudaStream_t st) {
   using Cfg = plx::DecodeCfg<D>;
-  static bool done[kMaxDevices], done_chunk[kMaxDevices];
+  static bool done[kMaxDevices], done_chunk[kMaxDevices], done_seg[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
+  const int P = plan.P;
+  if constexpr (!PAGED) {
+    if (plan.seg) {
+      auto kern = plx::plx_decode_seg_kernel<D, HAS_R>;
+      constexpr int smem = plx::SegCfg<D>::kSmemBytes;
+      if (ensure_smem(kern, smem, &done_seg[dev]) != PLX_OK) return PLX_ERR_CUDA;
+      kern<<<static_cast<unsigned>(P), plx::kSegThreads, smem, st>>>(*k32, *v32, kt, vt, p);
+      return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+    }
+  }
   if (p.chunk_tiles > 0) {
     auto kern = plx::plx_decode_chunk_kernel<D, HAS_R, PAGED>;
     if (ensure_smem(kern, Cfg::kChunkSmemBytes, &done_chunk[dev]) != PLX_OK) return PLX_ERR_CUDA;
@@ -504,8 +525,7 @@ int plx_decode_paged(const void* q, const void* r, const void* kpool, const void
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return PLX_ERR_ALIGN;
   const int S_max = max_pages * page_size;
-  const DecodePlan plan = plan_decode(B, Hq, Hkv, S_max, d, num_splits, false);
-  const int P = plan.P;
+  const DecodePlan plan = plan_decode(B, Hq, Hkv, S_max, d, num_splits, false, true);
   if (plan.ws_bytes > 0 && (!workspace || workspace_bytes < plan.ws_bytes)) return PLX_ERR_WORKSPACE;
   if (plan.ws_bytes > 0 && !aligned16(workspace)) return PLX_ERR_ALIGN;
   const int G = Hq / Hkv;
@@ -548,10 +568,10 @@ int plx_decode_paged(const void* q, const void* r, const void* kpool, const void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // (the partial-tile maps are for contiguous caches; page parts carry their own box)
   if (d == 128)
-    return r ? launch_decode<128, true, true>(km, vm, km, vm, p, P, st)
-             : launch_decode<128, false, true>(km, vm, km, vm, p, P, st);
-  return r ? launch_decode<64, true, true>(km, vm, km, vm, p, P, st)
-           : launch_decode<64, false, true>(km, vm, km, vm, p, P, st);
+    return r ? launch_decode<128, true, true>(km, vm, km, vm, nullptr, nullptr, p, plan, st)
+             : launch_decode<128, false, true>(km, vm, km, vm, nullptr, nullptr, p, plan, st);
+  return r ? launch_decode<64, true, true>(km, vm, km, vm, nullptr, nullptr, p, plan, st)
+           : launch_decode<64, false, true>(km, vm, km, vm, nullptr, nullptr, p, plan, st);
 }
 
 }  // extern "C"
@@ -674,12 +694,14 @@ int plx_bwd(const void* q, const void* k, const void* v, const void* r, const vo
 
 int plx_decode_num_splits(int B, int Hq, int Hkv, int S_max, int d) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128)) return decode_ctas(0, 4096);
-  return plan_decode(B, Hq, Hkv, S_max, d, 0, false).P;
+  return plan_decode(B, Hq, Hkv, S_max, d, 0, false, false).P;
 }
 
 size_t plx_decode_workspace_size(int B, int Hq, int Hkv, int S_max, int d, int num_splits) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128) || num_splits < 0) return 0;
-  return plan_decode(B, Hq, Hkv, S_max, d, num_splits, false).ws_bytes;
+  // the paged call's plan: it covers the contiguous call too (whose segment
+  // plan needs none), so one size serves both entry points
+  return plan_decode(B, Hq, Hkv, S_max, d, num_splits, false, true).ws_bytes;
 }
 
 }  // extern "C"
@@ -699,8 +721,7 @@ int decode_common(const void* q, const void* r, const void* kcache, const void* 
       (out && !aligned16(out)) || (rec_out && !aligned16(rec_out)) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return PLX_ERR_ALIGN;
-  const DecodePlan plan = plan_decode(B, Hq, Hkv, S_max, d, num_splits, rec_out != nullptr);
-  const int P = plan.P;
+  const DecodePlan plan = plan_decode(B, Hq, Hkv, S_max, d, num_splits, rec_out != nullptr, false);
   if (plan.ws_bytes > 0 && (!workspace || workspace_bytes < plan.ws_bytes)) return PLX_ERR_WORKSPACE;
   if (plan.ws_bytes > 0 && !aligned16(workspace)) return PLX_ERR_ALIGN;
   const int G = Hq / Hkv;
@@ -720,6 +741,11 @@ int decode_common(const void* q, const void* r, const void* kcache, const void* 
       make_map_3d(&kt, kcache, d, S_max, planes, plx::kDecTailRows) != PLX_OK ||
       make_map_3d(&vt, vcache, d, S_max, planes, plx::kDecTailRows) != PLX_OK)
     return PLX_ERR_CUDA;
+  // the segment plan streams kSegTileKeys-key stages
+  CUtensorMap k32, v32;
+  if (plan.seg && (make_map_3d(&k32, kcache, d, S_max, planes, plx::kSegTileKeys) != PLX_OK ||
+                   make_map_3d(&v32, vcache, d, S_max, planes, plx::kSegTileKeys) != PLX_OK))
+    return PLX_ERR_CUDA;
 
   plx::DecodeParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -737,10 +763,10 @@ int decode_common(const void* q, const void* r, const void* kcache, const void* 
   p.scale_log2 = scale * plx::kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 128)
-    return r ? launch_decode<128, true, false>(km, vm, kt, vt, p, P, st)
-             : launch_decode<128, false, false>(km, vm, kt, vt, p, P, st);
-  return r ? launch_decode<64, true, false>(km, vm, kt, vt, p, P, st)
-           : launch_decode<64, false, false>(km, vm, kt, vt, p, P, st);
+    return r ? launch_decode<128, true, false>(km, vm, kt, vt, &k32, &v32, p, plan, st)
+             : launch_decode<128, false, false>(km, vm, kt, vt, &k32, &v32, p, plan, st);
+  return r ? launch_decode<64, true, false>(km, vm, kt, vt, &k32, &v32, p, plan, st)
+           : launch_decode<64, false, false>(km, vm, kt, vt, &k32, &v32, p, plan, st);
 }
 
 }  // namespace
@@ -758,7 +784,7 @@ int plx_decode(const void* q, const void* r, const void* kcache, const void* vca
 size_t plx_decode_partial_size(int B, int Hq, int Hkv, int S_max, int d, int num_splits) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1 || Hq % Hkv || (d != 64 && d != 128) || num_splits < 0) return 0;
   return align256(static_cast<size_t>(B) * Hq * (2 * d + 4) * sizeof(float)) +
-         plan_decode(B, Hq, Hkv, S_max, d, num_splits, true).ws_bytes;
+         plan_decode(B, Hq, Hkv, S_max, d, num_splits, true, false).ws_bytes;
 }
 
 int plx_decode_partial(const void* q, const void* r, const void* kcache, const void* vcache,

@@ -123,13 +123,13 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 // Consumer: o += [P ; P*S] V over this warp's 16 keys of the stage's V tile
 // (transposed ldmatrix: b0 / b2 hold keys qc*2, qc*2+1 of the first eight,
 // b1 / b3 the same of the second eight, lower key in the low half).
-template <int D>
+template <int D, int TK = kDecTileKeys>
 __device__ __forceinline__ void value_mma(float (&o)[D / 8][4], const uint32_t (&pa)[4], uint32_t vbase, int vkey,
                                           int mi) {
 #pragma unroll
   for (int jp = 0; jp < D / 16; ++jp) {
     const int chunk = (2 * jp + (mi >> 1)) & 7;
-    const uint32_t addr = vbase + (jp >> 2) * (kDecTileKeys * 128) + sw128(vkey, chunk);
+    const uint32_t addr = vbase + (jp >> 2) * (TK * 128) + sw128(vkey, chunk);
     uint32_t b0, b1, b2, b3;
     ldsm_x4_t(addr, b0, b1, b2, b3);
     mma_bf16_16816(o[2 * jp], pa, b0, b1);
@@ -140,7 +140,7 @@ __device__ __forceinline__ void value_mma(float (&o)[D / 8][4], const uint32_t (
 // The same with the value rows of keys >= kend zeroed in the fragments, so
 // that a zero weight times whatever those rows hold (Inf, NaN) adds nothing.
 // key_lo = the key of this thread's first fragment element.
-template <int D>
+template <int D, int TK = kDecTileKeys>
 __device__ __forceinline__ void value_mma_masked(float (&o)[D / 8][4], const uint32_t (&pa)[4], uint32_t vbase,
                                                  int vkey, int mi, int key_lo, int kend) {
   const uint32_t m_lo = (key_lo < kend ? 0x0000ffffu : 0u) | (key_lo + 1 < kend ? 0xffff0000u : 0u);
@@ -148,7 +148,7 @@ __device__ __forceinline__ void value_mma_masked(float (&o)[D / 8][4], const uin
 #pragma unroll
   for (int jp = 0; jp < D / 16; ++jp) {
     const int chunk = (2 * jp + (mi >> 1)) & 7;
-    const uint32_t addr = vbase + (jp >> 2) * (kDecTileKeys * 128) + sw128(vkey, chunk);
+    const uint32_t addr = vbase + (jp >> 2) * (TK * 128) + sw128(vkey, chunk);
     uint32_t b0, b1, b2, b3;
     ldsm_x4_t(addr, b0, b1, b2, b3);
     b0 &= m_lo; b1 &= m_hi; b2 &= m_lo; b3 &= m_hi;
@@ -165,17 +165,17 @@ __device__ __forceinline__ void value_mma_masked(float (&o)[D / 8][4], const uin
 // live keys reach: the rows past them keep whatever the stage held before,
 // which the consumers mask out.  A part's 16 x 128-byte boxes start on 2 KB
 // boundaries, so the swizzle pattern of every row is the full tile's.
-template <int D>
+template <int D, int TK = kDecTileKeys>
 __device__ __forceinline__ void load_kv_tile(const CUtensorMap* kmap, const CUtensorMap* vmap, const CUtensorMap* kmap_t,
                                              const CUtensorMap* vmap_t, uint32_t kdst, uint32_t vdst, uint32_t bar,
                                              int key0, int live_from_key0, int kvrow, uint32_t extra) {
   constexpr int kHalves = D / 64;
-  if (live_from_key0 >= kDecTileKeys) {
-    mbar_arrive_expect_tx(bar, 2u * kDecTileKeys * D * 2 + extra);
+  if (live_from_key0 >= TK) {
+    mbar_arrive_expect_tx(bar, 2u * TK * D * 2 + extra);
 #pragma unroll
     for (int hf = 0; hf < kHalves; ++hf) {
-      tma_load_3d(kmap, kdst + hf * (kDecTileKeys * 128), bar, hf * 64, key0, kvrow);
-      tma_load_3d(vmap, vdst + hf * (kDecTileKeys * 128), bar, hf * 64, key0, kvrow);
+      tma_load_3d(kmap, kdst + hf * (TK * 128), bar, hf * 64, key0, kvrow);
+      tma_load_3d(vmap, vdst + hf * (TK * 128), bar, hf * 64, key0, kvrow);
     }
     return;
   }
@@ -185,8 +185,8 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* kmap, const CUte
     const uint32_t off = static_cast<uint32_t>(part * kDecTailRows * 128);
 #pragma unroll
     for (int hf = 0; hf < kHalves; ++hf) {
-      tma_load_3d(kmap_t, kdst + hf * (kDecTileKeys * 128) + off, bar, hf * 64, key0 + part * kDecTailRows, kvrow);
-      tma_load_3d(vmap_t, vdst + hf * (kDecTileKeys * 128) + off, bar, hf * 64, key0 + part * kDecTailRows, kvrow);
+      tma_load_3d(kmap_t, kdst + hf * (TK * 128) + off, bar, hf * 64, key0 + part * kDecTailRows, kvrow);
+      tma_load_3d(vmap_t, vdst + hf * (TK * 128) + off, bar, hf * 64, key0 + part * kDecTailRows, kvrow);
     }
   }
 }
@@ -887,6 +887,272 @@ plx_decode_chunk_kernel(const __grid_constant__ CUtensorMap kmap,
   // this CTA's results are written: the combine (launched as a programmatic
   // dependent) may be scheduled; it still waits for this grid to complete
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---- the segment plan: many short streams.  Each of kSegWarps warps of a
+// CTA owns whole segments (segments w, w + P*kSegWarps, ... of the list for
+// global warp w) and streams their keys through a ring of its own in
+// kSegTileKeys-key stages, its lane 0 issuing the TMA loads of the stage it
+// just finished (loads run on across the warp's segment boundaries).  A
+// warp holds a segment's whole online state, so a segment ends with quad
+// shuffles and direct stores: no cross-warp merge, no partial states, one
+// kernel.  The next segment's query and probe rows are fetched into
+// registers while the current one streams.
+constexpr int kSegTileKeys = 32;
+constexpr int kSegWarps = 4;
+constexpr int kSegThreads = kSegWarps * 32;
+
+template <int D>
+struct SegCfg {
+  static constexpr int kTileBytes = kSegTileKeys * D * 2;  // one of K or V
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kStages = D == 128 ? 3 : 6;          // per warp
+  static constexpr int kWarpBytes = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kSegWarps * kWarpBytes + 1024 + kSegWarps * kStages * 8;
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
+  static_assert(kSmemBytes <= 227 * 1024, "one CTA per SM");
+};
+
+// Position in one warp's segment stream: segment sg (of `total`), tile t of nt.
+struct SegWalk {
+  int sg, t, nt, live, total, stride;
+  __device__ __forceinline__ void set(const DecodeParams& p, int HN) {
+    nt = 0;
+    live = 0;
+    if (sg < total) {
+      live = dec_live(p, sg / HN);
+      nt = (live + kSegTileKeys - 1) / kSegTileKeys;
+    }
+  }
+  // first tile at or after segment sg (skipping segments with no live key); false past the end
+  __device__ __forceinline__ bool seek(const DecodeParams& p, int HN) {
+    for (;;) {
+      if (sg >= total) return false;
+      set(p, HN);
+      if (nt > 0) { t = 0; return true; }
+      sg += stride;
+    }
+  }
+  __device__ __forceinline__ bool next(const DecodeParams& p, int HN) {
+    if (++t < nt) return true;
+    sg += stride;
+    return seek(p, HN);
+  }
+};
+
+// q (rows 0..7) and rho (rows 8..15) of segment sg as the stacked A fragments
+// of the score MMA; rows past the group are zero
+template <int D, bool HAS_R>
+__device__ __forceinline__ void seg_load_qr(const DecodeParams& p, int sg, int HN, uint32_t (&af)[D / 16][4]) {
+  const int lane = threadIdx.x & 31, gr = lane >> 2, qc = lane & 3;
+  const int b = sg / HN, j = sg % HN;
+  const int g = j / p.n_hgroups, hg = j % p.n_hgroups;
+  const int nh = min(8, p.G - hg * 8);
+  const bool live = gr < nh;
+  const size_t row = static_cast<size_t>(b) * p.Hq + g * p.G + hg * 8 + (live ? gr : 0);
+  const uint32_t* qv = reinterpret_cast<const uint32_t*>(p.q + row * D);
+  const uint32_t* rv = HAS_R ? reinterpret_cast<const uint32_t*>(p.r + row * D) : nullptr;
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const int w0 = (ks * 16 + qc * 2) >> 1, w1 = (ks * 16 + 8 + qc * 2) >> 1;
+    af[ks][0] = live ? __ldg(qv + w0) : 0u;
+    af[ks][2] = live ? __ldg(qv + w1) : 0u;
+    af[ks][1] = (HAS_R && live) ? __ldg(rv + w0) : 0u;
+    af[ks][3] = (HAS_R && live) ? __ldg(rv + w1) : 0u;
+  }
+}
+
+template <int D, bool HAS_R>
+__global__ void __launch_bounds__(kSegThreads, 1)
+plx_decode_seg_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                      const __grid_constant__ CUtensorMap kmap_t, const __grid_constant__ CUtensorMap vmap_t,
+                      const DecodeParams p) {
+  using Cfg = SegCfg<D>;
+  constexpr int NS = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* ring = smem + warp * Cfg::kWarpBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSegWarps * Cfg::kWarpBytes) + warp * NS;
+  const int HN = p.Hkv * p.n_hgroups;
+
+  if (lane == 0) {
+    for (int s = 0; s < NS; ++s) mbar_init(smem_u32(&full[s]), 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&vmap);
+    tma_prefetch_desc(&kmap_t);
+    tma_prefetch_desc(&vmap_t);
+  }
+  __syncwarp();
+
+  const int stride = gridDim.x * kSegWarps;
+  const int first = blockIdx.x * kSegWarps + warp;
+  // lane 0's load cursor: the first NS tiles of this warp's stream
+  SegWalk ld{first, 0, 0, 0, p.B * HN, stride};
+  int issued = 0;
+  bool more = false;
+  auto issue = [&](int s) {
+    const uint32_t kdst = smem_u32(ring + s * Cfg::kStageBytes);
+    const int b = ld.sg / HN, g = (ld.sg % HN) / p.n_hgroups;
+    load_kv_tile<D, kSegTileKeys>(&kmap, &vmap, &kmap_t, &vmap_t, kdst, kdst + Cfg::kTileBytes,
+                                  smem_u32(&full[s]), ld.t * kSegTileKeys, ld.live - ld.t * kSegTileKeys,
+                                  b * p.Hkv + g, 0u);
+  };
+  if (lane == 0) {
+    more = ld.seek(p, HN);
+    while (more && issued < NS) {
+      issue(issued % NS);
+      ++issued;
+      more = ld.next(p, HN);
+    }
+  }
+
+  const int gr = lane >> 2, qc = lane & 3;
+  const int mi = lane >> 3, ri = lane & 7;
+  bool ok = true;
+  int k = 0;  // tiles consumed
+  uint32_t afn[D / 16][4];
+  if (first < p.B * HN) seg_load_qr<D, HAS_R>(p, first, HN, afn);
+  for (int sg = first; sg < p.B * HN && ok; sg += stride) {
+    uint32_t afrag[D / 16][4];
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) afrag[ks][e] = afn[ks][e];
+    if (sg + stride < p.B * HN) seg_load_qr<D, HAS_R>(p, sg + stride, HN, afn);  // in flight while this streams
+    const int b = sg / HN, j = sg % HN;
+    const int g = j / p.n_hgroups, hg = j % p.n_hgroups;
+    const int nh = min(8, p.G - hg * 8);
+    const size_t row0 = static_cast<size_t>(b) * p.Hq + g * p.G + hg * 8;
+    const int kend = dec_live(p, b);
+    const int nt = (kend + kSegTileKeys - 1) / kSegTileKeys;
+    if (nt == 0) {
+      // no live key: out = 0, lse = -inf (or an empty record)
+      if (p.rec_out) {
+        for (int idx = lane; idx < nh * (2 * D + 4); idx += 32)
+          p.rec_out[row0 * (2 * D + 4) + idx] = (idx % (2 * D + 4)) == 0 ? -INFINITY : 0.f;
+      } else {
+        for (int idx = lane; idx < nh * D; idx += 32) p.out[row0 * D + idx] = __float2bfloat16(0.f);
+        if (p.lse && lane < nh) p.lse[row0 + lane] = -INFINITY;
+      }
+      continue;
+    }
+
+    float o[D / 8][4];
+#pragma unroll
+    for (int jj = 0; jj < D / 8; ++jj) o[jj][0] = o[jj][1] = o[jj][2] = o[jj][3] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f, c_run = 0.f;
+    for (int t = 0; t < nt; ++t, ++k) {
+      const int s = k % NS;
+      // a wait that runs out stops this warp (its results are then undefined;
+      // the error word is set); no other warp waits for it
+      const bool landed = mbar_wait(smem_u32(&full[s]), (k / NS) & 1, kErrDecodeFull);
+      if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }
+      const uint32_t kbase = smem_u32(ring + s * Cfg::kStageBytes);
+      const uint32_t vbase = kbase + Cfg::kTileBytes;
+#pragma unroll
+      for (int s16 = 0; s16 < kSegTileKeys / 16; ++s16) {
+        const int kkey = s16 * 16 + (mi >> 1) * 8 + ri;
+        const int vkey = s16 * 16 + (mi & 1) * 8 + ri;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int chunk = (2 * ks + (mi & 1)) & 7;
+          const uint32_t addr = kbase + (ks >> 2) * (kSegTileKeys * 128) + sw128(kkey, chunk);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(addr, b0, b1, b2, b3);
+          mma_bf16_16816(acc[0], afrag[ks], b0, b1);
+          mma_bf16_16816(acc[1], afrag[ks], b2, b3);
+        }
+        const int key_lo = t * kSegTileKeys + s16 * 16 + qc * 2;  // key of acc[0][0]
+        // keys past the sequence take no part, whatever their rows hold
+        float x[4], sv[4];
+#pragma unroll
+        for (int nn = 0; nn < 2; ++nn)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const bool in = key_lo + nn * 8 + e < kend;
+            x[nn * 2 + e] = in ? acc[nn][e] * p.scale_log2 : -INFINITY;
+            sv[nn * 2 + e] = in ? acc[nn][2 + e] : 0.f;
+          }
+        float tmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+        const float m_new = fmaxf(m_run, tmax);
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        const float alpha = ex2(m_run - m_use);
+        float pr[4], ps[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pr[e] = ex2(x[e] - m_use);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ps[e] = HAS_R ? pr[e] * sv[e] : 0.f;
+        uint32_t pa[4];
+        pa[0] = pack_bf16(pr[0], pr[1]);
+        pa[1] = pack_bf16(ps[0], ps[1]);
+        pa[2] = pack_bf16(pr[2], pr[3]);
+        pa[3] = pack_bf16(ps[2], ps[3]);
+        const float psum = (pr[0] + pr[1]) + (pr[2] + pr[3]);
+        const float csum = (bf16_lo(pa[1]) + bf16_hi(pa[1])) + (bf16_lo(pa[3]) + bf16_hi(pa[3]));
+        l_run = l_run * alpha + psum;
+        c_run = c_run * alpha + csum;
+        m_run = m_new;
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int jj = 0; jj < D / 8; ++jj) {
+            o[jj][0] *= alpha; o[jj][1] *= alpha; o[jj][2] *= alpha; o[jj][3] *= alpha;
+          }
+        }
+        if (t * kSegTileKeys + s16 * 16 + 16 <= kend)  // warp-uniform: all 16 keys live
+          value_mma<D, kSegTileKeys>(o, pa, vbase, vkey, mi);
+        else
+          value_mma_masked<D, kSegTileKeys>(o, pa, vbase, vkey, mi, key_lo, kend);
+      }
+      // stage s is read: lane 0 refills it with the tile NS ahead in this warp's stream
+      __syncwarp();
+      if (lane == 0 && more) {
+        issue(s);
+        ++issued;
+        more = ld.next(p, HN);
+      }
+    }
+    if (!ok) break;
+
+    // ---- this segment is finished in the warp: the row's l and c over the quad
+    float l4 = l_run, c4 = c_run;
+    l4 += __shfl_xor_sync(0xffffffffu, l4, 1);
+    l4 += __shfl_xor_sync(0xffffffffu, l4, 2);
+    c4 += __shfl_xor_sync(0xffffffffu, c4, 1);
+    c4 += __shfl_xor_sync(0xffffffffu, c4, 2);
+    if (gr < nh) {
+      const size_t row = row0 + gr;
+      if (p.rec_out) {
+        float* rec = p.rec_out + row * (2 * D + 4);
+        if (qc == 0) { rec[0] = m_run; rec[1] = l4; rec[2] = c4; rec[3] = 0.f; }
+#pragma unroll
+        for (int jj = 0; jj < D / 8; ++jj) {
+          const int col = jj * 8 + qc * 2;
+          *reinterpret_cast<float2*>(rec + 4 + col) = make_float2(o[jj][0], o[jj][1]);
+          *reinterpret_cast<float2*>(rec + 4 + D + col) = make_float2(o[jj][2], o[jj][3]);
+        }
+      } else {
+        const float inv = l4 > 0.f ? 1.f / l4 : 0.f;
+        const float cl = c4 * inv;
+#pragma unroll
+        for (int jj = 0; jj < D / 8; ++jj) {
+          const float a0 = o[jj][0] * inv, a1 = o[jj][1] * inv;
+          const float r0 = a0 - (o[jj][2] * inv - cl * a0);
+          const float r1 = a1 - (o[jj][3] * inv - cl * a1);
+          *reinterpret_cast<__nv_bfloat162*>(p.out + row * D + jj * 8 + qc * 2) = __floats2bfloat162_rn(r0, r1);
+        }
+        if (qc == 0 && p.lse) p.lse[row] = l4 > 0.f ? (m_run + __log2f(l4)) * kLn2 : -INFINITY;
+      }
+    }
+  }
+  // every load issued must land before this CTA's shared memory goes away
+  if (lane == 0)
+    for (int j = max(k, issued - NS); j < issued; ++j)
+      mbar_wait(smem_u32(&full[j % NS]), (j / NS) & 1, kErrDecodeDrain);
 }
 
 // Finishes what the split kernel left: the segments cut by a partition
