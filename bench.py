@@ -1126,8 +1126,8 @@ def run_sweep(args):
 
 def run_profile_small(args):
     """--profile-small: one call of each small case the ncu summaries in
-    profiles/ capture (decode in both plans, the projection in both forms),
-    then exit; inputs larger than L2 but a few GB at most."""
+    profiles/ capture (decode in its three plans, the projection in both
+    forms), then exit; inputs larger than L2 but a few GB at most."""
     import torch
     from parameterized_local_linear_plx_b200 import build, inputs
     build.build()
@@ -1139,6 +1139,10 @@ def run_profile_small(args):
     del kc, vc
     # decode, chunked plan: B=64, context 4096 (1.07 GB of KV)
     q, kc, vc, r, sl = inputs.decode_inputs(64, 16, 8, 4096, 128, seed=0, device=dev)
+    plx.plx_decode(q, kc, vc, sl, r)
+    del kc, vc
+    # decode, segment plan: B=1024, context 128, lengths uniform in [64, 128] (537 MB of KV allocated)
+    q, kc, vc, r, sl = inputs.decode_inputs(1024, 16, 8, 128, 128, seed=0, seqlens="ragged", device=dev)
     plx.plx_decode(q, kc, vc, sl, r)
     del kc, vc
     # projection, prefill form: 2 x 4096 tokens, d_model 1024, W [6144, 1024]
