@@ -889,31 +889,36 @@ plx_decode_chunk_kernel(const __grid_constant__ CUtensorMap kmap,
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// ---- the segment plan: many short streams.  Each of kSegWarps warps of a
-// CTA owns whole segments (segments w, w + P*kSegWarps, ... of the list for
-// global warp w) and streams their keys through a ring of its own in
-// kSegTileKeys-key stages, its lane 0 issuing the TMA loads of the stage it
-// just finished (loads run on across the warp's segment boundaries).  A
-// warp holds a segment's whole online state, so a segment ends with quad
-// shuffles and direct stores: no cross-warp merge, no partial states, one
-// kernel.  The next segment's query and probe rows are fetched into
-// registers while the current one streams.
-constexpr int kSegTileKeys = 32;
-constexpr int kSegWarps = 4;
-constexpr int kSegThreads = kSegWarps * 32;
-
-template <int D>
+// ---- the segment plan: many short streams.  Each of the W warps of a CTA
+// owns whole segments and streams their keys through a ring of its own in
+// TK-key stages, its lane 0 issuing the TMA loads of the stage it just
+// finished (loads run on across the warp's segment boundaries).  Segments
+// are dealt round the CTAs first (segment k goes to CTA k mod P, warp
+// (k div P) mod W), so a batch with few segments still spreads over the
+// SMs.  A warp holds a segment's whole online state, so a segment ends with
+// quad shuffles and direct stores: no cross-warp merge, no partial states,
+// one kernel.  The next segment's query and probe rows are fetched into
+// registers while the current one streams.  Two shapes share the code: 4
+// warps with 32-key stages (more bytes in flight per warp, for fewer
+// segments) and 8 warps with 16-key stages (two warps per sub-partition to
+// hide each other's latencies, for many); both keep 192 KB of stages per SM.
+template <int D, int W, int TK>
 struct SegCfg {
-  static constexpr int kTileBytes = kSegTileKeys * D * 2;  // one of K or V
+  static constexpr int kThreads = W * 32;
+  static constexpr int kTileBytes = TK * D * 2;             // one of K or V
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = D == 128 ? 3 : 6;          // per warp
+  static constexpr int kStages = (D == 128 ? 3 : 6) * 32 / (TK * (W / 4));  // per warp
   static constexpr int kWarpBytes = kStages * kStageBytes;
-  static constexpr int kSmemBytes = kSegWarps * kWarpBytes + 1024 + kSegWarps * kStages * 8;
+  static constexpr int kSmemBytes = W * kWarpBytes + 1024 + W * kStages * 8;
+  static_assert(kStages >= 2, "a ring of at least two stages per warp");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kSmemBytes <= 227 * 1024, "one CTA per SM");
 };
+constexpr int kSegFewWarps = 4, kSegFewKeys = 32;   // shape for fewer segments
+constexpr int kSegManyWarps = 8, kSegManyKeys = 16; // shape for many segments
 
 // Position in one warp's segment stream: segment sg (of `total`), tile t of nt.
+template <int TK>
 struct SegWalk {
   int sg, t, nt, live, total, stride;
   __device__ __forceinline__ void set(const DecodeParams& p, int HN) {
@@ -921,7 +926,7 @@ struct SegWalk {
     live = 0;
     if (sg < total) {
       live = dec_live(p, sg / HN);
-      nt = (live + kSegTileKeys - 1) / kSegTileKeys;
+      nt = (live + TK - 1) / TK;
     }
   }
   // first tile at or after segment sg (skipping segments with no live key); false past the end
@@ -962,18 +967,18 @@ __device__ __forceinline__ void seg_load_qr(const DecodeParams& p, int sg, int H
   }
 }
 
-template <int D, bool HAS_R>
-__global__ void __launch_bounds__(kSegThreads, 1)
+template <int D, bool HAS_R, int W, int TK>
+__global__ void __launch_bounds__(W * 32, 1)
 plx_decode_seg_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                       const __grid_constant__ CUtensorMap kmap_t, const __grid_constant__ CUtensorMap vmap_t,
                       const DecodeParams p) {
-  using Cfg = SegCfg<D>;
+  using Cfg = SegCfg<D, W, TK>;
   constexpr int NS = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* ring = smem + warp * Cfg::kWarpBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSegWarps * Cfg::kWarpBytes) + warp * NS;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + W * Cfg::kWarpBytes) + warp * NS;
   const int HN = p.Hkv * p.n_hgroups;
 
   if (lane == 0) {
@@ -986,18 +991,17 @@ plx_decode_seg_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
   }
   __syncwarp();
 
-  const int stride = gridDim.x * kSegWarps;
-  const int first = blockIdx.x * kSegWarps + warp;
+  const int stride = gridDim.x * W;
+  const int first = warp * gridDim.x + blockIdx.x;
   // lane 0's load cursor: the first NS tiles of this warp's stream
-  SegWalk ld{first, 0, 0, 0, p.B * HN, stride};
+  SegWalk<TK> ld{first, 0, 0, 0, p.B * HN, stride};
   int issued = 0;
   bool more = false;
   auto issue = [&](int s) {
     const uint32_t kdst = smem_u32(ring + s * Cfg::kStageBytes);
     const int b = ld.sg / HN, g = (ld.sg % HN) / p.n_hgroups;
-    load_kv_tile<D, kSegTileKeys>(&kmap, &vmap, &kmap_t, &vmap_t, kdst, kdst + Cfg::kTileBytes,
-                                  smem_u32(&full[s]), ld.t * kSegTileKeys, ld.live - ld.t * kSegTileKeys,
-                                  b * p.Hkv + g, 0u);
+    load_kv_tile<D, TK>(&kmap, &vmap, &kmap_t, &vmap_t, kdst, kdst + Cfg::kTileBytes, smem_u32(&full[s]),
+                        ld.t * TK, ld.live - ld.t * TK, b * p.Hkv + g, 0u);
   };
   if (lane == 0) {
     more = ld.seek(p, HN);
@@ -1026,7 +1030,7 @@ plx_decode_seg_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     const int nh = min(8, p.G - hg * 8);
     const size_t row0 = static_cast<size_t>(b) * p.Hq + g * p.G + hg * 8;
     const int kend = dec_live(p, b);
-    const int nt = (kend + kSegTileKeys - 1) / kSegTileKeys;
+    const int nt = (kend + TK - 1) / TK;
     if (nt == 0) {
       // no live key: out = 0, lse = -inf (or an empty record)
       if (p.rec_out) {
@@ -1052,20 +1056,20 @@ plx_decode_seg_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       const uint32_t kbase = smem_u32(ring + s * Cfg::kStageBytes);
       const uint32_t vbase = kbase + Cfg::kTileBytes;
 #pragma unroll
-      for (int s16 = 0; s16 < kSegTileKeys / 16; ++s16) {
+      for (int s16 = 0; s16 < TK / 16; ++s16) {
         const int kkey = s16 * 16 + (mi >> 1) * 8 + ri;
         const int vkey = s16 * 16 + (mi & 1) * 8 + ri;
         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const int chunk = (2 * ks + (mi & 1)) & 7;
-          const uint32_t addr = kbase + (ks >> 2) * (kSegTileKeys * 128) + sw128(kkey, chunk);
+          const uint32_t addr = kbase + (ks >> 2) * (TK * 128) + sw128(kkey, chunk);
           uint32_t b0, b1, b2, b3;
           ldsm_x4(addr, b0, b1, b2, b3);
           mma_bf16_16816(acc[0], afrag[ks], b0, b1);
           mma_bf16_16816(acc[1], afrag[ks], b2, b3);
         }
-        const int key_lo = t * kSegTileKeys + s16 * 16 + qc * 2;  // key of acc[0][0]
+        const int key_lo = t * TK + s16 * 16 + qc * 2;  // key of acc[0][0]
         // keys past the sequence take no part, whatever their rows hold
         float x[4], sv[4];
 #pragma unroll
@@ -1103,10 +1107,10 @@ plx_decode_seg_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
             o[jj][0] *= alpha; o[jj][1] *= alpha; o[jj][2] *= alpha; o[jj][3] *= alpha;
           }
         }
-        if (t * kSegTileKeys + s16 * 16 + 16 <= kend)  // warp-uniform: all 16 keys live
-          value_mma<D, kSegTileKeys>(o, pa, vbase, vkey, mi);
+        if (t * TK + s16 * 16 + 16 <= kend)  // warp-uniform: all 16 keys live
+          value_mma<D, TK>(o, pa, vbase, vkey, mi);
         else
-          value_mma_masked<D, kSegTileKeys>(o, pa, vbase, vkey, mi, key_lo, kend);
+          value_mma_masked<D, TK>(o, pa, vbase, vkey, mi, key_lo, kend);
       }
       // stage s is read: lane 0 refills it with the tile NS ahead in this warp's stream
       __syncwarp();

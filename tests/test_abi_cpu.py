@@ -131,11 +131,12 @@ def test_split_planning(plx):
         assert plx.plx_decode_workspace_size(B, 16, 8, S, 128, 0) == (up(B * 16 * splits * 260 * 4) if splits > 1 else 0)
     assert plx.plx_decode_num_splits(2048, 16, 8, 16384, 128) == 2048 * 8  # one chunk per segment: no workspace
     # short segments (at most 256 keys): the segment plan, one warp per whole
-    # segment, four warps per CTA, at most one CTA per SM, no workspace of its
-    # own; the workspace size covers the paged call, which keeps the balanced
-    # plan (two partitions per SM for short segments)
+    # segment, segments dealt round the CTAs first, at most one CTA per SM and
+    # no more CTAs than segments, no workspace of its own; the workspace size
+    # covers the paged call, which keeps the balanced plan (two partitions
+    # per SM for short segments)
     assert plx.plx_decode_num_splits(2048, 16, 8, 256, 128) == n
-    assert plx.plx_decode_num_splits(1, 16, 8, 128, 128) == 2  # 8 segments: 2 CTAs
+    assert plx.plx_decode_num_splits(1, 16, 8, 128, 128) == 8  # 8 segments: 8 CTAs
     assert plx.plx_decode_workspace_size(1, 16, 8, 128, 128, 0) == up(2 * (2 * n) * 2 * 260 * 4)
     # bad shapes: size 0
     assert plx.plx_decode_workspace_size(1, 3, 2, 128, 128, 2) == 0

@@ -92,13 +92,15 @@ def test_decode_partitions_cross_sequences_and_head_groups(plx, splits):
     assert_close(o, ro, l, rl, f"partitions={splits} d=128")
 
 
-@pytest.mark.parametrize("B,S,d", [(40, 1000, 128), (300, 200, 128), (48, 700, 64), (700, 256, 64)])
+@pytest.mark.parametrize("B,S,d", [(40, 1000, 128), (300, 200, 128), (48, 700, 64), (700, 256, 64), (100, 128, 128),
+                                   (160, 96, 64)])
 def test_decode_many_segments(plx, B, S, d):
     """Batches with 128 (b, kv head) segments or more: of more than 256 keys
     they take the chunked plan (a CTA per chunk of a segment, chunk records
     merged per row), shorter ones the segment plan (one warp per whole
-    segment, several segments per warp); ragged lengths with empty sequences
-    among them; sampled batch entries."""
+    segment, several segments per warp; 8 warps with 16-key stages for more
+    than 4 x SMs segments of at most 128 keys); ragged lengths with empty
+    sequences among them; sampled batch entries."""
     q, kc, vc, r, _ = inputs.decode_inputs(B, 16, 8, S, d, seed=60 + B, device="cuda")
     g = torch.Generator(device="cuda").manual_seed(61)
     sl = torch.randint(0, S + 1, (B,), generator=g, device="cuda", dtype=torch.int32)
@@ -220,6 +222,7 @@ def _poison_tail(cache, seqlens):
     (3, 4, 2, 200, 64, 3),       # explicit partitions
     (5, 8, 1, 130, 128, 1),      # one partition over every segment
     (40, 16, 8, 1000, 128, 0),   # chunked plan (320 segments of > 256 keys)
+    (100, 16, 8, 128, 128, 0),   # segment plan, 8 warps per CTA and 16-key stages (800 segments)
 ])
 def test_decode_ignores_cache_rows_past_the_sequence(plx, B, Hq, Hkv, S, d, splits):
     """Keys past the sequence take no part whatever their rows hold: NaN and
