@@ -47,6 +47,27 @@ def test_slices_match_decode_and_oracle(plx, ranks, d):
     assert_close(out, ro, lse, rl, f"cp ranks={ranks} d={d}")
 
 
+def test_slices_of_many_short_segments(plx):
+    """Slices of 128 keys over 8 ranks at B=100 (800 (b, kv head) segments per
+    slice): each slice's records come from the segment plan's 8-warp shape,
+    with the key offset of its rank; against the plain decode and sampled
+    rows of the oracle."""
+    B, Hq, Hkv, S, d = 100, 16, 8, 1024, 128
+    q, kc, vc, r, _ = inputs.decode_inputs(B, Hq, Hkv, S, d, seed=31, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(32)
+    sl = torch.randint(0, S + 1, (B,), generator=g, device="cuda", dtype=torch.int32)
+    sl[0], sl[1], sl[2] = 0, 1, S
+    out, lse = emulate(plx, q, kc, vc, sl, r, 8)
+    ref_o, ref_l = plx.plx_decode(q, kc, vc, sl, r)
+    step = ref_o.float().abs().clamp_min(1.0) * 2.0 ** -7
+    assert bool(((out.float() - ref_o.float()).abs() <= step).all())
+    live = sl > 0
+    assert (lse[live] - ref_l[live]).abs().max().item() <= 1e-4
+    pick = [0, 1, 2, 37, 99]
+    ro, rl = oracle.decode_effective(q[pick].cpu(), r[pick].cpu(), kc[pick].cpu(), vc[pick].cpu(), sl[pick].cpu())
+    assert_close(out[pick], ro, lse[pick], rl, "cp slices of many short segments")
+
+
 def test_split_counts_empty_rows_and_rho_none(plx):
     B, Hq, Hkv, S, d = 3, 4, 2, 512, 128
     q, kc, vc, r, _ = inputs.decode_inputs(B, Hq, Hkv, S, d, seed=9, device="cuda")
