@@ -1177,7 +1177,7 @@ def main():
     ap.add_argument("--no-decode-configs", action="store_true", help="leave the decode configurations out of the "
                     "bench line")
     ap.add_argument("--profile-small", action="store_true", help="one call of each small case the ncu summaries "
-                    "capture (decode in both plans, the projection in both forms), then exit")
+                    "capture (decode in its three plans, the projection in both forms), then exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
